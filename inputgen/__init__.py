@@ -1,0 +1,183 @@
+"""Seeded synthetic inputs shared by the oracle side and the CUDA side.
+
+This module holds no attention arithmetic. It only draws iid N(0,1) values
+with a fixed seed, rounds them to bf16 with round-to-nearest-even, and knows
+the shapes of the five workloads. Both the fp64 oracle and the GPU path read
+the *same* bf16 bit patterns from here, so any difference between them comes
+from the attention computation alone.
+
+Workloads (sizes, dtypes, masks) follow the problem statement of the build;
+the values are synthetic because the pages measure on no dataset.
+
+Recipe
+------
+* workload ``k`` (0..4) draws from ``numpy.random.default_rng(20260 + k)``;
+* draws are float32 standard normals, taken in the order Q, K, V, dO;
+* the split-KV decode workload first draws its per-sequence cache lengths
+  with ``rng.integers(16384, 32769, size=B)``, then q, then the K cache one
+  sequence at a time (only the first ``seqlen[b]`` positions), then the V
+  cache the same way; cache positions at or past ``seqlen[b]`` are filled
+  with NaN so that a kernel that reads past the logical end poisons its own
+  result;
+* bf16 rounding is round-to-nearest-even on the fp32 bit pattern.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+__all__ = [
+    "Workload",
+    "WORKLOADS",
+    "bf16_round_bits",
+    "bf16_bits_to_f32",
+    "standard_normal_bf16",
+    "make_attention_inputs",
+    "make_decode_inputs",
+    "make_small_inputs",
+    "sample_row_blocks",
+]
+
+SEED_BASE = 20260
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One workload: shapes, dtype and masks, named by what it is."""
+
+    name: str
+    index: int
+    B: int
+    H: int
+    N: int  # sequence length (prefill) or cache capacity Lmax (decode)
+    d: int
+    dtype: str  # "f32" or "bf16"
+    causal: tuple = (False,)
+    kind: str = "fwd"  # "fwd", "bwd" or "decode"
+    seqlen_range: tuple | None = None
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def seed(self) -> int:
+        return SEED_BASE + self.index
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+
+WORKLOADS = {
+    "tiny_f32": Workload("tiny_f32", 0, B=1, H=1, N=128, d=64, dtype="f32",
+                         causal=(False, True)),
+    "prefill": Workload("prefill", 1, B=4, H=16, N=2048, d=128, dtype="bf16",
+                        causal=(False, True)),
+    "long_causal": Workload("long_causal", 2, B=1, H=32, N=16384, d=128,
+                            dtype="bf16", causal=(True,)),
+    "backward": Workload("backward", 3, B=2, H=16, N=4096, d=128, dtype="bf16",
+                         causal=(True,), kind="bwd"),
+    "decode": Workload("decode", 4, B=8, H=32, N=32768, d=128, dtype="bf16",
+                       kind="decode", seqlen_range=(16384, 32768)),
+}
+
+
+def bf16_round_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (round to nearest, ties to even).
+
+    Returns the 16-bit patterns as uint16. Inputs here are finite normals,
+    so no NaN/Inf special-casing is needed; NaN payloads are preserved
+    anyway by the quiet-bit OR below.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    rounded = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
+    out = rounded.astype(np.uint16)
+    nan = np.isnan(x)
+    if nan.any():
+        out[nan] = ((u[nan] >> np.uint32(16)) | np.uint32(0x40)).astype(np.uint16)
+    return out
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact float32 value of each bf16 bit pattern."""
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def standard_normal_bf16(rng: np.random.Generator, shape) -> np.ndarray:
+    """Draw float32 N(0,1) values and return their bf16 bit patterns."""
+    return bf16_round_bits(rng.standard_normal(shape, dtype=np.float32))
+
+
+def make_attention_inputs(w: Workload, with_grad: bool = False):
+    """Q, K, V (and dO) for a prefill / backward workload.
+
+    Returns a dict. For bf16 workloads the arrays are uint16 bit patterns
+    of shape [B, H, N, d]; for the fp32 workload they are float32.
+    """
+    rng = np.random.default_rng(w.seed)
+    shape = (w.B, w.H, w.N, w.d)
+    names = ["q", "k", "v"] + (["do"] if with_grad else [])
+    out = {}
+    for n in names:
+        if w.dtype == "f32":
+            out[n] = rng.standard_normal(shape, dtype=np.float32)
+        else:
+            out[n] = standard_normal_bf16(rng, shape)
+    return out
+
+
+def make_decode_inputs(w: Workload, seqlens=None):
+    """q [B,H,d], K/V caches [B,H,Lmax,d] (bf16 bits) and seqlens int32 [B].
+
+    Cache entries at or past ``seqlens[b]`` hold bf16 NaN (0x7FC0).
+    ``seqlens`` may be given to override the drawn lengths (edge cases);
+    the draw still happens so the stream of values is unchanged.
+    """
+    rng = np.random.default_rng(w.seed)
+    lo, hi = w.seqlen_range
+    drawn = rng.integers(lo, hi + 1, size=w.B).astype(np.int32)
+    lens = drawn if seqlens is None else np.asarray(seqlens, dtype=np.int32)
+    q = standard_normal_bf16(rng, (w.B, w.H, w.d))
+    kc = np.full((w.B, w.H, w.N, w.d), 0x7FC0, dtype=np.uint16)
+    vc = np.full((w.B, w.H, w.N, w.d), 0x7FC0, dtype=np.uint16)
+    for b in range(w.B):
+        kc[b, :, : lens[b]] = standard_normal_bf16(rng, (w.H, int(lens[b]), w.d))
+    for b in range(w.B):
+        vc[b, :, : lens[b]] = standard_normal_bf16(rng, (w.H, int(lens[b]), w.d))
+    return {"q": q, "kcache": kc, "vcache": vc, "seqlens": lens}
+
+
+def make_small_inputs(seed: int, B: int, H: int, N: int, d: int,
+                      with_grad: bool = False, dtype: str = "bf16"):
+    """Seeded inputs of any shape, for the small parity cases."""
+    rng = np.random.default_rng(seed)
+    shape = (B, H, N, d)
+    names = ["q", "k", "v"] + (["do"] if with_grad else [])
+    out = {}
+    for n in names:
+        if dtype == "f32":
+            out[n] = rng.standard_normal(shape, dtype=np.float32)
+        else:
+            out[n] = standard_normal_bf16(rng, shape)
+    return out
+
+
+def sample_row_blocks(w: Workload, count: int = 64, block: int = 128,
+                      seed_offset: int = 100):
+    """Seeded sample of (batch, head, row-block) triples for large workloads.
+
+    Draws from ``default_rng(seed + seed_offset)``; returns a sorted list of
+    distinct triples ``(b, h, blk)`` where rows ``blk*block .. +block`` form
+    the sampled query block.
+    """
+    rng = np.random.default_rng(w.seed + seed_offset)
+    nblk = (w.N + block - 1) // block
+    total = w.B * w.H * nblk
+    picks = rng.choice(total, size=min(count, total), replace=False)
+    out = []
+    for p in sorted(int(x) for x in picks):
+        b, rem = divmod(p, w.H * nblk)
+        h, blk = divmod(rem, nblk)
+        out.append((b, h, blk))
+    return out

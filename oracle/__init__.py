@@ -1,0 +1,17 @@
+"""fp64 CPU oracle (test infrastructure; never on the product path).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. It shares no code with the CUDA
+library in ``exact_attention_130_b200``.
+"""
+from .attention import (  # noqa: F401
+    attention_bwd,
+    attention_fwd,
+    attention_fwd_rows,
+    decode,
+    decode_split,
+    merge_partials,
+    online_attention_fwd,
+    scores,
+    softmax_rows,
+)

@@ -1,0 +1,48 @@
+"""The seeded input generator: bf16 rounding and reproducibility."""
+import numpy as np
+import torch
+
+import inputgen
+
+
+def test_bf16_rounding_matches_library():
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.standard_normal(100000).astype(np.float32),
+                        np.array([1.00390625, 1.01171875, -2.5e-39, 3.0e38,
+                                  0.0, -0.0], dtype=np.float32)])
+    ours = inputgen.bf16_round_bits(x)
+    lib = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy()
+    assert np.array_equal(ours.view(np.int16), lib)
+
+
+def test_bits_roundtrip():
+    bits = np.arange(0, 0x7F80, 37, dtype=np.uint16)
+    f = inputgen.bf16_bits_to_f32(bits)
+    assert np.array_equal(inputgen.bf16_round_bits(f), bits)
+
+
+def test_workloads_are_reproducible():
+    w = inputgen.WORKLOADS["tiny_f32"]
+    a = inputgen.make_attention_inputs(w)
+    b = inputgen.make_attention_inputs(w)
+    for n in ("q", "k", "v"):
+        assert a[n].dtype == np.float32 and a[n].shape == (1, 1, 128, 64)
+        assert np.array_equal(a[n], b[n])
+
+
+def test_decode_padding_is_nan():
+    w = inputgen.Workload("t", 4, B=3, H=2, N=40, d=16, dtype="bf16",
+                          kind="decode", seqlen_range=(5, 40))
+    x = inputgen.make_decode_inputs(w)
+    for b, n in enumerate(x["seqlens"]):
+        kc = inputgen.bf16_bits_to_f32(x["kcache"][b])
+        assert np.all(np.isfinite(kc[:, :n]))
+        assert np.all(np.isnan(kc[:, n:]))
+
+
+def test_row_block_sample():
+    w = inputgen.WORKLOADS["long_causal"]
+    s = inputgen.sample_row_blocks(w, 64)
+    assert len(s) == 64 and len(set(s)) == 64
+    assert all(0 <= h < 32 and 0 <= blk < 128 and b == 0 for b, h, blk in s)
+    assert s == inputgen.sample_row_blocks(w, 64)

@@ -1,0 +1,242 @@
+"""Python binding of libfa_sm100.so (exact attention for B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/fa.h. PyTorch supplies device
+memory and the current stream. There is no CPU fallback: if the library is
+missing, every call raises.
+
+Functions carry the C names:
+    fa_fwd, fa_fwd_f32, fa_bwd, fa_bwd_workspace_size,
+    fa_decode_splitkv, fa_decode_workspace_size,
+    fa_device_status, fa_set_wait_limit, fa_debug_skip_load
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+__all__ = [
+    "FAError", "library_path", "load_library", "exported_symbols",
+    "fa_fwd", "fa_fwd_f32", "fa_bwd", "fa_bwd_workspace_size",
+    "fa_decode_splitkv", "fa_decode_workspace_size", "fa_device_status",
+    "fa_set_wait_limit", "fa_debug_skip_load", "fa_abi_version",
+    "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+STATUS = {
+    0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
+    3: "FA_ERR_ALIGNMENT", 4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA",
+    6: "FA_ERR_TIMEOUT",
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libfa_sm100.so")
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_S = ctypes.c_size_t
+
+_SIGNATURES = {
+    "fa_status_string": (ctypes.c_char_p, [_I]),
+    "fa_last_error": (ctypes.c_char_p, []),
+    "fa_abi_version": (_I, []),
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
+    "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I,
+                    _P, _S, _P]),
+    "fa_decode_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I,
+                               _P, _S, _P]),
+    "fa_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
+    "fa_set_wait_limit": (None, [ctypes.c_ulonglong]),
+    "fa_debug_skip_load": (None, [_I]),
+}
+
+
+def load_library():
+    """Load libfa_sm100.so; raise if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with "
+                "`python -m exact_attention_130_b200.build` (there is no CPU fallback)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def exported_symbols():
+    """Names of the entry points include/fa.h declares."""
+    hdr = open(os.path.join(os.path.dirname(_HERE), "include", "fa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(fa_\w+)\s*\(", hdr, re.M)))
+
+
+def _check(status: int):
+    if status != 0:
+        lib = load_library()
+        raise FAError(status, lib.fa_last_error().decode(errors="replace"))
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fa_abi_version() -> int:
+    return load_library().fa_abi_version()
+
+
+def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None,
+           lse=None, stream=None):
+    """O, LSE = attention(q, k, v); bf16 [B, H, N, d] in and out."""
+    import torch
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                      scale, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None,
+               o=None, lse=None, stream=None):
+    """The fp32 forward: fp32 [B, H, N, d] in and out."""
+    import torch
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.float32, n)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check(lib.fa_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N,
+                          d, scale, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().fa_bwd_workspace_size(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
+           dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of sum(O * dO); bf16 tensors, fp32 lse."""
+    import torch
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
+                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, scale,
+                      int(bool(causal)), _ptr(workspace), workspace.numel(),
+                      _stream(stream)))
+    return dq, dk, dv
+
+
+def fa_decode_workspace_size(B: int, H: int, Lmax: int, d: int,
+                             num_splits: int = 0) -> int:
+    return int(load_library().fa_decode_workspace_size(B, H, Lmax, d, num_splits))
+
+
+def fa_decode_splitkv(q, kcache, vcache, seqlens, scale: float | None = None,
+                      num_splits: int = 0, o=None, lse=None, workspace=None,
+                      stream=None):
+    """Single-token attention over a KV cache, split-KV with LSE merge."""
+    import torch
+    lib = load_library()
+    _need(q, torch.bfloat16, "q")
+    _need(kcache, torch.bfloat16, "kcache")
+    _need(vcache, torch.bfloat16, "vcache")
+    _need(seqlens, torch.int32, "seqlens")
+    B, H, d = q.shape
+    Lmax = kcache.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = fa_decode_workspace_size(B, H, Lmax, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(lib.fa_decode_splitkv(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens),
+                                 _ptr(o), _ptr(lse), B, H, Lmax, d, scale,
+                                 num_splits, _ptr(workspace), workspace.numel(),
+                                 _stream(stream)))
+    return o, lse
+
+
+def fa_device_status(stream=None):
+    """Synchronise the stream; return (status, raw word) of the device."""
+    lib = load_library()
+    word = ctypes.c_uint(0)
+    st = lib.fa_device_status(_stream(stream), ctypes.byref(word))
+    return st, word.value
+
+
+def fa_set_wait_limit(nanoseconds: int):
+    load_library().fa_set_wait_limit(int(nanoseconds))
+
+
+def fa_debug_skip_load(enable: bool):
+    load_library().fa_debug_skip_load(int(bool(enable)))

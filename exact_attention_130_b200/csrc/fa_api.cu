@@ -1,0 +1,307 @@
+// fa_api.cu -- the C ABI of libfa_sm100.so: argument validation, per-device
+// state, TMA tensor-map encoding, and dispatch to the kernel launchers.
+// Every entry point validates before it touches the GPU and returns a status;
+// nothing here aborts or exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fa_internal.h"
+
+namespace fa {
+
+// One status word per device (each device gets its own copy of this
+// variable when the module loads there). Kernels write it when a bounded
+// wait gives up; fa_device_status() reads and clears it.
+__device__ unsigned int g_status_word;
+
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+
+struct DeviceState {
+  bool ready = false;
+  int num_sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  unsigned int* status_word = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<int> g_debug_skip{0};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status invalid(fa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+// Current device, its SM count and status word; set up once per device.
+fa_status device_ctx(cudaStream_t stream, LaunchCtx* ctx) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return invalid(FA_ERR_UNSUPPORTED, "device index %d", dev);
+  DeviceState& ds = g_dev[dev];
+  if (!ds.ready) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!ds.ready) {
+      cudaDeviceProp prop;
+      e = cudaGetDeviceProperties(&prop, dev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+      if (prop.major != 10 || prop.minor != 0)
+        return invalid(FA_ERR_UNSUPPORTED,
+                       "device %d is sm_%d%d; this library is built for sm_100a (B200)", dev,
+                       prop.major, prop.minor);
+      void* addr = nullptr;
+      e = cudaGetSymbolAddress(&addr, g_status_word);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+      ds.num_sms = prop.multiProcessorCount;
+      ds.cc_major = prop.major;
+      ds.cc_minor = prop.minor;
+      ds.status_word = static_cast<unsigned int*>(addr);
+      ds.ready = true;
+    }
+  }
+  ctx->stream = stream;
+  ctx->status_word = ds.status_word;
+  ctx->wait_limit_ns = g_wait_limit_ns.load();
+  ctx->num_sms = ds.num_sms;
+  ctx->debug_skip_load = 0;
+  return FA_OK;
+}
+
+fa_status check_bhnd(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1)
+    return invalid(FA_ERR_INVALID_ARG, "B, H, N must be >= 1 (got %d, %d, %d)", B, H, N);
+  const long long rows = (long long)B * H * N;
+  if (rows > 0x7fffffffLL)
+    return invalid(FA_ERR_INVALID_ARG, "B*H*N = %lld exceeds 2^31-1", rows);
+  if (d != 64 && d != 128) return invalid(FA_ERR_UNSUPPORTED, "head dim %d (need 64 or 128)", d);
+  return FA_OK;
+}
+
+fa_status check_scale(float scale) {
+  if (!std::isfinite(scale) || !(scale > 0.f))
+    return invalid(FA_ERR_INVALID_ARG, "scale must be finite and > 0 (got %g)", (double)scale);
+  return FA_OK;
+}
+
+fa_status check_ptrs(std::initializer_list<const void*> ptrs, const char* names) {
+  int i = 0;
+  for (const void* p : ptrs) {
+    if (p == nullptr) return invalid(FA_ERR_INVALID_ARG, "null pointer (argument %d of %s)", i, names);
+    if (!aligned16(p))
+      return invalid(FA_ERR_ALIGNMENT, "pointer %d of %s is not 16-byte aligned", i, names);
+    ++i;
+  }
+  return FA_OK;
+}
+
+}  // namespace
+
+void set_last_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+}
+
+fa_status cuda_fail(cudaError_t e, const char* what) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%s)", what, cudaGetErrorString(e),
+           cudaGetErrorName(e));
+  return FA_ERR_CUDA;
+}
+
+fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t inner,
+                       uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows,
+                       bool swizzle128) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return invalid(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const uint64_t elem = is_bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {inner, rows, outer};
+  cuuint64_t strides[2] = {inner * elem, inner * rows * elem};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return invalid(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+  return FA_OK;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+const char* fa_last_error(void) { return t_last_error; }
+
+int fa_abi_version(void) { return 100; }
+
+void fa_set_wait_limit(unsigned long long ns) {
+  g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs);
+}
+
+void fa_debug_skip_load(int enable) { g_debug_skip.store(enable ? 1 : 0); }
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, k, v, o, lse}, "fa_fwd(q,k,v,o,lse)")) != FA_OK) return st;
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (causal != 0 && causal != 1) return invalid(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  ctx.debug_skip_load = g_debug_skip.exchange(0);
+  return launch_fwd_bf16(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx);
+}
+
+fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B,
+                     int H, int N, int d, float scale, int causal, cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, k, v, o, lse}, "fa_fwd_f32(q,k,v,o,lse)")) != FA_OK) return st;
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (causal != 0 && causal != 1) return invalid(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  return launch_fwd_f32(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_bhnd(B, H, N, d) != FA_OK) return 0;
+  return bwd_workspace_bytes(B, H, N, d);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 float scale, int causal, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv},
+                       "fa_bwd(q,k,v,o,lse,dO,dq,dk,dv)")) != FA_OK)
+    return st;
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (causal != 0 && causal != 1) return invalid(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  const size_t need = bwd_workspace_bytes(B, H, N, d);
+  if (workspace == nullptr || workspace_bytes < need)
+    return invalid(FA_ERR_WORKSPACE, "fa_bwd needs %zu bytes of workspace (got %zu)", need,
+                   workspace ? workspace_bytes : size_t(0));
+  if (!aligned16(workspace)) return invalid(FA_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  return launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal != 0, workspace,
+                    ctx);
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Lmax, int d, int num_splits) {
+  if (B < 1 || H < 1 || Lmax < 1 || (d != 64 && d != 128) || num_splits < 0 || num_splits > 1024)
+    return 0;
+  // the automatic chunk count depends only on the shape (and the SM count,
+  // for which the size is taken at its maximum so a buffer sized here fits
+  // any device of this family)
+  const int chunks = decode_num_chunks(B, H, Lmax, num_splits, 0);
+  return decode_workspace_bytes(B, H, d, chunks);
+}
+
+fa_status fa_decode_splitkv(const void* q, const void* kcache, const void* vcache,
+                            const int* seqlens, void* o, float* lse, int B, int H, int Lmax, int d,
+                            float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, kcache, vcache, o, lse}, "fa_decode_splitkv(q,kcache,vcache,o,lse)")) !=
+      FA_OK)
+    return st;
+  if (seqlens == nullptr || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return invalid(FA_ERR_INVALID_ARG, "seqlens must be a non-null, 4-byte aligned int32 array");
+  if (B < 1 || H < 1 || Lmax < 1)
+    return invalid(FA_ERR_INVALID_ARG, "B, H, Lmax must be >= 1 (got %d, %d, %d)", B, H, Lmax);
+  if ((long long)B * H * Lmax > 0x7fffffffLL)
+    return invalid(FA_ERR_INVALID_ARG, "B*H*Lmax exceeds 2^31-1");
+  if (d != 64 && d != 128) return invalid(FA_ERR_UNSUPPORTED, "head dim %d (need 64 or 128)", d);
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (num_splits < 0 || num_splits > 1024)
+    return invalid(FA_ERR_INVALID_ARG, "num_splits must be in [0, 1024] (got %d)", num_splits);
+  const int chunks = decode_num_chunks(B, H, Lmax, num_splits, 0);
+  const size_t need = decode_workspace_bytes(B, H, d, chunks);
+  if (workspace == nullptr || workspace_bytes < need)
+    return invalid(FA_ERR_WORKSPACE, "fa_decode_splitkv needs %zu bytes of workspace (got %zu)",
+                   need, workspace ? workspace_bytes : size_t(0));
+  if (!aligned16(workspace)) return invalid(FA_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Lmax, d, scale, chunks,
+                       workspace, ctx);
+}
+
+fa_status fa_device_status(cudaStream_t stream, unsigned int* detail) {
+  if (detail) *detail = 0;
+  LaunchCtx ctx;
+  fa_status st = device_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  if (word) {
+    e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+  }
+  if (detail) *detail = word;
+  if (word) {
+    set_last_error("a device-side wait gave up: kernel %u, site %u", word >> 16, (word >> 8) & 0xff);
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

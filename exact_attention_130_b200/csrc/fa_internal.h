@@ -1,0 +1,62 @@
+// fa_internal.h -- declarations shared by the host API and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "fa.h"
+
+namespace fa {
+
+// Everything a launcher needs besides the tensors.
+struct LaunchCtx {
+  cudaStream_t stream;
+  unsigned int* status_word;      // device address of the status word
+  unsigned long long wait_limit_ns;
+  int num_sms;
+  int debug_skip_load;            // test hook, see fa_debug_skip_load()
+};
+
+// Kernel ids recorded in the status word.
+enum KernelId : unsigned int {
+  KID_FWD = 1,
+  KID_FWD_F32 = 2,
+  KID_BWD_PRE = 3,
+  KID_BWD = 4,
+  KID_BWD_POST = 5,
+  KID_DECODE = 6,
+  KID_DECODE_MERGE = 7,
+};
+
+// Records a message for fa_last_error() on this thread.
+void set_last_error(const char* fmt, ...);
+fa_status cuda_fail(cudaError_t e, const char* what);
+
+// 3-D tiled tensor map over a [outer, rows, inner] bf16 or fp32 tensor
+// (inner contiguous), box = box_inner x box_rows x 1, 128-byte swizzle when
+// `swizzle128` (box_inner * elem must then be 128 bytes), zero fill out of
+// bounds.
+fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t inner,
+                       uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows,
+                       bool swizzle128);
+
+fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int N, int d, float scale, bool causal,
+                          const LaunchCtx& ctx);
+fa_status launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                         int B, int H, int N, int d, float scale, bool causal,
+                         const LaunchCtx& ctx);
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                     int H, int N, int d, float scale, bool causal, void* workspace,
+                     const LaunchCtx& ctx);
+size_t bwd_workspace_bytes(int B, int H, int N, int d);
+int decode_num_chunks(int B, int H, int Lmax, int num_splits, int num_sms);
+size_t decode_workspace_bytes(int B, int H, int d, int chunks);
+fa_status launch_decode(const void* q, const void* kcache, const void* vcache,
+                        const int* seqlens, void* o, float* lse, int B, int H, int Lmax, int d,
+                        float scale, int chunks, void* workspace, const LaunchCtx& ctx);
+
+}  // namespace fa

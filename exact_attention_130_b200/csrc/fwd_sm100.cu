@@ -1,0 +1,469 @@
+// fwd_sm100.cu -- attention forward for B200 (sm_100a), bf16 in, fp32 accumulate.
+//
+// What it computes ("Bellek Duvarinin Fizigi", sections "Online Softmax" and
+// "Forward gecisin iskeleti"; notation of "FlashAttention'i Anlamak Bolum 1",
+// 0.2): for every query row i, O_i = sum_j softmax_j(S_i) V_j with
+// S_ij = scale * q_i . k_j, and LSE_i = ln sum_j exp(S_ij). S and P never
+// leave the chip: Q, K, V tiles are brought into shared memory by TMA, S and
+// the output accumulator O~ sit in tensor memory (TMEM), and the row softmax
+// is carried by the running maximum m and running sum l, rescaled by
+// exp(m_old - m_new) whenever m grows; O = O~ / l once, at the end.
+//
+// Exponentials use base 2: scores are multiplied by scale * log2(e) and every
+// exp(x) becomes 2^(x log2 e) ("Online Softmax", last paragraph); the saved
+// LSE is converted back to the natural logarithm.
+//
+// Causal mask ("Maskeleme ve Dropout"): K/V tiles wholly above the diagonal
+// are never loaded or multiplied; the diagonal tile gets -inf in the masked
+// entries before the row maximum is taken.
+//
+// B200 design (not the pages' A100/H100 kernels):
+//  * persistent grid, one CTA per SM, 10 warps:
+//      warps 0-3  softmax for Q tile 0 (one TMEM lane = one query row)
+//      warps 4-7  softmax for Q tile 1
+//      warp  8    TMA producer (Q tiles once per work unit, K/V ring)
+//      warp  9    tcgen05 MMA issuer (one thread)
+//  * a work unit is 2 Q tiles of 128 rows of one (batch, head); both share
+//    every K/V tile, which halves K/V shared-memory traffic per FLOP;
+//  * TMEM (512 columns): S_0 | S_1 | O_0 | O_1. The softmax writes P as bf16
+//    over the first half of its S columns and the PV MMA reads it from TMEM,
+//    so P never touches shared memory;
+//  * while one softmax warpgroup works on its S, the tensor core runs the
+//    other tile's QK^T and PV (ping-pong between the two Q tiles);
+//  * O~ is rescaled only when a row maximum grows by more than 2^8 (the
+//    final division by l is exact whatever reference maximum was used), so
+//    the O read-modify-write almost never runs;
+//  * causal units are ordered longest first so the persistent CTAs finish
+//    together;
+//  * every mbarrier wait is bounded in time; a wait that runs out records
+//    the failure in the device status word and the CTA returns.
+#include <cfloat>
+
+#include "fa_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kBM = 128;  // query rows per Q tile
+constexpr int kBN = 128;  // keys per K/V tile
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when m grows by > 2^8
+constexpr float kLn2 = 0.69314718055994530942f;
+
+// barrier slots
+enum : int {
+  B_Q_FULL = 0,    // +t
+  B_Q_EMPTY = 2,   // +t
+  B_S_FULL = 4,    // +t
+  B_P_FULL = 6,    // +t
+  B_O_FULL = 8,    // +t
+  B_O_EMPTY = 10,  // +t
+  B_DRAIN = 12,
+  B_K_FULL = 16,   // +stage
+  B_V_FULL = 20,   // +stage
+  B_KV_EMPTY = 24, // +stage
+  B_COUNT = 28
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kSub = D / 64;             // 128-byte column groups per row
+  static constexpr int kSubBytes = 128 * 128;     // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kSub * kSubBytes;
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kOffMisc = kOffBar + 8 * B_COUNT;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+};
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  int N;
+  int BH;
+  int n_kv;       // K/V tiles per head
+  int n_pairs;    // Q-tile pairs per head
+  int num_units;  // BH * n_pairs
+  float scale_log2;
+  unsigned int* status;
+  unsigned long long limit_ns;
+  int debug_skip;
+};
+
+__device__ __forceinline__ void unit_coords(int u, const FwdParams& p, int& bh, int& pair) {
+  // longest (highest) Q-tile pairs first; all heads of a pair level together
+  pair = p.n_pairs - 1 - u / p.BH;
+  bh = u % p.BH;
+}
+
+template <bool CAUSAL>
+__device__ __forceinline__ int kv_tiles_for(int qtile, int n_kv) {
+  if (CAUSAL) return min(qtile + 1, n_kv);
+  return n_kv;
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kOffBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * uint32_t(i); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(BAR(B_Q_FULL + t), 1);
+      mbar_init(BAR(B_Q_EMPTY + t), 1);
+      mbar_init(BAR(B_S_FULL + t), 1);
+      mbar_init(BAR(B_P_FULL + t), 4);
+      mbar_init(BAR(B_O_FULL + t), 1);
+      mbar_init(BAR(B_O_EMPTY + t), 4);
+    }
+    mbar_init(BAR(B_DRAIN), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(BAR(B_K_FULL + s), 1);
+      mbar_init(BAR(B_V_FULL + s), 1);
+      mbar_init(BAR(B_KV_EMPTY + s), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    tma_prefetch_map(&tmQ);
+    tma_prefetch_map(&tmK);
+    tma_prefetch_map(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_FWD};
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int kv_issued = 0, unit_iter = 0;
+      int q_cnt[2] = {0, 0};
+      int k_cnt[L::kStages], v_cnt[L::kStages];
+      for (int s = 0; s < L::kStages; ++s) k_cnt[s] = v_cnt[s] = 0;
+      bool skip_pending = p.debug_skip && blockIdx.x == 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++unit_iter) {
+        int bh, pair;
+        unit_coords(u, p, bh, pair);
+        const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
+        for (int t = 0; t < 2 && ok; ++t) {
+          ok = wait_bounded(BAR(B_Q_EMPTY + t), (unit_iter & 1) ^ 1, wc, 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(BAR(B_Q_FULL + t), L::kTileBytes);
+          for (int c = 0; c < L::kSub; ++c)
+            tma_load_3d(sbase + L::kOffQ + t * L::kTileBytes + c * L::kSubBytes, &tmQ,
+                        BAR(B_Q_FULL + t), c * 64, (2 * pair + t) * kBM, bh);
+          ++q_cnt[t];
+        }
+        for (int j = 0; ok && j < n1; ++j, ++kv_issued) {
+          const int s = kv_issued % L::kStages;
+          const uint32_t ph = (kv_issued / L::kStages) & 1;
+          ok = wait_bounded(BAR(B_KV_EMPTY + s), ph ^ 1, wc, 2);
+          if (!ok) break;
+          mbar_arrive_expect_tx(BAR(B_K_FULL + s), L::kTileBytes);
+          for (int c = 0; c < L::kSub; ++c)
+            tma_load_3d(sbase + L::kOffK + s * L::kTileBytes + c * L::kSubBytes, &tmK,
+                        BAR(B_K_FULL + s), c * 64, j * kBN, bh);
+          ++k_cnt[s];
+          if (skip_pending) {
+            skip_pending = false;  // test hook: this V tile never arrives
+          } else {
+            mbar_arrive_expect_tx(BAR(B_V_FULL + s), L::kTileBytes);
+            for (int c = 0; c < L::kSub; ++c)
+              tma_load_3d(sbase + L::kOffV + s * L::kTileBytes + c * L::kSubBytes, &tmV,
+                          BAR(B_V_FULL + s), c * 64, j * kBN, bh);
+            ++v_cnt[s];
+          }
+        }
+      }
+      if (*abort_flag) {
+        // let every copy this thread started land before the CTA exits
+        for (int t = 0; t < 2; ++t)
+          if (q_cnt[t]) wait_bounded(BAR(B_Q_FULL + t), (q_cnt[t] - 1) & 1, wc, 3, true);
+        for (int s = 0; s < L::kStages; ++s) {
+          if (k_cnt[s]) wait_bounded(BAR(B_K_FULL + s), (k_cnt[s] - 1) & 1, wc, 3, true);
+          if (v_cnt[s]) wait_bounded(BAR(B_V_FULL + s), (v_cnt[s] - 1) & 1, wc, 3, true);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, false, true);
+      const uint32_t colS[2] = {L::kColS0, L::kColS1};
+      const uint32_t colO[2] = {L::kColO0, L::kColO1};
+      auto issue_qk = [&](int t, int stage) {
+        const uint32_t qa = sbase + L::kOffQ + t * L::kTileBytes;
+        const uint32_t kb = sbase + L::kOffK + stage * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
+          mma_ss(tmem + colS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                 idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int stage, bool acc) {
+        const uint32_t vb = sbase + L::kOffV + stage * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8,
+                 sdesc_sw128(vb + kk * 16 * 128, L::kSubBytes, 1024), idesc_pv,
+                 (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      int kv_used = 0, unit_iter = 0;
+      int p_cnt[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++unit_iter) {
+        int bh, pair;
+        unit_coords(u, p, bh, pair);
+        const int n[2] = {kv_tiles_for<CAUSAL>(2 * pair, p.n_kv),
+                          kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv)};
+        for (int t = 0; t < 2 && ok; ++t)
+          ok = wait_bounded(BAR(B_Q_FULL + t), unit_iter & 1, wc, 10);
+        if (!ok) break;
+        {
+          const int s0 = kv_used % L::kStages;
+          ok = wait_bounded(BAR(B_K_FULL + s0), (kv_used / L::kStages) & 1, wc, 11);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(0, s0);
+          tc_commit(BAR(B_S_FULL + 0));
+          issue_qk(1, s0);
+          tc_commit(BAR(B_S_FULL + 1));
+        }
+        int k_ready = 0;
+        for (int j = 0; ok && j < n[1]; ++j) {
+          const int s = (kv_used + j) % L::kStages;
+          ok = wait_bounded(BAR(B_V_FULL + s), ((kv_used + j) / L::kStages) & 1, wc, 12);
+          if (!ok) break;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= n[t]) continue;
+            if (j == 0) {
+              ok = wait_bounded(BAR(B_O_EMPTY + t), (unit_iter & 1) ^ 1, wc, 13);
+              if (!ok) break;
+            }
+            ok = wait_bounded(BAR(B_P_FULL + t), p_cnt[t] & 1, wc, 14);
+            if (!ok) break;
+            ++p_cnt[t];
+            tc_fence_after();
+            issue_pv(t, s, j > 0);
+            if (j + 1 < n[t]) {
+              const int s2 = (kv_used + j + 1) % L::kStages;
+              if (k_ready < j + 1) {
+                ok = wait_bounded(BAR(B_K_FULL + s2), ((kv_used + j + 1) / L::kStages) & 1, wc,
+                                  15);
+                if (!ok) break;
+                k_ready = j + 1;
+                tc_fence_after();
+              }
+              issue_qk(t, s2);
+              tc_commit(BAR(B_S_FULL + t));
+            } else {
+              tc_commit(BAR(B_O_FULL + t));
+              tc_commit(BAR(B_Q_EMPTY + t));
+            }
+          }
+          if (!ok) break;
+          tc_commit(BAR(B_KV_EMPTY + s));
+        }
+        kv_used += n[1];
+      }
+      // every MMA issued above must be finished before TMEM is released
+      tc_commit(BAR(B_DRAIN));
+      wait_bounded(BAR(B_DRAIN), 0, wc, 16, true);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;          // Q tile of this warpgroup
+    const int wq = warp & 3;          // TMEM lane quadrant of this warp
+    const int r = wq * 32 + lane;     // row inside the Q tile
+    const uint32_t lane_base = uint32_t(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (t ? L::kColS1 : L::kColS0);
+    const uint32_t tO = tmem + lane_base + (t ? L::kColO1 : L::kColO0);
+    const float c = p.scale_log2;
+    int s_cnt = 0, unit_iter = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++unit_iter) {
+      int bh, pair;
+      unit_coords(u, p, bh, pair);
+      const int qt = 2 * pair + t;
+      const int nt = kv_tiles_for<CAUSAL>(qt, p.n_kv);
+      const int row = qt * kBM + r;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        ok = wait_bounded(BAR(B_S_FULL + t), s_cnt & 1, wc, 20);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld128_wait(tS, sr);
+        float s[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
+        // mask: the diagonal tile under the causal mask, and keys >= N
+        int limit = p.N - j * kBN;
+        if (CAUSAL && j == qt) limit = min(limit, r + 1);
+        if (limit < kBN) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) s[i] = (i < limit) ? s[i] : -INFINITY;
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int i = 4; i < 128; i += 4) {
+          mx0 = fmaxf(mx0, s[i]);
+          mx1 = fmaxf(mx1, s[i + 1]);
+          mx2 = fmaxf(mx2, s[i + 2]);
+          mx3 = fmaxf(mx3, s[i + 3]);
+        }
+        const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c);
+        if (j == 0) {
+          m = m_new;
+        } else if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
+          // O~ holds the sum up to tile j-1 (its MMA finished before S_j was
+          // committed): multiply it by 2^(m_old - m_new)
+          const float alpha = ex2_approx(m - m_new);
+          m = m_new;
+          l *= alpha;
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t orow[32];
+            tmem_ld32_wait(tO + ch * 32, orow);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+            tmem_st32(tO + ch * 32, orow);
+          }
+        }
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        uint32_t pk[64];
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float p0 = ex2_approx(fmaf(s[2 * i], c, neg_m));
+          const float p1 = ex2_approx(fmaf(s[2 * i + 1], c, neg_m));
+          rs0 += p0;
+          rs1 += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st64(tS, pk);  // P (bf16) over the first 64 columns of S
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_P_FULL + t));
+        l += rs0 + rs1;
+      }
+      if (!ok) break;
+      // epilogue: O = O~ / l, LSE = ln2 * (m + log2 l)
+      ok = wait_bounded(BAR(B_O_FULL + t), unit_iter & 1, wc, 21);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      uint16_t* orow_g = reinterpret_cast<uint16_t*>(p.o) + (size_t(bh) * p.N + size_t(row)) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t orow[32];
+        tmem_ld32_wait(tO + ch * 32, orow);
+        if (row < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow_g + ch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(orow[8 * v4 + 0]) * inv_l,
+                              __uint_as_float(orow[8 * v4 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(orow[8 * v4 + 2]) * inv_l,
+                              __uint_as_float(orow[8 * v4 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(orow[8 * v4 + 4]) * inv_l,
+                              __uint_as_float(orow[8 * v4 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(orow[8 * v4 + 6]) * inv_l,
+                              __uint_as_float(orow[8 * v4 + 7]) * inv_l);
+            dst[v4] = w;
+          }
+        }
+      }
+      if (row < p.N) p.lse[size_t(bh) * p.N + row] = (m + lg2_approx(l)) * kLn2;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_O_EMPTY + t));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool CAUSAL>
+fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                 const FwdParams& p, const LaunchCtx& ctx) {
+  auto kern = fwd_kernel<D, CAUSAL>;
+  const int smem = Layout<D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fwd)");
+  const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
+  kern<<<grid, kThreads, smem, ctx.stream>>>(mq, mk, mv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
+  return FA_OK;
+}
+
+}  // namespace
+
+fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int N, int d, float scale, bool causal,
+                          const LaunchCtx& ctx) {
+  const uint64_t BH = uint64_t(B) * uint64_t(H);
+  CUtensorMap mq, mk, mv;
+  fa_status st;
+  if ((st = make_tmap_3d(&mq, q, true, d, N, BH, 64, 128, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mk, k, true, d, N, BH, 64, 128, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mv, v, true, d, N, BH, 64, 128, true)) != FA_OK) return st;
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.N = N;
+  p.BH = int(BH);
+  p.n_kv = (N + kBN - 1) / kBN;
+  p.n_pairs = (p.n_kv + 1) / 2;
+  p.num_units = p.BH * p.n_pairs;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = ctx.status_word;
+  p.limit_ns = ctx.wait_limit_ns;
+  p.debug_skip = ctx.debug_skip_load;
+  if (d == 128) return causal ? launch<128, true>(mq, mk, mv, p, ctx)
+                              : launch<128, false>(mq, mk, mv, p, ctx);
+  return causal ? launch<64, true>(mq, mk, mv, p, ctx) : launch<64, false>(mq, mk, mv, p, ctx);
+}
+
+}  // namespace fa

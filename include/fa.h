@@ -1,0 +1,187 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library libfa_sm100.so
+ *
+ * The library computes exact scaled dot-product attention
+ *
+ *     S = scale * Q K^T  (+ causal mask),  P = softmax_row(S),  O = P V
+ *
+ * without ever writing S or P to device memory: K/V tiles stream through
+ * shared memory, S and the output accumulator live in tensor memory, and the
+ * row softmax is carried by the running maximum / running sum recurrence.
+ * Definitions followed:
+ *   - "FlashAttention'i Anlamak Bolum 1" (blog.edumints.com), 0.2 Notasyon:
+ *     the function S = QK^T/sqrt(d) + B, P = softmax_row(S), O = PV.
+ *   - "Bellek Duvarinin Fizigi" (webturing Principia): "Online Softmax" and
+ *     "Forward gecisin iskeleti" (tiling, running max/sum, final division),
+ *     "Maskeleme ve Dropout" (causal mask with skipped tiles),
+ *     "Geri Yayilim" (backward by recomputing P from the saved log-sum-exp),
+ *     "Decode Asamasi: Flash-Decoding" (split-KV decode merged by LSE).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Layout: row-major [B, H, N, d], contiguous (head dim fastest). The
+ *    per-row log-sum-exp is fp32 [B, H, N]. bf16 tensors are passed as
+ *    void* holding IEEE bfloat16.
+ *  - LSE_i = ln sum_j exp(S_ij), natural logarithm, scale already inside S.
+ *  - Causal: query i sees key j iff j <= i (N_q = N_k = N).
+ *  - Ownership: every pointer is caller-owned DEVICE memory; the library
+ *    never frees or retains it past the call. The library allocates no
+ *    device memory per call (it keeps one 4-byte device status word per
+ *    device, a __device__ variable of the library).
+ *  - Alignment: every tensor pointer must be 16-byte aligned (TMA needs
+ *    16-byte global addresses), else FA_ERR_ALIGNMENT.
+ *  - Execution: all device work is enqueued on `stream` (0 = legacy default
+ *    stream) and the call returns without synchronising. Argument errors are
+ *    returned before anything is launched and leave outputs untouched.
+ *  - Errors: FA_ERR_CUDA carries the CUDA error text (fa_last_error()).
+ *    A kernel wait that exceeds its time limit does not hang the GPU: the
+ *    kernel records it in the device status word and returns; the host sees
+ *    it as FA_ERR_TIMEOUT from fa_device_status().
+ *  - The library never aborts or exits the process.
+ */
+#ifndef FA_SM100_H
+#define FA_SM100_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, non-finite scale   */
+    FA_ERR_UNSUPPORTED = 2,   /* head dim or device not supported           */
+    FA_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned           */
+    FA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than needed   */
+    FA_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed          */
+    FA_ERR_TIMEOUT = 6        /* a device-side wait gave up (see above)     */
+} fa_status;
+
+/* Static, human-readable name of a status code. */
+const char* fa_status_string(fa_status s);
+
+/* Text of the last FA_ERR_CUDA / validation failure on the calling thread. */
+const char* fa_last_error(void);
+
+/* Version of this ABI (major * 100 + minor). */
+int fa_abi_version(void);
+
+/*
+ * fa_fwd -- attention forward, bf16 in / bf16 out, fp32 accumulation.
+ *   q, k, v : bf16 [B, H, N, d]          (input, device)
+ *   o       : bf16 [B, H, N, d]          (output, device)
+ *   lse     : fp32 [B, H, N]             (output, device; natural log)
+ *   B, H, N : >= 1;  B*H*N <= 2^31 - 1
+ *   d       : 64 or 128 (else FA_ERR_UNSUPPORTED)
+ *   scale   : finite, usually 1/sqrt(d)
+ *   causal  : 0 or 1
+ * Passages: "Forward gecisin iskeleti" (tiles of Q, K, V; running m, l and
+ * O~; O = diag(l)^-1 O~ at the end), "Online Softmax" (exp2 form with the
+ * scores pre-scaled by log2 e), "Maskeleme ve Dropout" (tiles above the
+ * diagonal skipped, the diagonal tile masked before the row maximum).
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o,
+                 float* lse, int B, int H, int N, int d, float scale,
+                 int causal, cudaStream_t stream);
+
+/*
+ * fa_fwd_f32 -- the same forward on fp32 tensors, computed in fp32.
+ *   q, k, v, o : fp32 [B, H, N, d];  lse : fp32 [B, H, N]
+ *   d : 64 or 128; N <= 4096 (a small-problem path: fp32 inputs are not
+ *   rounded to a tensor-core type, so this path runs on the CUDA cores).
+ * Passages as for fa_fwd.
+ */
+fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o,
+                     float* lse, int B, int H, int N, int d, float scale,
+                     int causal, cudaStream_t stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of scratch fa_bwd needs: an fp32 dQ
+ * accumulator [B, H, N, d] and the fp32 vector D [B, H, N], each padded to
+ * 256 bytes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd -- attention backward by recomputation.
+ *   q, k, v, o, dO : bf16 [B, H, N, d]   (input; o is fa_fwd's output)
+ *   lse            : fp32 [B, H, N]      (input; fa_fwd's output)
+ *   dq, dk, dv     : bf16 [B, H, N, d]   (output)
+ *   workspace      : device scratch of >= fa_bwd_workspace_size() bytes,
+ *                    16-byte aligned; its contents on entry do not matter
+ *                    and are overwritten.
+ * Computes D = rowsum(dO * O), then per key tile recomputes
+ * P = exp(S - LSE), dV = P^T dO, dP = dO V^T, dS = P * (dP - D),
+ * dK = scale dS^T Q, dQ = scale dS K ("Geri Yayilim").
+ * d : 64 or 128. Deterministic for dK and dV; dQ is summed with fp32
+ * atomics, so its low bits may differ between runs.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dO, void* dq, void* dk,
+                 void* dv, int B, int H, int N, int d, float scale,
+                 int causal, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream);
+
+/*
+ * fa_decode_workspace_size -- bytes of scratch fa_decode_splitkv needs for
+ * per-chunk partial results: fp32 [B, H, C, d] outputs and fp32 [B, H, C]
+ * log-sum-exps, C = the chunk count the call will use (num_splits, or the
+ * automatic choice when num_splits == 0).
+ */
+size_t fa_decode_workspace_size(int B, int H, int Lmax, int d, int num_splits);
+
+/*
+ * fa_decode_splitkv -- one query token per (sequence, head) against a KV
+ * cache, split along the cache into C chunks whose partial (o_c, lse_c) are
+ * merged by log-sum-exp ("Decode Asamasi: Flash-Decoding").
+ *   q               : bf16 [B, H, d]
+ *   kcache, vcache  : bf16 [B, H, Lmax, d]
+ *   seqlens         : int32 [B] on the device; keys 0 .. seqlens[b]-1 are
+ *                     visible; 1 <= seqlens[b] <= Lmax is the caller's
+ *                     contract (values outside it are clamped to [0, Lmax]
+ *                     and a sequence with no visible key gets O = 0 and
+ *                     LSE = -inf)
+ *   o               : bf16 [B, H, d];  lse : fp32 [B, H]
+ *   num_splits      : chunks per sequence, 0 = automatic, <= 1024
+ *   workspace       : >= fa_decode_workspace_size(B, H, Lmax, d, num_splits)
+ * Cache positions at or past seqlens[b] are never read. d : 128 or 64.
+ * Deterministic: chunks are merged in a fixed order.
+ */
+fa_status fa_decode_splitkv(const void* q, const void* kcache,
+                            const void* vcache, const int* seqlens, void* o,
+                            float* lse, int B, int H, int Lmax, int d,
+                            float scale, int num_splits, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fa_device_status -- synchronises `stream`, reads and clears the current
+ * device's status word. Returns FA_ERR_TIMEOUT if any kernel of this
+ * library gave up a wait since the last check, FA_ERR_CUDA if the
+ * synchronisation itself failed, else FA_OK. *detail (may be NULL) gets the
+ * raw word: kernel id << 16 | wait site << 8 | 1.
+ */
+fa_status fa_device_status(cudaStream_t stream, unsigned int* detail);
+
+/*
+ * fa_set_wait_limit -- time limit of every device-side wait, in
+ * nanoseconds, for launches made after the call (default 2e9, i.e. 2 s;
+ * 0 restores the default). Process-wide.
+ */
+void fa_set_wait_limit(unsigned long long nanoseconds);
+
+/*
+ * fa_debug_skip_load -- test hook: when nonzero, the next fa_fwd launch has
+ * its first CTA skip one V-tile load, so that the consumer's wait runs out
+ * and the kernel reports FA_ERR_TIMEOUT instead of producing output. Reset
+ * to 0 by that launch.
+ */
+void fa_debug_skip_load(int enable);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H */

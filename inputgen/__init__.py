@@ -14,15 +14,18 @@ Recipe
 * workload ``k`` (0..4) draws from ``numpy.random.default_rng(20260 + k)``;
 * draws are float32 standard normals, taken in the order Q, K, V, dO;
 * the split-KV decode workload first draws its per-sequence cache lengths
-  with ``rng.integers(16384, 32769, size=B)``, then q, then the K cache one
-  sequence at a time (only the first ``seqlen[b]`` positions), then the V
-  cache the same way; cache positions at or past ``seqlen[b]`` are filled
-  with NaN so that a kernel that reads past the logical end poisons its own
-  result;
+  with ``rng.integers(16384, 32769, size=B)``, then q; the K (V) cache rows
+  of sequence b come from their own generator,
+  ``default_rng(SeedSequence([seed, 1 (2 for V), b]))``, drawn head by
+  head as [seqlen[b], d] blocks, so sequences can be drawn in parallel; cache
+  positions at or past ``seqlen[b]`` are filled with NaN so that a kernel
+  that reads past the logical end poisons its own result;
 * bf16 rounding is round-to-nearest-even on the fp32 bit pattern.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -139,12 +142,21 @@ def make_decode_inputs(w: Workload, seqlens=None):
     drawn = rng.integers(lo, hi + 1, size=w.B).astype(np.int32)
     lens = drawn if seqlens is None else np.asarray(seqlens, dtype=np.int32)
     q = standard_normal_bf16(rng, (w.B, w.H, w.d))
-    kc = np.full((w.B, w.H, w.N, w.d), 0x7FC0, dtype=np.uint16)
-    vc = np.full((w.B, w.H, w.N, w.d), 0x7FC0, dtype=np.uint16)
-    for b in range(w.B):
-        kc[b, :, : lens[b]] = standard_normal_bf16(rng, (w.H, int(lens[b]), w.d))
-    for b in range(w.B):
-        vc[b, :, : lens[b]] = standard_normal_bf16(rng, (w.H, int(lens[b]), w.d))
+    kc = np.empty((w.B, w.H, w.N, w.d), dtype=np.uint16)
+    vc = np.empty((w.B, w.H, w.N, w.d), dtype=np.uint16)
+
+    def fill(job):
+        which, b = job
+        cache = kc if which == 1 else vc
+        n = int(lens[b])
+        g = np.random.default_rng(np.random.SeedSequence([w.seed, which, b]))
+        cache[b, :, n:] = 0x7FC0
+        for h in range(w.H):  # one head at a time keeps the fp32 draw small
+            cache[b, h, :n] = standard_normal_bf16(g, (n, w.d))
+
+    jobs = [(which, b) for which in (1, 2) for b in range(w.B)]
+    with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, jobs))
     return {"q": q, "kcache": kc, "vcache": vc, "seqlens": lens}
 
 

@@ -1,0 +1,88 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments before touching the device."""
+import ctypes
+import subprocess
+
+import pytest
+
+import exact_attention_130_b200 as fa
+
+EXPECTED = {
+    "fa_status_string", "fa_last_error", "fa_abi_version", "fa_fwd",
+    "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd",
+    "fa_decode_workspace_size", "fa_decode_splitkv", "fa_device_status",
+    "fa_set_wait_limit", "fa_debug_skip_load",
+}
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return fa.load_library()
+
+
+def test_header_declares_expected_entry_points():
+    assert set(fa.exported_symbols()) == EXPECTED
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    dyn = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in fa.exported_symbols():
+        assert name in dyn, name
+        assert getattr(lib, name) is not None
+
+
+def test_status_strings(lib):
+    for code, name in fa.STATUS.items():
+        assert lib.fa_status_string(code).decode() == name
+    assert lib.fa_abi_version() == 100
+
+
+def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=8, d=64,
+         scale=0.125, causal=0):
+    P = ctypes.c_void_p
+    return lib.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, scale, causal,
+                      None)
+
+
+def test_fwd_argument_errors_need_no_device(lib):
+    assert _fwd(lib, q=0) == 1                    # null pointer
+    assert _fwd(lib, k=24) == 3                   # not 16-byte aligned
+    assert b"16-byte" in lib.fa_last_error()
+    assert _fwd(lib, N=0) == 1
+    assert _fwd(lib, B=-1) == 1
+    assert _fwd(lib, d=96) == 2                   # unsupported head dim
+    assert _fwd(lib, scale=float("nan")) == 1
+    assert _fwd(lib, scale=-1.0) == 1
+    assert _fwd(lib, causal=2) == 1
+    assert _fwd(lib, B=1 << 16, H=1 << 16, N=2) == 1   # B*H*N overflow
+
+
+def test_bwd_and_decode_argument_errors(lib):
+    P = ctypes.c_void_p
+    # workspace too small
+    st = lib.fa_bwd(P(16), P(16), P(16), P(16), P(16), P(16), P(16), P(16),
+                    P(16), 1, 1, 8, 64, 0.125, 0, P(16), 8, None)
+    assert st == 4
+    st = lib.fa_decode_splitkv(P(16), P(16), P(16), P(16), P(16), P(16), 1, 1,
+                               8, 64, 0.125, 0, P(16), 0, None)
+    assert st == 4
+    st = lib.fa_decode_splitkv(P(16), P(16), P(16), P(0), P(16), P(16), 1, 1,
+                               8, 64, 0.125, 0, P(16), 1 << 20, None)
+    assert st == 1
+    st = lib.fa_decode_splitkv(P(16), P(16), P(16), P(16), P(16), P(16), 1, 1,
+                               8, 64, 0.125, 2000, P(16), 1 << 20, None)
+    assert st == 1
+
+
+def test_workspace_sizes(lib):
+    # dQ accumulator (fp32 [B,H,N,d]) + D (fp32 [B,H,N]), each 256-aligned
+    assert fa.fa_bwd_workspace_size(2, 16, 4096, 128) == 2 * 16 * 4096 * 128 * 4 + 2 * 16 * 4096 * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 0, 64) == 0
+    # decode: C chunks of partial outputs and LSEs
+    ws = fa.fa_decode_workspace_size(8, 32, 32768, 128, 16)
+    assert ws == 8 * 32 * 16 * 128 * 4 + 8 * 32 * 16 * 4
+    assert fa.fa_decode_workspace_size(8, 32, 32768, 128, 0) == ws  # auto = 16 here
+    assert fa.fa_decode_workspace_size(1, 1, 100, 128, 0) > 0
+    assert fa.fa_decode_workspace_size(1, 1, 100, 96, 0) == 0

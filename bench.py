@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of the prefill
+workload (B=4, H=16, N=2048, d=128, bf16, iid N(0,1) inputs):
+  1. fa_fwd, no mask             (O, LSE)
+  2. fa_fwd, causal mask         (O, LSE)
+  3. fa_bwd, causal mask         (dQ, dK, dV from step 2's O and LSE and a dO)
+  4. fa_decode_splitkv           (one new query token per sequence and head
+                                  against the step's K/V as the cache,
+                                  every cache length 2048)
+The metric is attention TFLOP/s: FLOPs are 4 B H N^2 d per forward (halved
+under the causal mask), 2.5x that for the backward, 4 H L d per decoded
+token; `value` is the whole-job throughput over all ranks. The JSON line also
+carries a per-kernel breakdown with each kernel's fraction of its roofline
+(tensor peak for the forward/backward, HBM bandwidth for decode).
+
+Inputs are resident in HBM when the timed region starts; L2 (126 MB) is
+flushed between timed steps by writing a 256 MB buffer outside the timed
+events. `e2e` repeats the measurement through the same C ABI calls with the
+step's inputs copied from pinned host memory and every output copied back,
+inside the timed region.
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (weak
+scaling, no collective on the data path); the timed region is bracketed by a
+barrier and a device synchronise on both sides and the per-rank time is
+reduced with MAX.
+
+--impl reference times the fp64 CPU oracle (the only reference this build
+has) on a bounded sample of the same workload per step, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("attention fwd/bwd TFLOP/s (bf16,d=128) as % of B200 tensor peak; "
+          "decode HBM GB/s")
+WORKLOAD_NAME = "prefill"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world, local):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _reduce(world, x: float, op: str) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def dist_max(world, x: float) -> float:
+    """Slowest rank's time: the job is done when the last rank is."""
+    return _reduce(world, x, "max")
+
+
+def dist_sum(world, x: float) -> float:
+    """Work summed over ranks (weak scaling: every rank runs its own batch)."""
+    return _reduce(world, x, "sum")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region (NVML, every 5 ms)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2,
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sync_boost": 0x10,
+        "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no clocks rather than fail
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0}
+        names = [n for n, bit in self.REASONS.items()
+                 if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# peaks and recorded DRAM traffic
+# ---------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "source": "measured (MEASURED_PEAKS.json, burst)"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_source_hash(name: str) -> str:
+    files = {"fwd": "fwd_sm100.cu", "bwd_main": "bwd_sm100.cu",
+             "decode_split": "decode_sm100.cu"}
+    path = os.path.join(ROOT, "exact_attention_130_b200", "csrc", files.get(name, ""))
+    try:
+        return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except Exception:
+        return ""
+
+
+def recorded_traffic(name: str):
+    """DRAM bytes per launch from the committed ncu capture, if the kernel
+    source is unchanged since it was taken; else None."""
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        k = rec["kernels"][name]
+        if k["source_sha256_16"] != kernel_source_hash(name):
+            return None
+        return float(k["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import exact_attention_130_b200 as fa
+    import inputgen
+    from exact_attention_130_b200 import counters as C
+
+    dist_init(world, local)
+    w = inputgen.WORKLOADS[WORKLOAD_NAME]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    x = inputgen.make_attention_inputs(w, with_grad=True)
+    host = {n: torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).pin_memory()
+            for n in ("q", "k", "v", "do")}
+    dev = {n: t.cuda() for n, t in host.items()}
+    lens = torch.full((B,), N, dtype=torch.int32, device="cuda")
+    qdec = dev["q"][:, :, -1].contiguous()
+    out = {
+        "o_full": torch.empty_like(dev["q"]), "lse_full": torch.empty((B, H, N), dtype=torch.float32, device="cuda"),
+        "o_causal": torch.empty_like(dev["q"]), "lse_causal": torch.empty((B, H, N), dtype=torch.float32, device="cuda"),
+        "dq": torch.empty_like(dev["q"]), "dk": torch.empty_like(dev["q"]), "dv": torch.empty_like(dev["q"]),
+        "o_dec": torch.empty_like(qdec), "lse_dec": torch.empty((B, H), dtype=torch.float32, device="cuda"),
+    }
+    ws_bwd = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    ws_dec = torch.empty(fa.fa_decode_workspace_size(B, H, N, d, 0), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def step(src):
+        fa.fa_fwd(src["q"], src["k"], src["v"], causal=False, o=out["o_full"], lse=out["lse_full"])
+        fa.fa_fwd(src["q"], src["k"], src["v"], causal=True, o=out["o_causal"], lse=out["lse_causal"])
+        fa.fa_bwd(src["q"], src["k"], src["v"], out["o_causal"], out["lse_causal"], src["do"],
+                  causal=True, dq=out["dq"], dk=out["dk"], dv=out["dv"], workspace=ws_bwd)
+        fa.fa_decode_splitkv(src["qdec"], src["k"], src["v"], lens, o=out["o_dec"],
+                             lse=out["lse_dec"], workspace=ws_dec)
+
+    src_dev = dict(dev, qdec=qdec)
+    launches_per_step = 1 + 1 + 3 + 2
+    flops = {
+        "fwd": C.fwd_flops(B, H, N, d, False) + C.fwd_flops(B, H, N, d, True),
+        "bwd_main": C.bwd_flops(B, H, N, d, True),
+        "decode_split": C.decode_flops(H, [N] * B, d),
+    }
+    step_flops = sum(flops.values())
+    dec_bytes = C.decode_bytes(H, [N] * B, d)
+
+    def timed(fn, k):
+        """Run k steps; return summed device ms of the steps (L2 flushed in between)."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(k)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(k)]
+        for i in range(k):
+            flush.zero_()
+            starts[i].record()
+            fn()
+            ends[i].record()
+        torch.cuda.synchronize()
+        return sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+
+    # warm-up
+    for _ in range(args.warmup):
+        step(src_dev)
+    torch.cuda.synchronize()
+    st, word = fa.fa_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
+
+    # 1. headline: device-resident inputs
+    sampler = ClockSampler(local)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        ms = timed(lambda: step(src_dev), args.steps)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    ms_max = dist_max(world, ms)
+    total_flops = dist_sum(world, step_flops * args.steps)
+    value = total_flops / (ms_max * 1e-3) / 1e12
+
+    # 2. per-kernel breakdown (CUDA events around every launch, same steps)
+    fa.fa_profile_begin()
+    timed(lambda: step(src_dev), args.steps)
+    prof = fa.fa_profile_end()
+    peaks = load_peaks()
+    kernels = {}
+    for name, (n, tot) in prof.items():
+        avg = tot / n
+        entry = {"launches": n, "avg_ms": round(avg, 5)}
+        if name in ("fwd", "bwd_main"):
+            tf = flops[name] * args.steps / (tot * 1e-3) / 1e12
+            entry.update({"tflops": round(tf, 1), "frac_of_tensor_peak": round(tf / peaks["bf16_tflops"], 4)})
+        elif name == "decode_split":
+            gbs = dec_bytes * args.steps / (tot * 1e-3) / 1e9
+            entry.update({"gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)})
+        kernels[name] = entry
+    dominant = max(prof, key=lambda k: prof[k][1])
+    dn, dtot = prof[dominant]
+    # algorithmic work of one launch: the forward runs twice per step (no mask,
+    # causal), the backward main kernel once
+    per_launch_flops = flops["fwd"] / 2 if dominant == "fwd" else flops.get(dominant, 0.0)
+    if dominant in ("fwd", "bwd_main"):
+        achieved = flops[dominant] * args.steps / (dtot * 1e-3) / 1e12
+        roofline = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 1),
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": round(achieved / peaks["bf16_tflops"], 4),
+                    "traffic": recorded_traffic(dominant),
+                    "algorithmic_per_launch": per_launch_flops,
+                    "peak_source": peaks["source"]}
+    else:
+        achieved = dec_bytes * args.steps / (dtot * 1e-3) / 1e9
+        roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4),
+                    "traffic": recorded_traffic(dominant),
+                    "algorithmic_per_launch": dec_bytes, "peak_source": peaks["source"]}
+
+    # 3. end to end through the same calls with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+        host_qdec = host["q"][:, :, -1].contiguous().pin_memory()
+        bufs = {n: torch.empty_like(t) for n, t in dev.items()}
+        bufs["qdec"] = torch.empty_like(qdec)
+        h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_qdec.numel() * 2
+        d2h = sum(t.numel() * t.element_size() for t in out.values())
+
+        def e2e_step():
+            for n in ("q", "k", "v", "do"):
+                bufs[n].copy_(host[n], non_blocking=True)
+            bufs["qdec"].copy_(host_qdec, non_blocking=True)
+            step(bufs)
+            for k, t in out.items():
+                h_out[k].copy_(t, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        dist_barrier(world)
+        e_ms = timed(e2e_step, args.steps)
+        dist_barrier(world)
+        e_ms = dist_max(world, e_ms)
+        e2e = {"value": round(total_flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e_ms / args.steps, 4)}
+
+    st, word = fa.fa_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(x, w)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (iid N(0,1), seeded, bf16 round-to-nearest-even)",
+        "config": {
+            "workload": "prefill B=4 H=16 N=2048 d=128; step = fwd (no mask) + fwd (causal) "
+                        "+ bwd (causal) + split-KV decode of one token per sequence over the "
+                        "step's K/V (cache length 2048)",
+            "B": B, "H": H, "N": N, "d": d, "step_gflop": round(step_flops / 1e9, 3),
+            "l2": "flushed between timed steps (256 MB write outside the timed events)",
+            "parallelism": f"replicas x{world} (independent heads, no collective)",
+        },
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "impl": "ours",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def cpu_baseline(x, w, heads=16):
+    """The fp64 oracle on a bounded sample: the step on `heads` heads of
+    batch entry 0 (fwd no mask, fwd causal, bwd causal, decode of the last
+    row), timed on the host cores."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import inputgen
+    import oracle
+    from exact_attention_130_b200 import counters as C
+
+    def f64(b):
+        return inputgen.bf16_bits_to_f32(b).astype(np.float64)
+
+    q, k, v, do = (f64(x[n][0, :heads]) for n in ("q", "k", "v", "do"))
+    t0 = time.perf_counter()
+    oracle.attention_fwd(q, k, v, w.scale, False)
+    oracle.attention_fwd(q, k, v, w.scale, True)
+    oracle.attention_bwd(q, k, v, do, w.scale, True)
+    oracle.decode(q[None, :, -1], k[None], v[None], np.array([w.N]), w.scale)
+    dt = time.perf_counter() - t0
+    fl = (C.fwd_flops(1, heads, w.N, w.d, False) + C.fwd_flops(1, heads, w.N, w.d, True)
+          + C.bwd_flops(1, heads, w.N, w.d, True) + C.decode_flops(heads, [w.N], w.d))
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": round(fl / dt / 1e12, 5), "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"the step on {heads} of {w.B * w.H} heads (batch entry 0), "
+                      f"fp64 numpy, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle as it stands, rank 0 only
+# ---------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import inputgen
+    import oracle
+    from exact_attention_130_b200 import counters as C
+
+    w = inputgen.WORKLOADS[WORKLOAD_NAME]
+    x = inputgen.make_attention_inputs(w, with_grad=True)
+
+    def f64(b):
+        return inputgen.bf16_bits_to_f32(b).astype(np.float64)
+
+    heads = 1  # one (batch, head) of the workload per step
+    def one(i):
+        b, h = divmod(i % (w.B * w.H), w.H)
+        q, k, v, do = (f64(x[n][b, h:h + heads]) for n in ("q", "k", "v", "do"))
+        oracle.attention_fwd(q, k, v, w.scale, False)
+        oracle.attention_fwd(q, k, v, w.scale, True)
+        oracle.attention_bwd(q, k, v, do, w.scale, True)
+        oracle.decode(q[None, :, -1], k[None], v[None], np.array([w.N]), w.scale)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(args.warmup + i)
+    dt = time.perf_counter() - t0
+    fl = (C.fwd_flops(1, heads, w.N, w.d, False) + C.fwd_flops(1, heads, w.N, w.d, True)
+          + C.bwd_flops(1, heads, w.N, w.d, True) + C.decode_flops(heads, [w.N], w.d))
+    value = fl * args.steps / dt / 1e12
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    sample = f"one (batch, head) of the prefill workload per step, fp64 numpy oracle"
+    line = {
+        "metric": METRIC, "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (iid N(0,1), seeded, bf16 round-to-nearest-even)",
+        "config": {"workload": "prefill B=4 H=16 N=2048 d=128; step = fwd (no mask) + fwd "
+                               "(causal) + bwd (causal) + decode, on a sample of one head",
+                   "B": w.B, "H": w.H, "N": w.N, "d": w.d},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -22,7 +22,7 @@ __all__ = [
     "fa_fwd", "fa_fwd_f32", "fa_bwd", "fa_bwd_workspace_size",
     "fa_decode_splitkv", "fa_decode_workspace_size", "fa_device_status",
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_abi_version",
-    "STATUS",
+    "fa_profile_begin", "fa_profile_end", "STATUS", "KERNEL_NAMES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -65,7 +65,12 @@ _SIGNATURES = {
     "fa_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "fa_set_wait_limit": (None, [ctypes.c_ulonglong]),
     "fa_debug_skip_load": (None, [_I]),
+    "fa_profile_begin": (None, []),
+    "fa_profile_end": (_I, [ctypes.POINTER(_I), ctypes.POINTER(ctypes.c_double), _I]),
 }
+
+KERNEL_NAMES = {1: "fwd", 2: "fwd_f32", 3: "bwd_pre", 4: "bwd_main", 5: "bwd_post",
+                6: "decode_split", 7: "decode_merge"}
 
 
 def load_library():
@@ -240,3 +245,18 @@ def fa_set_wait_limit(nanoseconds: int):
 
 def fa_debug_skip_load(enable: bool):
     load_library().fa_debug_skip_load(int(bool(enable)))
+
+
+def fa_profile_begin():
+    load_library().fa_profile_begin()
+
+
+def fa_profile_end():
+    """Stop per-kernel timing; return {kernel name: (launches, total ms)}."""
+    lib = load_library()
+    launches = (ctypes.c_int * 8)()
+    total = (ctypes.c_double * 8)()
+    rc = lib.fa_profile_end(launches, total, 8)
+    if rc < 0:
+        raise FAError(5, "fa_profile_end: a CUDA event call failed")
+    return {KERNEL_NAMES[k]: (launches[k], total[k]) for k in KERNEL_NAMES if launches[k]}

@@ -281,11 +281,17 @@ fa_status launch(const DecParams& p, int B, const LaunchCtx& ctx) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   dim3 g1(p.C, p.H, B);
-  decode_split_kernel<D><<<g1, kThreads, smem, ctx.stream>>>(p);
+  {
+    ProfileScope prof(KID_DECODE, ctx.stream);
+    decode_split_kernel<D><<<g1, kThreads, smem, ctx.stream>>>(p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode split kernel launch");
   dim3 g2(p.H, B);
-  decode_merge_kernel<D><<<g2, D, 0, ctx.stream>>>(p);
+  {
+    ProfileScope prof(KID_DECODE_MERGE, ctx.stream);
+    decode_merge_kernel<D><<<g2, D, 0, ctx.stream>>>(p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode merge kernel launch");
   return FA_OK;

@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "fa_internal.h"
 
@@ -119,7 +120,40 @@ fa_status check_ptrs(std::initializer_list<const void*> ptrs, const char* names)
   return FA_OK;
 }
 
+struct ProfRecord {
+  unsigned int kid;
+  cudaEvent_t start, stop;
+};
+std::atomic<bool> g_prof_on{false};
+std::mutex g_prof_mu;
+std::vector<ProfRecord> g_prof;
+
 }  // namespace
+
+ProfileScope::ProfileScope(unsigned int kernel_id, cudaStream_t stream)
+    : kid_(kernel_id), stream_(stream) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  if (cudaEventCreate(&start_) != cudaSuccess) {
+    start_ = nullptr;
+    return;
+  }
+  if (cudaEventRecord(start_, stream_) != cudaSuccess) {
+    cudaEventDestroy(start_);
+    start_ = nullptr;
+  }
+}
+
+ProfileScope::~ProfileScope() {
+  if (!start_) return;
+  cudaEvent_t stop = nullptr;
+  if (cudaEventCreate(&stop) != cudaSuccess || cudaEventRecord(stop, stream_) != cudaSuccess) {
+    if (stop) cudaEventDestroy(stop);
+    cudaEventDestroy(start_);
+    return;
+  }
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof.push_back({kid_, start_, stop});
+}
 
 void set_last_error(const char* fmt, ...) {
   va_list ap;
@@ -280,6 +314,40 @@ fa_status fa_decode_splitkv(const void* q, const void* kcache, const void* vcach
   if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
   return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Lmax, d, scale, chunks,
                        workspace, ctx);
+}
+
+void fa_profile_begin(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) {
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  g_prof.clear();
+  g_prof_on.store(true);
+}
+
+int fa_profile_end(int* launches, double* total_ms, int capacity) {
+  g_prof_on.store(false);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (int k = 0; k < capacity; ++k) {
+    if (launches) launches[k] = 0;
+    if (total_ms) total_ms[k] = 0.0;
+  }
+  int rc = 8;
+  for (auto& r : g_prof) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess)
+      rc = -1;
+    if (int(r.kid) < capacity) {
+      if (launches) launches[r.kid] += 1;
+      if (total_ms) total_ms[r.kid] += ms;
+    }
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  g_prof.clear();
+  return rc;
 }
 
 fa_status fa_device_status(cudaStream_t stream, unsigned int* detail) {

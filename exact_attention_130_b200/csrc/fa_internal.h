@@ -30,6 +30,21 @@ enum KernelId : unsigned int {
   KID_DECODE_MERGE = 7,
 };
 
+// Brackets one kernel launch with CUDA events when profiling is on
+// (fa_profile_begin); no-op otherwise.
+class ProfileScope {
+ public:
+  ProfileScope(unsigned int kernel_id, cudaStream_t stream);
+  ~ProfileScope();
+  ProfileScope(const ProfileScope&) = delete;
+  ProfileScope& operator=(const ProfileScope&) = delete;
+
+ private:
+  unsigned int kid_;
+  cudaStream_t stream_;
+  cudaEvent_t start_ = nullptr;
+};
+
 // Records a message for fa_last_error() on this thread.
 void set_last_error(const char* fmt, ...);
 fa_status cuda_fail(cudaError_t e, const char* what);

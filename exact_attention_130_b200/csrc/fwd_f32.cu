@@ -103,8 +103,11 @@ template <int D, bool CAUSAL>
 fa_status launch(const float* q, const float* k, const float* v, float* o, float* lse, int BH,
                  int N, float scale, const LaunchCtx& ctx) {
   dim3 grid((N + kRows - 1) / kRows, BH);
-  fwd_f32_kernel<D, CAUSAL><<<grid, kThreads, 0, ctx.stream>>>(q, k, v, o, lse, N,
-                                                                scale * 1.4426950408889634f);
+  {
+    ProfileScope prof(KID_FWD_F32, ctx.stream);
+    fwd_f32_kernel<D, CAUSAL><<<grid, kThreads, 0, ctx.stream>>>(q, k, v, o, lse, N,
+                                                                  scale * 1.4426950408889634f);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd_f32 kernel launch");
   return FA_OK;

@@ -432,7 +432,10 @@ fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fwd)");
   const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
-  kern<<<grid, kThreads, smem, ctx.stream>>>(mq, mk, mv, p);
+  {
+    ProfileScope prof(KID_FWD, ctx.stream);
+    kern<<<grid, kThreads, smem, ctx.stream>>>(mq, mk, mv, p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
   return FA_OK;

@@ -100,8 +100,9 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o,
 
 /*
  * fa_bwd_workspace_size -- bytes of scratch fa_bwd needs: an fp32 dQ
- * accumulator [B, H, N, d] and the fp32 vector D [B, H, N], each padded to
- * 256 bytes.
+ * accumulator [B, H, N, d], then two fp32 vectors [B, H, Np] (the saved LSE
+ * in base 2, and D = rowsum(dO * O)), Np = N rounded up to a multiple of
+ * 128; each part starts on a 256-byte boundary. Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -179,6 +180,21 @@ void fa_set_wait_limit(unsigned long long nanoseconds);
  * to 0 by that launch.
  */
 void fa_debug_skip_load(int enable);
+
+/*
+ * Per-kernel timing, off by default. Between fa_profile_begin() and
+ * fa_profile_end() every kernel this library launches is bracketed by a pair
+ * of CUDA events recorded on its launching stream. fa_profile_end()
+ * synchronises those events, stops recording and writes, for each kernel id
+ * k in [0, capacity), the number of launches (launches[k]) and their summed
+ * device time in milliseconds (total_ms[k]). Kernel ids: 1 forward (bf16),
+ * 2 forward (fp32), 3 backward preprocess, 4 backward main, 5 backward dQ
+ * conversion, 6 decode split, 7 decode merge. Returns the number of ids
+ * (8), or -1 if a CUDA call failed. Not thread-safe against concurrent
+ * begin/end pairs; launches from several threads are recorded.
+ */
+void fa_profile_begin(void);
+int fa_profile_end(int* launches, double* total_ms, int capacity);
 
 #ifdef __cplusplus
 }

@@ -20,7 +20,8 @@ import re
 __all__ = [
     "FAError", "library_path", "load_library", "exported_symbols",
     "fa_fwd", "fa_fwd_f32", "fa_bwd", "fa_bwd_workspace_size",
-    "fa_decode_splitkv", "fa_decode_workspace_size", "fa_device_status",
+    "fa_decode_splitkv", "fa_decode_workspace_size", "fa_decode_splitkv_static",
+    "fa_device_status",
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_abi_version",
     "fa_profile_begin", "fa_profile_end", "STATUS", "KERNEL_NAMES",
 ]
@@ -62,6 +63,7 @@ _SIGNATURES = {
     "fa_decode_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I,
                                _P, _S, _P]),
+    "fa_decode_splitkv_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "fa_set_wait_limit": (None, [ctypes.c_ulonglong]),
     "fa_debug_skip_load": (None, [_I]),
@@ -228,6 +230,29 @@ def fa_decode_splitkv(q, kcache, vcache, seqlens, scale: float | None = None,
                                  _ptr(o), _ptr(lse), B, H, Lmax, d, scale,
                                  num_splits, _ptr(workspace), workspace.numel(),
                                  _stream(stream)))
+    return o, lse
+
+
+def fa_decode_splitkv_static(q, kcache, vcache, seqlens, scale: float | None = None,
+                             num_splits: int = 0, o=None, lse=None, stream=None):
+    """fa_decode_splitkv with the partials in the library's own 8 MiB device
+    buffer: for callers that cannot allocate device memory while decoding.
+    Calls that may overlap on the GPU share that buffer and must be
+    serialised by the caller."""
+    import torch
+    lib = load_library()
+    _need(q, torch.bfloat16, "q")
+    _need(kcache, torch.bfloat16, "kcache")
+    _need(vcache, torch.bfloat16, "vcache")
+    _need(seqlens, torch.int32, "seqlens")
+    B, H, d = q.shape
+    Lmax = kcache.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(lib.fa_decode_splitkv_static(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens),
+                                        _ptr(o), _ptr(lse), B, H, Lmax, d, scale,
+                                        num_splits, _stream(stream)))
     return o, lse
 
 

@@ -26,6 +26,8 @@
 //    per token;
 //  * positions at or past seqlens[b] are never read;
 //  * all waits are bounded in time (see sm100_ptx.cuh).
+#include <mutex>
+
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -348,3 +350,87 @@ fa_status launch_decode(const void* q, const void* kcache, const void* vcache, c
 }
 
 }  // namespace fa
+
+// ---------------------------------------------------------------------------
+// Decode without any device allocation.
+//
+// fa_decode_splitkv needs a caller-provided workspace for the per-chunk
+// partial results. Some callers cannot allocate device memory at the moment
+// they decode: code running inside a stream capture, code driven by an
+// allocator that forbids cudaMalloc on the hot path, or a host that owns no
+// memory pool of its own. For them the partials live in the fixed buffer
+// below, which is part of the library image: every GPU that loads the
+// library reserves kStaticScratchBytes of device memory for it until the
+// process exits. Nothing here calls cudaMalloc, cudaFree or any allocating
+// routine.
+// ---------------------------------------------------------------------------
+namespace fa {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+void* g_scratch_ptr[kMaxScratchDevices] = {};  // device address per device
+std::mutex g_scratch_mu;
+
+}  // namespace
+}  // namespace fa
+
+extern "C" fa_status fa_decode_splitkv_static(const void* q, const void* kcache,
+                                              const void* vcache, const int* seqlens, void* o,
+                                              float* lse, int B, int H, int Lmax, int d,
+                                              float scale, int num_splits, cudaStream_t stream) {
+  using namespace fa;
+  auto bad = [](fa_status st, const char* msg) {
+    set_last_error("fa_decode_splitkv_static: %s", msg);
+    return st;
+  };
+  const void* ptrs[5] = {q, kcache, vcache, o, lse};
+  for (const void* ptr : ptrs) {
+    if (ptr == nullptr) return bad(FA_ERR_INVALID_ARG, "null tensor pointer");
+    if (reinterpret_cast<uintptr_t>(ptr) & 15u)
+      return bad(FA_ERR_ALIGNMENT, "a tensor pointer is not 16-byte aligned");
+  }
+  if (seqlens == nullptr || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return bad(FA_ERR_INVALID_ARG, "seqlens must be a non-null, 4-byte aligned int32 array");
+  if (B < 1 || H < 1 || Lmax < 1 || (long long)B * H * Lmax > 0x7fffffffLL)
+    return bad(FA_ERR_INVALID_ARG, "B, H, Lmax must be >= 1 with B*H*Lmax < 2^31");
+  if (d != 64 && d != 128) return bad(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+  if (!(scale > 0.f) || scale == INFINITY) return bad(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (num_splits < 0 || num_splits > 1024)
+    return bad(FA_ERR_INVALID_ARG, "num_splits must be in [0, 1024]");
+  const int chunks = decode_num_chunks(B, H, Lmax, num_splits, 0);
+  const size_t need = decode_workspace_bytes(B, H, d, chunks);
+  if (need > kStaticScratchBytes) {
+    set_last_error(
+        "fa_decode_splitkv_static: this shape needs %zu bytes of scratch, more than the %zu "
+        "bytes built into the library; call fa_decode_splitkv with a workspace instead",
+        need, kStaticScratchBytes);
+    return FA_ERR_WORKSPACE;
+  }
+  LaunchCtx ctx;
+  fa_status st = current_launch_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxScratchDevices) return bad(FA_ERR_UNSUPPORTED, "device index too large");
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+      // once per device, with that device current: the host-side name of the
+      // array is only a stand-in, the kernel needs its device address
+      void* addr = nullptr;
+      e = cudaGetSymbolAddress(&addr, g_decode_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static decode scratch)");
+      g_scratch_ptr[dev] = addr;
+    }
+    scratch = g_scratch_ptr[dev];
+  }
+  // every chunk writes its own partial (empty chunks write weight 0), so no
+  // part of the scratch has to start at zero
+  return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Lmax, d, scale, chunks, scratch,
+                       ctx);
+}

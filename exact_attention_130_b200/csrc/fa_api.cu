@@ -168,6 +168,10 @@ fa_status cuda_fail(cudaError_t e, const char* what) {
   return FA_ERR_CUDA;
 }
 
+fa_status current_launch_ctx(cudaStream_t stream, LaunchCtx* ctx) {
+  return device_ctx(stream, ctx);
+}
+
 fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t inner,
                        uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows,
                        bool swizzle128) {

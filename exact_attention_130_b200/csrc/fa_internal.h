@@ -45,6 +45,10 @@ class ProfileScope {
   cudaEvent_t start_ = nullptr;
 };
 
+// Launch context of the current device (SM count, status word, wait limit),
+// setting the device up on first use.
+fa_status current_launch_ctx(cudaStream_t stream, LaunchCtx* ctx);
+
 // Records a message for fa_last_error() on this thread.
 void set_last_error(const char* fmt, ...);
 fa_status cuda_fail(cudaError_t e, const char* what);

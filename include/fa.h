@@ -158,6 +158,33 @@ fa_status fa_decode_splitkv(const void* q, const void* kcache,
                             size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * fa_decode_splitkv_static -- fa_decode_splitkv for callers that cannot
+ * allocate device memory when they decode (inside a stream capture, under an
+ * allocator that forbids cudaMalloc on the hot path, or with no memory pool
+ * of their own). No counterpart on the pages: it is the same computation,
+ * with the per-chunk partials kept in an 8 MiB buffer that is part of the
+ * library image instead of a caller workspace. Arguments as for
+ * fa_decode_splitkv, minus the workspace.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *    Every GPU that loads the library holds the 8 MiB until the process
+ *    exits.
+ *  - The first call on each device looks up the buffer's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Shapes whose partials exceed 8 MiB (B * H * C * (d + 1) * 4 bytes, C the
+ *    chunk count) are rejected with FA_ERR_WORKSPACE and a message saying so.
+ *  - All calls share the one buffer, which keeps the last call's contents;
+ *    nothing in it needs to start at zero. Calls that can overlap on the GPU
+ *    (different streams without ordering between them) race on it and give
+ *    wrong results: serialise them.
+ */
+fa_status fa_decode_splitkv_static(const void* q, const void* kcache,
+                                   const void* vcache, const int* seqlens,
+                                   void* o, float* lse, int B, int H, int Lmax,
+                                   int d, float scale, int num_splits,
+                                   cudaStream_t stream);
+
+/*
  * fa_device_status -- synchronises `stream`, reads and clears the current
  * device's status word. Returns FA_ERR_TIMEOUT if any kernel of this
  * library gave up a wait since the last check, FA_ERR_CUDA if the

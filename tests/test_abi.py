@@ -12,7 +12,7 @@ EXPECTED = {
     "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd",
     "fa_decode_workspace_size", "fa_decode_splitkv", "fa_device_status",
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_profile_begin",
-    "fa_profile_end",
+    "fa_profile_end", "fa_decode_splitkv_static",
 }
 
 

@@ -189,7 +189,7 @@ def load_peaks():
 
 
 def kernel_source_hash(name: str) -> str:
-    files = {"fwd": "fwd_sm100.cu", "bwd_main": "bwd_sm100.cu",
+    files = {"fwd": "fwd_sm100.cu", "bwd_dkdv": "bwd_sm100.cu", "bwd_dq": "bwd_sm100.cu",
              "decode_split": "decode_sm100.cu"}
     path = os.path.join(ROOT, "exact_attention_130_b200", "csrc", files.get(name, ""))
     try:
@@ -202,7 +202,8 @@ def kernel_source_hash(name: str) -> str:
 # profiles/traffic.json when a capture of exactly that launch is recorded
 BENCH_LAUNCH = {
     "fwd": "bench step: fwd B=4 H=16 N=2048 d=128 (mean of no mask and causal)",
-    "bwd_main": "bench step: bwd causal B=4 H=16 N=2048 d=128",
+    "bwd_dkdv": "bench step: bwd causal B=4 H=16 N=2048 d=128",
+    "bwd_dq": "bench step: bwd causal B=4 H=16 N=2048 d=128",
     "decode_split": "bench step: decode B=4 H=16 cache 2048 d=128",
 }
 
@@ -262,13 +263,21 @@ def run_ours(args, world, rank, local):
                              lse=out["lse_dec"], workspace=ws_dec)
 
     src_dev = dict(dev, qdec=qdec)
-    launches_per_step = 1 + 1 + 3 + 2
+    launches_per_step = 1 + 1 + 3 + 2  # fwd, fwd, bwd (pre, dK/dV, dQ), decode (split, merge)
+    # FLOPs by the measurement's convention (the headline): forward 4 B H N^2 d
+    # (halved under the causal mask), backward 2.5x the causal forward
+    step_flops = (C.fwd_flops(B, H, N, d, False) + C.fwd_flops(B, H, N, d, True)
+                  + C.bwd_flops(B, H, N, d, True) + C.decode_flops(H, [N] * B, d))
+    # tensor-core work each kernel actually performs per step (for the per-kernel
+    # rates): the dK/dV kernel runs S^T, dP^T, dV, dK (2x the causal forward),
+    # the dQ kernel S, dP, dQ (1.5x)
+    fc = C.fwd_flops(B, H, N, d, True)
     flops = {
-        "fwd": C.fwd_flops(B, H, N, d, False) + C.fwd_flops(B, H, N, d, True),
-        "bwd_main": C.bwd_flops(B, H, N, d, True),
+        "fwd": C.fwd_flops(B, H, N, d, False) + fc,
+        "bwd_dkdv": 2.0 * fc,
+        "bwd_dq": 1.5 * fc,
         "decode_split": C.decode_flops(H, [N] * B, d),
     }
-    step_flops = sum(flops.values())
     dec_bytes = C.decode_bytes(H, [N] * B, d)
 
     def timed(fn, k):
@@ -312,7 +321,7 @@ def run_ours(args, world, rank, local):
     for name, (n, tot) in prof.items():
         avg = tot / n
         entry = {"launches": n, "avg_ms": round(avg, 5)}
-        if name in ("fwd", "bwd_main"):
+        if name in ("fwd", "bwd_dkdv", "bwd_dq"):
             tf = flops[name] * args.steps / (tot * 1e-3) / 1e12
             entry.update({"tflops": round(tf, 1), "frac_of_tensor_peak": round(tf / peaks["bf16_tflops"], 4)})
         elif name == "decode_split":
@@ -321,10 +330,10 @@ def run_ours(args, world, rank, local):
         kernels[name] = entry
     dominant = max(prof, key=lambda k: prof[k][1])
     dn, dtot = prof[dominant]
-    # algorithmic work of one launch: the forward runs twice per step (no mask,
-    # causal), the backward main kernel once
+    # work of one launch: the forward runs twice per step (no mask, causal), the
+    # backward kernels once
     per_launch_flops = flops["fwd"] / 2 if dominant == "fwd" else flops.get(dominant, 0.0)
-    if dominant in ("fwd", "bwd_main"):
+    if dominant in ("fwd", "bwd_dkdv", "bwd_dq"):
         achieved = flops[dominant] * args.steps / (dtot * 1e-3) / 1e12
         roofline = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 1),
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",

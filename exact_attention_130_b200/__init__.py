@@ -71,7 +71,7 @@ _SIGNATURES = {
     "fa_profile_end": (_I, [ctypes.POINTER(_I), ctypes.POINTER(ctypes.c_double), _I]),
 }
 
-KERNEL_NAMES = {1: "fwd", 2: "fwd_f32", 3: "bwd_pre", 4: "bwd_main", 5: "bwd_post",
+KERNEL_NAMES = {1: "fwd", 2: "fwd_f32", 3: "bwd_pre", 4: "bwd_dkdv", 5: "bwd_dq",
                 6: "decode_split", 7: "decode_merge"}
 
 

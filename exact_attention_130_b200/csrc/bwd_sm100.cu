@@ -5,86 +5,64 @@
 // every block of P on chip as P = exp(S - L) and forms
 //     dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D),
 //     dQ = scale * dS K,  dK = scale * dS^T Q,
-// so neither S nor P is ever stored.
+// so neither S nor P (nor dS) is ever stored.
 //
 // Three kernels on the caller's stream:
-//  1. bwd_pre   D_i = sum_c dO_ic O_ic (fp32), the saved LSE converted to
-//               base 2, both padded to a multiple of 128 rows (padding rows get
-//               LSE = +inf, so their P is exactly 0), and the fp32 dQ
-//               accumulator zeroed.
-//  2. bwd_main  one CTA per (batch*head, 128-key tile); the K and V tiles stay
-//               in shared memory while the Q and dO tiles of every query tile
-//               that can see these keys stream past (under the causal mask,
-//               query tiles below the diagonal only). Per query tile:
-//                 S^T  = K Q^T      (tcgen05, TMEM)
-//                 dP^T = V dO^T     (tcgen05, TMEM)
-//                 P^T  = 2^(S^T scale log2e - L2), dS^T = scale P^T (dP^T - D)
-//                        (one TMEM lane = one key row; P^T goes back to TMEM
-//                        as bf16, dS^T to shared memory in the 128-byte
-//                        swizzled layout)
-//                 dV  += P^T dO     (A from TMEM)
-//                 dK  += dS^T Q     (A = dS^T, K-major)
-//                 dQ_i = dS K       (A = the same dS^T buffer read MN-major)
-//               dV and dK accumulate in TMEM for the whole key tile; dQ_i is
-//               added into the fp32 accumulator with vector atomics by four
-//               dedicated warps.
-//  3. bwd_post  dQ = bf16(accumulator).
-// The scale is folded into dS before it is rounded to bf16, so dK and dQ need
-// no further scaling.
+//  1. bwd_pre   D_i = sum_c dO_ic O_ic (fp32) and the saved LSE in base 2, both
+//               padded to a multiple of 128 rows (padding rows get LSE = +inf,
+//               so their P is exactly 0).
+//  2. bwd_dkdv  one CTA per (batch*head, 128-key tile). K and V of the tile stay
+//               in shared memory; the Q and dO rows of every query that can see
+//               these keys stream past in blocks of 64. Per block:
+//                 S^T = K Q^T, dP^T = V dO^T          (tcgen05 -> TMEM)
+//                 P^T = 2^(S^T scale log2e - L2),
+//                 dS^T = scale P^T (dP^T - D)        (CUDA cores, one TMEM lane
+//                                                      = one key row)
+//                 dV += P^T dO, dK += dS^T Q          (tcgen05, A from TMEM)
+//               dV and dK accumulate in TMEM for the whole key tile.
+//  3. bwd_dq    one CTA per (batch*head, 128-query tile). Q and dO stay in shared
+//               memory; K and V stream past in blocks of 64 keys. Per block:
+//                 S = Q K^T, dP = dO V^T; dS = scale P (dP - D); dQ += dS K.
+// The scale is folded into dS before it is rounded to bf16.
 //
-// Warp roles of bwd_main (320 threads):
-//   warps 0-3  compute (exp, dS) and the dK/dV epilogue
-//   warp  4    TMA producer        warp 5  MMA issuer
-//   warps 6-9  dQ readers (TMEM -> atomics into the accumulator)
-// TMEM: S^T | dP^T (later dQ_i) | dV | dK = 512 columns at d = 128.
+// Splitting dQ from dK/dV recomputes S and dP once more (7 tensor-core GEMMs
+// instead of 5) but needs no atomics and keeps the tensor core busy: in both
+// kernels two compute warpgroups take alternate 64-wide blocks, each with its
+// own S/dP buffer in TMEM, so the exponentials of one block overlap the MMAs of
+// the other (TMEM: buffer 0 | buffer 1 | two 128-column accumulators).
+//
+// Warp roles (320 threads): warps 0-3 compute for buffer 0, warps 4-7 for
+// buffer 1, warp 8 TMA producer, warp 9 MMA issuer.
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace fa {
 namespace {
 
-constexpr int kBlk = 128;  // keys per CTA and queries per step
+constexpr int kTile = 128;   // rows of the resident tile (keys or queries)
+constexpr int kSub = 64;     // rows of a streamed block
 constexpr int kThreads = 320;
-constexpr int kLoadWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kStages = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// barrier slots (shared by both kernels)
 enum : int {
-  B_KV_FULL = 0,
-  B_Q_FULL = 1,    // +stage (2)
-  B_Q_EMPTY = 3,   // +stage (2)
-  B_S_FULL = 5,
-  B_DP_FULL = 6,
-  B_P_READY = 7,
-  B_DQ_FULL = 8,
-  B_DQ_EMPTY = 9,
-  B_ACC_DONE = 10,
-  B_DRAIN = 11,
-  B_COUNT = 12
-};
-
-template <int D>
-struct BwdLayout {
-  static constexpr int kSub = D / 64;
-  static constexpr int kSubBytes = 128 * 128;
-  static constexpr int kTileBytes = kSub * kSubBytes;  // 128 rows x D bf16
-  static constexpr int kStages = 2;
-  static constexpr int kOffK = 0;
-  static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffQ = 2 * kTileBytes;                       // + s * tile
-  static constexpr int kOffDO = kOffQ + kStages * kTileBytes;        // + s * tile
-  static constexpr int kOffDS = kOffDO + kStages * kTileBytes;       // 128 x 128 bf16
-  static constexpr int kOffBar = kOffDS + 2 * kSubBytes;
-  static constexpr int kOffMisc = kOffBar + 8 * B_COUNT;
-  static constexpr int kSmemBytes = kOffMisc + 32 + 1024;
-  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  B_RES_FULL = 0,      // the resident tiles (K,V or Q,dO)
+  B_ST_FULL = 1,       // +stage: a streamed block landed
+  B_ST_EMPTY = 5,      // +stage: its MMAs are done
+  B_S_FULL = 9,        // +buffer: S and dP of a block are in TMEM
+  B_P_READY = 11,      // +buffer: P / dS written back to TMEM
+  B_ACC_DONE = 13,
+  B_DRAIN = 14,
+  B_COUNT = 15
 };
 
 struct BwdParams {
   const uint16_t* o;
   const uint16_t* dO;
   const float* lse;
-  float* dq_acc;   // [BH, N, D] fp32
   float* lse2;     // [BH, Np] base-2 LSE, +inf in padding rows
   float* dvec;     // [BH, Np] D, 0 in padding rows
   uint16_t* dq;
@@ -98,18 +76,42 @@ struct BwdParams {
 
 __device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
+// Shared-memory plan. Row-major tiles of bf16 with 128-byte rows, stored as
+// D/64 column groups of rows x 128 bytes, 128-byte swizzled (TMA box 64
+// columns x rows).
+template <int D>
+struct Plan {
+  static constexpr int kGroups = D / 64;
+  static constexpr int kResSub = kTile * 128;            // 16 KB per column group
+  static constexpr int kResTile = kGroups * kResSub;      // one resident tile
+  static constexpr int kBlkSub = kSub * 128;              // 8 KB per column group
+  static constexpr int kBlkTile = kGroups * kBlkSub;      // one streamed tile
+  static constexpr int kOffRes0 = 0;
+  static constexpr int kOffRes1 = kResTile;
+  static constexpr int kOffStage = 2 * kResTile;
+  // a stage: two streamed tiles, then (dK/dV kernel) 64 floats of L2 and of D
+  static constexpr int kStageBytes = ((2 * kBlkTile + 512) + 1023) / 1024 * 1024;
+  static constexpr int kOffBar = kOffStage + kStages * kStageBytes;
+  static constexpr int kOffMisc = kOffBar + 8 * B_COUNT;
+  static constexpr int kSmemBytes = kOffMisc + 32 + 1024;
+  // TMEM columns: buffer b holds S (64 columns) then dP (64 columns)
+  static constexpr uint32_t kColAcc0 = 256, kColAcc1 = 256 + D;
+  __device__ static constexpr uint32_t col_s(int b) { return b ? 128u : 0u; }
+  __device__ static constexpr uint32_t col_dp(int b) { return b ? 192u : 64u; }
+};
+
 // --------------------------------------------------------------------------
-// 1. preprocess: one warp per row
+// 1. preprocess: one warp per (padded) row
 // --------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   constexpr int kPer = D / 32;
-  const int warp = (blockIdx.x * 256 + threadIdx.x) >> 5;
+  const long long warp = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const long long total = (long long)p.BH * p.Np;
+  const long long total = static_cast<long long>(p.BH) * p.Np;
   if (warp >= total) return;
-  const int bh = warp / p.Np;
-  const int row = warp % p.Np;
+  const int bh = int(warp / p.Np);
+  const int row = int(warp % p.Np);
   float dsum = 0.f;
   if (row < p.N) {
     const size_t base = (size_t(bh) * p.N + row) * D + lane * kPer;
@@ -118,12 +120,10 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
       const uint2 b = *reinterpret_cast<const uint2*>(p.dO + base);
       dsum = bf16f(a.x & 0xffffu) * bf16f(b.x & 0xffffu) + bf16f(a.x >> 16) * bf16f(b.x >> 16) +
              bf16f(a.y & 0xffffu) * bf16f(b.y & 0xffffu) + bf16f(a.y >> 16) * bf16f(b.y >> 16);
-      *reinterpret_cast<float4*>(p.dq_acc + base) = make_float4(0.f, 0.f, 0.f, 0.f);
     } else {
       const uint32_t a = *reinterpret_cast<const uint32_t*>(p.o + base);
       const uint32_t b = *reinterpret_cast<const uint32_t*>(p.dO + base);
       dsum = bf16f(a & 0xffffu) * bf16f(b & 0xffffu) + bf16f(a >> 16) * bf16f(b >> 16);
-      *reinterpret_cast<float2*>(p.dq_acc + base) = make_float2(0.f, 0.f);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
@@ -135,44 +135,26 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   }
 }
 
-// --------------------------------------------------------------------------
-// 2. main kernel
-// --------------------------------------------------------------------------
-template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const BwdParams p) {
-  using L = BwdLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// Common prologue of both main kernels: barriers, TMEM, abort flag.
+template <int D>
+__device__ __forceinline__ uint32_t setup_cta(uint8_t* smem, int warp, volatile int*& abort_flag) {
+  using L = Plan<D>;
   const uint32_t sbase = smem_u32(smem);
-  auto BAR = [&](int i) -> uint32_t { return sbase + L::kOffBar + 8u * uint32_t(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // key tiles with the most query tiles first (under the causal mask the
-  // lowest key tiles see every query tile), every head of a level together
-  const int jt = blockIdx.x / p.BH;  // key tile
-  const int bh = blockIdx.x % p.BH;
-  const int i0 = CAUSAL ? jt : 0;
-  const int n_it = p.n_tiles - i0;
-
+  abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   if (threadIdx.x == 0) {
-    mbar_init(BAR(B_KV_FULL), 1);
-    for (int s = 0; s < L::kStages; ++s) {
-      mbar_init(BAR(B_Q_FULL + s), 1);
-      mbar_init(BAR(B_Q_EMPTY + s), 1);
+    auto bar = [&](int i) { return sbase + L::kOffBar + 8u * i; };
+    mbar_init(bar(B_RES_FULL), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(B_ST_FULL + s), 1);
+      mbar_init(bar(B_ST_EMPTY + s), 1);
     }
-    mbar_init(BAR(B_S_FULL), 1);
-    mbar_init(BAR(B_DP_FULL), 1);
-    mbar_init(BAR(B_P_READY), 4);
-    mbar_init(BAR(B_DQ_FULL), 1);
-    mbar_init(BAR(B_DQ_EMPTY), 4);
-    mbar_init(BAR(B_ACC_DONE), 1);
-    mbar_init(BAR(B_DRAIN), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(B_S_FULL + b), 1);
+      mbar_init(bar(B_P_READY + b), 4);
+    }
+    mbar_init(bar(B_ACC_DONE), 1);
+    mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -183,246 +165,215 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  return *tmem_slot;
+}
+
+// MMA of one streamed block against a resident tile, both K-major operands:
+// D[128 x 64] = R[128 x D] * B[64 x D]^T
+template <int D>
+__device__ __forceinline__ void mma_rows_x_block(uint32_t d_tmem, uint32_t res, uint32_t blk) {
+  using L = Plan<D>;
+  constexpr uint32_t idesc = idesc_bf16(kTile, kSub, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t ra = res + (kk >> 2) * L::kResSub + (kk & 3) * 32;
+    const uint32_t rb = blk + (kk >> 2) * L::kBlkSub + (kk & 3) * 32;
+    mma_ss(d_tmem, sdesc_sw128(ra, 16, 1024), sdesc_sw128(rb, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// Accumulating MMA with A (128 x 64, bf16) in TMEM and B a streamed block of
+// 64 rows x D read MN-major: D[128 x D] += A * B
+template <int D>
+__device__ __forceinline__ void mma_tmem_x_block(uint32_t d_tmem, uint32_t a_tmem, uint32_t blk,
+                                                 bool accumulate) {
+  using L = Plan<D>;
+  constexpr uint32_t idesc = idesc_bf16(kTile, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < kSub / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(blk + kk * 2048, L::kBlkSub, 1024), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// bf16 row of a TMEM accumulator (this thread's lane) -> global
+template <int D>
+__device__ __forceinline__ void store_acc_row(uint32_t t_acc, uint16_t* dst, bool valid) {
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t v[32];
+    tmem_ld32_wait(t_acc + ch * 32, v);
+    if (valid) {
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(v[8 * v4 + 0]), __uint_as_float(v[8 * v4 + 1]));
+        w.y = pack_bf16x2(__uint_as_float(v[8 * v4 + 2]), __uint_as_float(v[8 * v4 + 3]));
+        w.z = pack_bf16x2(__uint_as_float(v[8 * v4 + 4]), __uint_as_float(v[8 * v4 + 5]));
+        w.w = pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7]));
+        *reinterpret_cast<uint4*>(dst + ch * 32 + 8 * v4) = w;
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// 2. dK, dV: key-tile-outer
+// --------------------------------------------------------------------------
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ64, const __grid_constant__ CUtensorMap tmDO64,
+                    const __grid_constant__ CUtensorMap tmK128, const __grid_constant__ CUtensorMap tmV128,
+                    const BwdParams p) {
+  using L = Plan<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + L::kOffBar + 8u * uint32_t(i); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // key tiles that see the most query blocks first, all heads of a level together
+  const int jt = blockIdx.x / p.BH;
+  const int bh = blockIdx.x % p.BH;
+  const int q_start = CAUSAL ? jt * kTile : 0;
+  const int n_blk = (p.N - q_start + kSub - 1) / kSub;
+  volatile int* abort_flag;
+  const uint32_t tmem = setup_cta<D>(smem, warp, abort_flag);
   const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_BWD};
+  const uint32_t sK = sbase + L::kOffRes0, sV = sbase + L::kOffRes1;
 
   if (warp == kLoadWarp) {
-    // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int q_cnt[2] = {0, 0};
-      mbar_arrive_expect_tx(BAR(B_KV_FULL), 2 * L::kTileBytes);
-      for (int c = 0; c < L::kSub; ++c) {
-        tma_load_3d(sbase + L::kOffK + c * L::kSubBytes, &tmK, BAR(B_KV_FULL), c * 64, jt * kBlk, bh);
-        tma_load_3d(sbase + L::kOffV + c * L::kSubBytes, &tmV, BAR(B_KV_FULL), c * 64, jt * kBlk, bh);
+      int cnt[kStages] = {0, 0, 0, 0};
+      mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kResTile);
+      for (int c = 0; c < L::kGroups; ++c) {
+        tma_load_3d(sK + c * L::kResSub, &tmK128, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
+        tma_load_3d(sV + c * L::kResSub, &tmV128, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
       }
-      for (int it = 0; it < n_it; ++it) {
-        const int s = it & 1;
-        if (!wait_bounded(BAR(B_Q_EMPTY + s), ((it >> 1) & 1) ^ 1, wc, 1)) break;
-        const int i = i0 + it;
-        mbar_arrive_expect_tx(BAR(B_Q_FULL + s), 2 * L::kTileBytes);
-        for (int c = 0; c < L::kSub; ++c) {
-          tma_load_3d(sbase + L::kOffQ + s * L::kTileBytes + c * L::kSubBytes, &tmQ,
-                      BAR(B_Q_FULL + s), c * 64, i * kBlk, bh);
-          tma_load_3d(sbase + L::kOffDO + s * L::kTileBytes + c * L::kSubBytes, &tmDO,
-                      BAR(B_Q_FULL + s), c * 64, i * kBlk, bh);
+      for (int it = 0; it < n_blk; ++it) {
+        const int s = it % kStages;
+        if (!wait_bounded(BAR(B_ST_EMPTY + s), ((it / kStages) & 1) ^ 1, wc, 1)) break;
+        const int q0 = q_start + it * kSub;
+        const uint32_t st = sbase + L::kOffStage + s * L::kStageBytes;
+        mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kBlkTile + 512);
+        for (int c = 0; c < L::kGroups; ++c) {
+          tma_load_3d(st + c * L::kBlkSub, &tmQ64, BAR(B_ST_FULL + s), c * 64, q0, bh);
+          tma_load_3d(st + L::kBlkTile + c * L::kBlkSub, &tmDO64, BAR(B_ST_FULL + s), c * 64, q0, bh);
         }
-        ++q_cnt[s];
+        const size_t vo = size_t(bh) * p.Np + q0;
+        bulk_load(st + 2 * L::kBlkTile, p.lse2 + vo, 256, BAR(B_ST_FULL + s));
+        bulk_load(st + 2 * L::kBlkTile + 256, p.dvec + vo, 256, BAR(B_ST_FULL + s));
+        ++cnt[s];
       }
       if (*abort_flag) {
-        wait_bounded(BAR(B_KV_FULL), 0, wc, 2, true);
-        for (int s = 0; s < 2; ++s)
-          if (q_cnt[s]) wait_bounded(BAR(B_Q_FULL + s), (q_cnt[s] - 1) & 1, wc, 2, true);
+        wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
+        for (int s = 0; s < kStages; ++s)
+          if (cnt[s]) wait_bounded(BAR(B_ST_FULL + s), (cnt[s] - 1) & 1, wc, 2, true);
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_kk = idesc_bf16(kBlk, kBlk, false, false);  // S^T, dP^T
-      constexpr uint32_t id_kmn = idesc_bf16(kBlk, D, false, true);     // dV, dK
-      constexpr uint32_t id_mnmn = idesc_bf16(kBlk, D, true, true);     // dQ
-      const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sDS = sbase + L::kOffDS;
-      bool ok = wait_bounded(BAR(B_KV_FULL), 0, wc, 10);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it & 1;
-        const uint32_t sQ = sbase + L::kOffQ + s * L::kTileBytes;
-        const uint32_t sDO = sbase + L::kOffDO + s * L::kTileBytes;
-        ok = wait_bounded(BAR(B_Q_FULL + s), (it >> 1) & 1, wc, 11);
+      auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
+      auto issue_sdp = [&](int it) {  // S^T and dP^T of block `it` into buffer it&1
+        const int b = it & 1;
+        const uint32_t st = stage_addr(it);
+        mma_rows_x_block<D>(tmem + L::col_s(b), sK, st);
+        mma_rows_x_block<D>(tmem + L::col_dp(b), sV, st + L::kBlkTile);
+        tc_commit(BAR(B_S_FULL + b));
+      };
+      bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
+      for (int it = 0; ok && it < 2 && it < n_blk; ++it) {
+        ok = wait_bounded(BAR(B_ST_FULL + it % kStages), (it / kStages) & 1, wc, 11);
         if (!ok) break;
         tc_fence_after();
-        // S^T = K Q^T  (A: K tile, B: Q tile, both K-major)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
-          mma_ss(tmem + L::kColS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024),
-                 id_kk, kk > 0);
-        }
-        tc_commit(BAR(B_S_FULL));
-        // dP^T reuses the columns dQ_{i-1} occupied: wait for its readers
-        if (it > 0) {
-          ok = wait_bounded(BAR(B_DQ_EMPTY), (it - 1) & 1, wc, 12);
+        issue_sdp(it);
+      }
+      for (int it = 0; ok && it < n_blk; ++it) {
+        const int b = it & 1;
+        ok = wait_bounded(BAR(B_P_READY + b), (it >> 1) & 1, wc, 12);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t st = stage_addr(it);
+        mma_tmem_x_block<D>(tmem + L::kColAcc0, tmem + L::col_s(b), st + L::kBlkTile, it > 0);  // dV += P^T dO
+        mma_tmem_x_block<D>(tmem + L::kColAcc1, tmem + L::col_dp(b), st, it > 0);               // dK += dS^T Q
+        tc_commit(BAR(B_ST_EMPTY + it % kStages));
+        if (it + 2 < n_blk) {
+          ok = wait_bounded(BAR(B_ST_FULL + (it + 2) % kStages), ((it + 2) / kStages) & 1, wc, 13);
           if (!ok) break;
           tc_fence_after();
+          issue_sdp(it + 2);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
-          mma_ss(tmem + L::kColDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024),
-                 id_kk, kk > 0);
-        }
-        tc_commit(BAR(B_DP_FULL));
-        ok = wait_bounded(BAR(B_P_READY), it & 1, wc, 13);
-        if (!ok) break;
-        tc_fence_after();
-        // dV += P^T dO   (A: P^T bf16 in TMEM over the S columns; B: dO MN-major)
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
-          mma_ts(tmem + L::kColDV, tmem + L::kColS + kk * 8,
-                 sdesc_sw128(sDO + kk * 2048, L::kSubBytes, 1024), id_kmn, (it > 0 || kk > 0));
-        // dK += dS^T Q   (A: dS^T K-major in smem; B: Q MN-major)
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
-          mma_ss(tmem + L::kColDK, sdesc_sw128(sDS + off, 16, 1024),
-                 sdesc_sw128(sQ + kk * 2048, L::kSubBytes, 1024), id_kmn, (it > 0 || kk > 0));
-        }
-        // dQ_i = dS K    (A: the dS^T buffer read MN-major; B: K MN-major)
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
-          mma_ss(tmem + L::kColDP, sdesc_sw128(sDS + kk * 2048, L::kSubBytes, 1024),
-                 sdesc_sw128(sK + kk * 2048, L::kSubBytes, 1024), id_mnmn, kk > 0);
-        tc_commit(BAR(B_DQ_FULL));
-        tc_commit(BAR(B_Q_EMPTY + s));
       }
       tc_commit(BAR(B_ACC_DONE));
       tc_commit(BAR(B_DRAIN));
       wait_bounded(BAR(B_DRAIN), 0, wc, 14, true);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ compute warps
-    const int r = warp * 32 + lane;  // key row inside the tile
-    const int key = jt * kBlk + r;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base + L::kColS;
-    const uint32_t tDP = tmem + lane_base + L::kColDP;
+  } else {
+    // ------------------------------------------------------------ compute warpgroups
+    const int b = warp >> 2;          // buffer of this warpgroup
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;   // key row in the tile
+    const int key = jt * kTile + r;
+    const bool row_valid = key < p.N;
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_base + L::col_s(b);
+    const uint32_t tDP = tmem + lane_base + L::col_dp(b);
     const float c = p.scale_log2;
-    uint8_t* ds_row = smem + L::kOffDS + r * 128;
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int i = i0 + it;
-      const float* l2 = p.lse2 + size_t(bh) * p.Np + size_t(i) * kBlk;
-      const float* dv = p.dvec + size_t(bh) * p.Np + size_t(i) * kBlk;
-      ok = wait_bounded(BAR(B_S_FULL), it & 1, wc, 20);
+    for (int it = b; it < n_blk; it += 2) {
+      ok = wait_bounded(BAR(B_S_FULL + b), (it >> 1) & 1, wc, 20);
+      if (ok) ok = wait_bounded(BAR(B_ST_FULL + it % kStages), (it / kStages) & 1, wc, 21);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld128_wait(tS, sr);
-      // P^T row: 2^(s c - L2_q); zero for masked entries
-      const bool row_valid = key < p.N;
-      const int qlim = (CAUSAL && i == jt) ? r : 0;  // queries q < qlim are masked
-      float pr[128];
+      const int q0 = q_start + it * kSub;
+      const float* l2 = reinterpret_cast<const float*>(smem + L::kOffStage + (it % kStages) * L::kStageBytes +
+                                                       2 * L::kBlkTile);
+      const float* dd = l2 + 64;
+      // queries q0 + i with i < qmask are hidden from this key (causal)
+      const int qmask = CAUSAL ? min(max(key - q0, 0), kSub) : 0;
+      uint32_t sr[64];
+      tmem_ld64_wait(tS, sr);
+      float pr[64];
 #pragma unroll
-      for (int q4 = 0; q4 < 32; ++q4) {
-        const float4 lv = __ldg(reinterpret_cast<const float4*>(l2) + q4);
-        const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int q = 4 * q4 + e;
-          const float x = ex2_approx(fmaf(__uint_as_float(sr[q]), c, -lq[e]));
-          pr[q] = (row_valid && q >= qlim) ? x : 0.f;
-        }
+      for (int i = 0; i < 64; ++i) {
+        const float x = ex2_approx(fmaf(__uint_as_float(sr[i]), c, -l2[i]));
+        pr[i] = (row_valid && i >= qmask) ? x : 0.f;
       }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {  // P^T (bf16) over the first 64 S columns
+      {
         uint32_t pk[32];
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          pk[q] = pack_bf16x2(pr[64 * half + 2 * q], pr[64 * half + 2 * q + 1]);
-        tmem_st32(tS + 32 * half, pk);
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
+        tmem_st32(tS, pk);  // P^T over the first 32 columns of S^T
       }
-      ok = wait_bounded(BAR(B_DP_FULL), it & 1, wc, 21);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      // dS^T = scale * P^T (dP^T - D), written to smem in the 128B-swizzled
-      // K-major layout: row r, 16-byte chunk ch of group g at
-      // g*16KB + r*128 + ((ch ^ (r%8)) * 16)
+      uint32_t dr[64];
+      tmem_ld64_wait(tDP, dr);
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int ch4 = 0; ch4 < 4; ++ch4) {  // 32 queries per TMEM load
-        uint32_t dr[32];
-        tmem_ld32_wait(tDP + ch4 * 32, dr);
-        float dd[32];
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 dvv = __ldg(reinterpret_cast<const float4*>(dv) + ch4 * 8 + q4);
-          dd[4 * q4 + 0] = dvv.x;
-          dd[4 * q4 + 1] = dvv.y;
-          dd[4 * q4 + 2] = dvv.z;
-          dd[4 * q4 + 3] = dvv.w;
+        for (int i = 0; i < 32; ++i) {
+          const float a = pr[2 * i] * p.scale * (__uint_as_float(dr[2 * i]) - dd[2 * i]);
+          const float e = pr[2 * i + 1] * p.scale * (__uint_as_float(dr[2 * i + 1]) - dd[2 * i + 1]);
+          pk[i] = pack_bf16x2(a, e);
         }
-#pragma unroll
-        for (int ck = 0; ck < 4; ++ck) {  // 8 queries = one 16-byte chunk
-          const int qb = ch4 * 32 + ck * 8;
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int q0 = qb + 2 * e;
-            const float a = pr[q0] * p.scale * (__uint_as_float(dr[ck * 8 + 2 * e]) - dd[ck * 8 + 2 * e]);
-            const float b = pr[q0 + 1] * p.scale *
-                            (__uint_as_float(dr[ck * 8 + 2 * e + 1]) - dd[ck * 8 + 2 * e + 1]);
-            w[e] = pack_bf16x2(a, b);
-          }
-          const int g = qb >> 6;
-          const int chunk = (qb & 63) >> 3;
-          *reinterpret_cast<uint4*>(ds_row + g * L::kSubBytes + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        tmem_st32(tDP, pk);  // dS^T over the first 32 columns of dP^T
       }
       tmem_st_wait();
-      fence_proxy_async_smem();  // make the dS^T stores visible to the tensor core
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_P_READY));
+      if (lane == 0) mbar_arrive(BAR(B_P_READY + b));
     }
-    // epilogue: dV and dK rows of this key tile
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK
     if (ok) {
       ok = wait_bounded(BAR(B_ACC_DONE), 0, wc, 22);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
       tc_fence_after();
-      const uint32_t tDV = tmem + lane_base + L::kColDV;
-      const uint32_t tDK = tmem + lane_base + L::kColDK;
       const size_t gro = (size_t(bh) * p.N + key) * D;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t src = which ? tDK : tDV;
-        uint16_t* dst = (which ? p.dk : p.dv) + gro;
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t v[32];
-          tmem_ld32_wait(src + ch * 32, v);
-          if (key < p.N) {
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(v[8 * v4 + 0]), __uint_as_float(v[8 * v4 + 1]));
-              w.y = pack_bf16x2(__uint_as_float(v[8 * v4 + 2]), __uint_as_float(v[8 * v4 + 3]));
-              w.z = pack_bf16x2(__uint_as_float(v[8 * v4 + 4]), __uint_as_float(v[8 * v4 + 5]));
-              w.w = pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7]));
-              *reinterpret_cast<uint4*>(dst + ch * 32 + 8 * v4) = w;
-            }
-          }
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ dQ readers (warps 6-9)
-    const int quad = warp & 3;         // TMEM lane quadrant this warp may access
-    const int r = quad * 32 + lane;    // query row inside the tile
-    const uint32_t tDQ = tmem + (uint32_t(quad * 32) << 16) + L::kColDP;
-    for (int it = 0; it < n_it; ++it) {
-      const int q = (i0 + it) * kBlk + r;
-      bool ok = wait_bounded(BAR(B_DQ_FULL), it & 1, wc, 30);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float* dst = p.dq_acc + (size_t(bh) * p.N + q) * D;
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32_wait(tDQ + ch * 32, v);
-        if (q < p.N) {
-#pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            atomicAdd(reinterpret_cast<float4*>(dst + ch * 32 + 4 * v4),
-                      make_float4(__uint_as_float(v[4 * v4]), __uint_as_float(v[4 * v4 + 1]),
-                                  __uint_as_float(v[4 * v4 + 2]), __uint_as_float(v[4 * v4 + 3])));
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_DQ_EMPTY));
+      if (b == 0)
+        store_acc_row<D>(tmem + lane_base + L::kColAcc0, p.dv + gro, row_valid);
+      else
+        store_acc_row<D>(tmem + lane_base + L::kColAcc1, p.dk + gro, row_valid);
     }
   }
 
@@ -435,66 +386,216 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // --------------------------------------------------------------------------
-// 3. dQ accumulator -> bf16
+// 3. dQ: query-tile-outer
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc,
-                                                       uint16_t* __restrict__ dq, size_t n4) {
-  const size_t i = size_t(blockIdx.x) * 256 + threadIdx.x;
-  if (i >= n4) return;
-  const float4 v = reinterpret_cast<const float4*>(acc)[i];
-  uint2 w;
-  w.x = pack_bf16x2(v.x, v.y);
-  w.y = pack_bf16x2(v.z, v.w);
-  reinterpret_cast<uint2*>(dq)[i] = w;
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ128, const __grid_constant__ CUtensorMap tmDO128,
+                  const __grid_constant__ CUtensorMap tmK64, const __grid_constant__ CUtensorMap tmV64,
+                  const BwdParams p) {
+  using L = Plan<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + L::kOffBar + 8u * uint32_t(i); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // query tiles that see the most key blocks first (causal: the last ones)
+  const int lvl = blockIdx.x / p.BH;
+  const int it_q = CAUSAL ? p.n_tiles - 1 - lvl : lvl;
+  const int bh = blockIdx.x % p.BH;
+  const int k_end = CAUSAL ? min(p.N, (it_q + 1) * kTile) : p.N;
+  const int n_blk = (k_end + kSub - 1) / kSub;
+  volatile int* abort_flag;
+  const uint32_t tmem = setup_cta<D>(smem, warp, abort_flag);
+  const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_BWD_DQ};
+  const uint32_t sQ = sbase + L::kOffRes0, sDO = sbase + L::kOffRes1;
+
+  if (warp == kLoadWarp) {
+    if (lane == 0) {
+      int cnt[kStages] = {0, 0, 0, 0};
+      mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kResTile);
+      for (int c = 0; c < L::kGroups; ++c) {
+        tma_load_3d(sQ + c * L::kResSub, &tmQ128, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
+        tma_load_3d(sDO + c * L::kResSub, &tmDO128, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
+      }
+      for (int it = 0; it < n_blk; ++it) {
+        const int s = it % kStages;
+        if (!wait_bounded(BAR(B_ST_EMPTY + s), ((it / kStages) & 1) ^ 1, wc, 1)) break;
+        const uint32_t st = sbase + L::kOffStage + s * L::kStageBytes;
+        mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kBlkTile);
+        for (int c = 0; c < L::kGroups; ++c) {
+          tma_load_3d(st + c * L::kBlkSub, &tmK64, BAR(B_ST_FULL + s), c * 64, it * kSub, bh);
+          tma_load_3d(st + L::kBlkTile + c * L::kBlkSub, &tmV64, BAR(B_ST_FULL + s), c * 64, it * kSub, bh);
+        }
+        ++cnt[s];
+      }
+      if (*abort_flag) {
+        wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
+        for (int s = 0; s < kStages; ++s)
+          if (cnt[s]) wait_bounded(BAR(B_ST_FULL + s), (cnt[s] - 1) & 1, wc, 2, true);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
+      auto issue_sdp = [&](int it) {  // S and dP of key block `it` into buffer it&1
+        const int b = it & 1;
+        const uint32_t st = stage_addr(it);
+        mma_rows_x_block<D>(tmem + L::col_s(b), sQ, st);
+        mma_rows_x_block<D>(tmem + L::col_dp(b), sDO, st + L::kBlkTile);
+        tc_commit(BAR(B_S_FULL + b));
+      };
+      bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
+      for (int it = 0; ok && it < 2 && it < n_blk; ++it) {
+        ok = wait_bounded(BAR(B_ST_FULL + it % kStages), (it / kStages) & 1, wc, 11);
+        if (!ok) break;
+        tc_fence_after();
+        issue_sdp(it);
+      }
+      for (int it = 0; ok && it < n_blk; ++it) {
+        const int b = it & 1;
+        ok = wait_bounded(BAR(B_P_READY + b), (it >> 1) & 1, wc, 12);
+        if (!ok) break;
+        tc_fence_after();
+        mma_tmem_x_block<D>(tmem + L::kColAcc0, tmem + L::col_dp(b), stage_addr(it), it > 0);  // dQ += dS K
+        tc_commit(BAR(B_ST_EMPTY + it % kStages));
+        if (it + 2 < n_blk) {
+          ok = wait_bounded(BAR(B_ST_FULL + (it + 2) % kStages), ((it + 2) / kStages) & 1, wc, 13);
+          if (!ok) break;
+          tc_fence_after();
+          issue_sdp(it + 2);
+        }
+      }
+      tc_commit(BAR(B_ACC_DONE));
+      tc_commit(BAR(B_DRAIN));
+      wait_bounded(BAR(B_DRAIN), 0, wc, 14, true);
+    }
+  } else {
+    const int b = warp >> 2;
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;   // query row in the tile
+    const int q = it_q * kTile + r;
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_base + L::col_s(b);
+    const uint32_t tDP = tmem + lane_base + L::col_dp(b);
+    const float c = p.scale_log2;
+    const float l2q = p.lse2[size_t(bh) * p.Np + it_q * kTile + r];  // +inf past N
+    const float dq_ = p.dvec[size_t(bh) * p.Np + it_q * kTile + r];
+    bool ok = true;
+    for (int it = b; it < n_blk; it += 2) {
+      ok = wait_bounded(BAR(B_S_FULL + b), (it >> 1) & 1, wc, 20);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int k0 = it * kSub;
+      // keys k0 + i with i >= klim are hidden (causal: key > q; or key >= N)
+      int klim = p.N - k0;
+      if (CAUSAL) klim = min(klim, q - k0 + 1);
+      klim = max(min(klim, kSub), 0);
+      uint32_t sr[64];
+      tmem_ld64_wait(tS, sr);
+      uint32_t dr[64];
+      tmem_ld64_wait(tDP, dr);
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), c, -l2q));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), c, -l2q));
+        const float a = (2 * i < klim) ? p0 * p.scale * (__uint_as_float(dr[2 * i]) - dq_) : 0.f;
+        const float e = (2 * i + 1 < klim) ? p1 * p.scale * (__uint_as_float(dr[2 * i + 1]) - dq_) : 0.f;
+        pk[i] = pack_bf16x2(a, e);
+      }
+      tmem_st32(tDP, pk);  // dS over the first 32 columns of dP
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_P_READY + b));
+    }
+    if (ok) {
+      ok = wait_bounded(BAR(B_ACC_DONE), 0, wc, 22);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok && b == 0) {
+      tc_fence_after();
+      store_acc_row<D>(tmem + lane_base + L::kColAcc0, p.dq + (size_t(bh) * p.N + q) * D, q < p.N);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <int D, bool CAUSAL>
-fa_status launch_main(const CUtensorMap* maps, const BwdParams& p, const LaunchCtx& ctx) {
-  auto kern = bwd_main_kernel<D, CAUSAL>;
-  const int smem = BwdLayout<D>::kSmemBytes;
+template <typename Kern>
+fa_status launch_main(Kern kern, unsigned kid, int smem, unsigned grid, const CUtensorMap* m,
+                      const BwdParams& p, const LaunchCtx& ctx, const char* what) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(bwd)");
-  const unsigned grid = unsigned(p.n_tiles) * unsigned(p.BH);
+  if (e != cudaSuccess) return cuda_fail(e, what);
   {
-    ProfileScope prof(KID_BWD, ctx.stream);
-    kern<<<grid, kThreads, smem, ctx.stream>>>(maps[0], maps[1], maps[2], maps[3], p);
+    ProfileScope prof(kid, ctx.stream);
+    kern<<<grid, kThreads, smem, ctx.stream>>>(m[0], m[1], m[2], m[3], p);
   }
   e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "bwd main kernel launch");
+  if (e != cudaSuccess) return cuda_fail(e, what);
   return FA_OK;
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_all(const void* q, const void* k, const void* v, const void* dO, const BwdParams& p,
+                     const LaunchCtx& ctx) {
+  const int smem = Plan<D>::kSmemBytes;
+  const unsigned grid = unsigned(p.n_tiles) * unsigned(p.BH);
+  CUtensorMap m[4];
+  fa_status st;
+  // dK/dV: queries and dO stream in blocks of 64 rows, K and V tiles of 128
+  if ((st = make_tmap_3d(&m[0], q, true, D, p.N, p.BH, 64, kSub, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&m[1], dO, true, D, p.N, p.BH, 64, kSub, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&m[2], k, true, D, p.N, p.BH, 64, kTile, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&m[3], v, true, D, p.N, p.BH, 64, kTile, true)) != FA_OK) return st;
+  st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid, m, p, ctx, "bwd dK/dV kernel");
+  if (st != FA_OK) return st;
+  // dQ: Q and dO tiles of 128 rows, K and V stream in blocks of 64
+  if ((st = make_tmap_3d(&m[0], q, true, D, p.N, p.BH, 64, kTile, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&m[1], dO, true, D, p.N, p.BH, 64, kTile, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&m[2], k, true, D, p.N, p.BH, 64, kSub, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&m[3], v, true, D, p.N, p.BH, 64, kSub, true)) != FA_OK) return st;
+  return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid, m, p, ctx, "bwd dQ kernel");
 }
 
 }  // namespace
 
 size_t bwd_workspace_bytes(int B, int H, int N, int d) {
+  (void)d;
   const size_t bh = size_t(B) * H;
-  const size_t np = (size_t(N) + kBlk - 1) / kBlk * kBlk;
-  return align256(bh * N * d * 4) + 2 * align256(bh * np * 4);
+  const size_t np = (size_t(N) + kTile - 1) / kTile * kTile;
+  return 2 * align256(bh * np * 4);
 }
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                      float scale, bool causal, void* workspace, const LaunchCtx& ctx) {
   const int BH = B * H;
-  if (BH > 65535) {
-    set_last_error("fa_bwd: B*H = %d exceeds 65535", BH);
-    return FA_ERR_UNSUPPORTED;
-  }
   BwdParams p;
   p.o = static_cast<const uint16_t*>(o);
   p.dO = static_cast<const uint16_t*>(dO);
   p.lse = lse;
   p.N = N;
-  p.n_tiles = (N + kBlk - 1) / kBlk;
-  p.Np = p.n_tiles * kBlk;
+  p.n_tiles = (N + kTile - 1) / kTile;
+  p.Np = p.n_tiles * kTile;
   p.BH = BH;
+  if ((long long)p.n_tiles * BH > 0x7fffffffLL) {
+    set_last_error("fa_bwd: too many tiles");
+    return FA_ERR_UNSUPPORTED;
+  }
   char* ws = static_cast<char*>(workspace);
-  p.dq_acc = reinterpret_cast<float*>(ws);
-  p.lse2 = reinterpret_cast<float*>(ws + align256(size_t(BH) * N * d * 4));
-  p.dvec = reinterpret_cast<float*>(ws + align256(size_t(BH) * N * d * 4) +
-                                    align256(size_t(BH) * p.Np * 4));
+  p.lse2 = reinterpret_cast<float*>(ws);
+  p.dvec = reinterpret_cast<float*>(ws + align256(size_t(BH) * p.Np * 4));
   p.dq = static_cast<uint16_t*>(dq);
   p.dk = static_cast<uint16_t*>(dk);
   p.dv = static_cast<uint16_t*>(dv);
@@ -503,7 +604,6 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
 
-  // 1. preprocess
   {
     const long long warps = (long long)BH * p.Np;
     const long long blocks = (warps * 32 + 255) / 256;
@@ -515,28 +615,9 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "bwd preprocess launch");
   }
-  // 2. main
-  CUtensorMap maps[4];
-  const void* srcs[4] = {q, k, v, dO};
-  for (int m = 0; m < 4; ++m) {
-    fa_status st = make_tmap_3d(&maps[m], srcs[m], true, d, N, BH, 64, 128, true);
-    if (st != FA_OK) return st;
-  }
-  fa_status st;
   if (d == 128)
-    st = causal ? launch_main<128, true>(maps, p, ctx) : launch_main<128, false>(maps, p, ctx);
-  else
-    st = causal ? launch_main<64, true>(maps, p, ctx) : launch_main<64, false>(maps, p, ctx);
-  if (st != FA_OK) return st;
-  // 3. dQ to bf16
-  {
-    const size_t n4 = size_t(BH) * N * d / 4;
-    ProfileScope prof(KID_BWD_POST, ctx.stream);
-    bwd_post_kernel<<<unsigned((n4 + 255) / 256), 256, 0, ctx.stream>>>(p.dq_acc, p.dq, n4);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "bwd dQ conversion launch");
-  }
-  return FA_OK;
+    return causal ? launch_all<128, true>(q, k, v, dO, p, ctx) : launch_all<128, false>(q, k, v, dO, p, ctx);
+  return causal ? launch_all<64, true>(q, k, v, dO, p, ctx) : launch_all<64, false>(q, k, v, dO, p, ctx);
 }
 
 }  // namespace fa

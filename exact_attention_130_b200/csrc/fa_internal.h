@@ -24,8 +24,8 @@ enum KernelId : unsigned int {
   KID_FWD = 1,
   KID_FWD_F32 = 2,
   KID_BWD_PRE = 3,
-  KID_BWD = 4,
-  KID_BWD_POST = 5,
+  KID_BWD = 4,      // dK/dV kernel
+  KID_BWD_DQ = 5,   // dQ kernel
   KID_DECODE = 6,
   KID_DECODE_MERGE = 7,
 };

@@ -33,8 +33,9 @@
 //  * O~ is rescaled only when a row maximum grows by more than 2^8 (the
 //    final division by l is exact whatever reference maximum was used), so
 //    the O read-modify-write almost never runs;
-//  * causal units are ordered longest first so the persistent CTAs finish
-//    together;
+//  * work units are handed out head-major (K/V reuse in L2); under the
+//    causal mask each CTA takes complementary pairs of Q-tile levels, so
+//    the persistent CTAs carry equal work;
 //  * every mbarrier wait is bounded in time; a wait that runs out records
 //    the failure in the device status word and the CTA returns.
 #include <cfloat>
@@ -90,17 +91,50 @@ struct FwdParams {
   int BH;
   int n_kv;       // K/V tiles per head
   int n_pairs;    // Q-tile pairs per head
-  int num_units;  // BH * n_pairs
+  int cpp;        // causal: couples of pairs per head, ceil(n_pairs / 2)
+  int num_items;  // work items handed out round-robin to the CTAs
   float scale_log2;
   unsigned int* status;
   unsigned long long limit_ns;
   int debug_skip;
 };
 
-__device__ __forceinline__ void unit_coords(int u, const FwdParams& p, int& bh, int& pair) {
-  // longest (highest) Q-tile pairs first; all heads of a pair level together
-  pair = p.n_pairs - 1 - u / p.BH;
-  bh = u % p.BH;
+// Work list. A unit is one (head, Q-tile pair). CTA c takes items c, c + G,
+// c + 2G, ... (G = grid size), so all three roles walk the same sequence.
+//  * no mask: item = unit, head-major, so the ~G units in flight share few
+//    heads and their K/V tiles stay in L2;
+//  * causal: item = a couple of pairs (n_pairs-1-k, k) of one head, the
+//    heavier first; a couple always costs 2 n_pairs + 1 K/V tile steps, so
+//    equal item counts mean equal work, and the couples of one head run
+//    side by side (L2 reuse again). With n_pairs odd the middle pair is a
+//    couple on its own.
+// Advances (item, half) and returns the unit, or false at the end.
+template <bool CAUSAL>
+__device__ __forceinline__ bool next_unit(const FwdParams& p, int& item, int& half, int& bh,
+                                          int& pair) {
+  if (item >= p.num_items) return false;
+  if (!CAUSAL) {
+    bh = item / p.n_pairs;
+    pair = item % p.n_pairs;
+    item += gridDim.x;
+    return true;
+  }
+  bh = item / p.cpp;
+  const int k = item % p.cpp;
+  const int hi = p.n_pairs - 1 - k;
+  if (half == 0) {
+    pair = hi;
+    if (hi == k) {
+      item += gridDim.x;
+    } else {
+      half = 1;
+    }
+  } else {
+    pair = k;
+    half = 0;
+    item += gridDim.x;
+  }
+  return true;
 }
 
 template <bool CAUSAL>
@@ -168,9 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < L::kStages; ++s) k_cnt[s] = v_cnt[s] = 0;
       bool skip_pending = p.debug_skip && blockIdx.x == 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++unit_iter) {
-        int bh, pair;
-        unit_coords(u, p, bh, pair);
+      int item = blockIdx.x, half = 0, bh, pair;
+      for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
         const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
         for (int t = 0; t < 2 && ok; ++t) {
           ok = wait_bounded(BAR(B_Q_EMPTY + t), (unit_iter & 1) ^ 1, wc, 1);
@@ -241,9 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int kv_used = 0, unit_iter = 0;
       int p_cnt[2] = {0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++unit_iter) {
-        int bh, pair;
-        unit_coords(u, p, bh, pair);
+      int item = blockIdx.x, half = 0, bh, pair;
+      for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
         const int n[2] = {kv_tiles_for<CAUSAL>(2 * pair, p.n_kv),
                           kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv)};
         for (int t = 0; t < 2 && ok; ++t)
@@ -311,9 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     int s_cnt = 0, unit_iter = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++unit_iter) {
-      int bh, pair;
-      unit_coords(u, p, bh, pair);
+    int item = blockIdx.x, half = 0, bh, pair;
+    for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
       const int qt = 2 * pair + t;
       const int nt = kv_tiles_for<CAUSAL>(qt, p.n_kv);
       const int row = qt * kBM + r;
@@ -431,7 +462,7 @@ fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
   const int smem = Layout<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fwd)");
-  const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
+  const int grid = p.num_items < ctx.num_sms ? p.num_items : ctx.num_sms;
   {
     ProfileScope prof(KID_FWD, ctx.stream);
     kern<<<grid, kThreads, smem, ctx.stream>>>(mq, mk, mv, p);
@@ -459,7 +490,8 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   p.BH = int(BH);
   p.n_kv = (N + kBN - 1) / kBN;
   p.n_pairs = (p.n_kv + 1) / 2;
-  p.num_units = p.BH * p.n_pairs;
+  p.cpp = (p.n_pairs + 1) / 2;
+  p.num_items = causal ? p.BH * p.cpp : p.BH * p.n_pairs;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;

@@ -99,10 +99,10 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o,
                      int causal, cudaStream_t stream);
 
 /*
- * fa_bwd_workspace_size -- bytes of scratch fa_bwd needs: an fp32 dQ
- * accumulator [B, H, N, d], then two fp32 vectors [B, H, Np] (the saved LSE
- * in base 2, and D = rowsum(dO * O)), Np = N rounded up to a multiple of
- * 128; each part starts on a 256-byte boundary. Returns 0 for invalid sizes.
+ * fa_bwd_workspace_size -- bytes of scratch fa_bwd needs: two fp32 vectors
+ * [B, H, Np] (the saved LSE in base 2, and D = rowsum(dO * O)), Np = N
+ * rounded up to a multiple of 128, each starting on a 256-byte boundary.
+ * Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -114,11 +114,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *   workspace      : device scratch of >= fa_bwd_workspace_size() bytes,
  *                    16-byte aligned; its contents on entry do not matter
  *                    and are overwritten.
- * Computes D = rowsum(dO * O), then per key tile recomputes
- * P = exp(S - LSE), dV = P^T dO, dP = dO V^T, dS = P * (dP - D),
- * dK = scale dS^T Q, dQ = scale dS K ("Geri Yayilim").
- * d : 64 or 128. Deterministic for dK and dV; dQ is summed with fp32
- * atomics, so its low bits may differ between runs.
+ * Computes D = rowsum(dO * O), then recomputes P = exp(S - LSE) block by
+ * block and forms dV = P^T dO, dP = dO V^T, dS = P * (dP - D),
+ * dK = scale dS^T Q ("Geri Yayilim") in a key-tile-outer kernel and
+ * dQ = scale dS K in a query-tile-outer kernel. d : 64 or 128.
+ * Deterministic: bitwise identical results on every run.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
                  const float* lse, const void* dO, void* dq, void* dk,
@@ -215,8 +215,8 @@ void fa_debug_skip_load(int enable);
  * synchronises those events, stops recording and writes, for each kernel id
  * k in [0, capacity), the number of launches (launches[k]) and their summed
  * device time in milliseconds (total_ms[k]). Kernel ids: 1 forward (bf16),
- * 2 forward (fp32), 3 backward preprocess, 4 backward main, 5 backward dQ
- * conversion, 6 decode split, 7 decode merge. Returns the number of ids
+ * 2 forward (fp32), 3 backward preprocess, 4 backward dK/dV, 5 backward
+ * dQ, 6 decode split, 7 decode merge. Returns the number of ids
  * (8), or -1 if a CUDA call failed. Not thread-safe against concurrent
  * begin/end pairs; launches from several threads are recorded.
  */

@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kLoadWarp) {
     if (lane == 0) {
-      int cnt[kStages] = {0, 0, 0, 0};
+      int issued = 0;
       mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kResTile);
       for (int c = 0; c < L::kGroups; ++c) {
         tma_load_3d(sK + c * L::kResSub, &tmK128, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
@@ -262,12 +262,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t vo = size_t(bh) * p.Np + q0;
         bulk_load(st + 2 * L::kBlkTile, p.lse2 + vo, 256, BAR(B_ST_FULL + s));
         bulk_load(st + 2 * L::kBlkTile + 256, p.dvec + vo, 256, BAR(B_ST_FULL + s));
-        ++cnt[s];
+        ++issued;
       }
       if (*abort_flag) {
         wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
-        for (int s = 0; s < kStages; ++s)
-          if (cnt[s]) wait_bounded(BAR(B_ST_FULL + s), (cnt[s] - 1) & 1, wc, 2, true);
+        for (int s = 0; s < kStages; ++s) {
+          const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
+          if (cnt > 0) wait_bounded(BAR(B_ST_FULL + s), (cnt - 1) & 1, wc, 2, true);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -413,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kLoadWarp) {
     if (lane == 0) {
-      int cnt[kStages] = {0, 0, 0, 0};
+      int issued = 0;
       mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kResTile);
       for (int c = 0; c < L::kGroups; ++c) {
         tma_load_3d(sQ + c * L::kResSub, &tmQ128, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
@@ -428,12 +430,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(st + c * L::kBlkSub, &tmK64, BAR(B_ST_FULL + s), c * 64, it * kSub, bh);
           tma_load_3d(st + L::kBlkTile + c * L::kBlkSub, &tmV64, BAR(B_ST_FULL + s), c * 64, it * kSub, bh);
         }
-        ++cnt[s];
+        ++issued;
       }
       if (*abort_flag) {
         wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
-        for (int s = 0; s < kStages; ++s)
-          if (cnt[s]) wait_bounded(BAR(B_ST_FULL + s), (cnt[s] - 1) & 1, wc, 2, true);
+        for (int s = 0; s < kStages; ++s) {
+          const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
+          if (cnt > 0) wait_bounded(BAR(B_ST_FULL + s), (cnt - 1) & 1, wc, 2, true);
+        }
       }
     }
   } else if (warp == kMmaWarp) {

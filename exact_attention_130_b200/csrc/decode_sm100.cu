@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kThreads)
     if (lane == 0) {
       const uint16_t* kb = p.kc + (bh * p.Lmax + t0) * D;
       const uint16_t* vb = p.vc + (bh * p.Lmax + t0) * D;
-      int issued[kStages] = {0, 0, 0, 0};
+      int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kStages;
         if (!wait_bounded(EMPTY(s), ((i / kStages) & 1) ^ 1, wc, 1)) break;
@@ -125,11 +125,13 @@ __global__ void __launch_bounds__(kThreads)
         mbar_arrive_expect_tx(FULL(s), 2 * bytes);
         bulk_load(sbase + L::kOffK + s * L::kTileBytes, kb + size_t(i) * kTileT * D, bytes, FULL(s));
         bulk_load(sbase + L::kOffV + s * L::kTileBytes, vb + size_t(i) * kTileT * D, bytes, FULL(s));
-        ++issued[s];
+        ++issued;
       }
       if (*abort_flag)
-        for (int s = 0; s < kStages; ++s)
-          if (issued[s]) wait_bounded(FULL(s), (issued[s] - 1) & 1, wc, 2, true);
+        for (int s = 0; s < kStages; ++s) {
+          const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
+          if (cnt > 0) wait_bounded(FULL(s), (cnt - 1) & 1, wc, 2, true);
+        }
     }
   } else {
     // ---------------------------------------------------------------- consumers

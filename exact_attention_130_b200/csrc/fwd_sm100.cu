@@ -18,11 +18,14 @@
 // entries before the row maximum is taken.
 //
 // B200 design (not the pages' A100/H100 kernels):
-//  * persistent grid, one CTA per SM, 10 warps:
+//  * persistent grid, one CTA per SM, 12 warps:
 //      warps 0-3  softmax for Q tile 0 (one TMEM lane = one query row)
 //      warps 4-7  softmax for Q tile 1
 //      warp  8    TMA producer (Q tiles once per work unit, K/V ring)
 //      warp  9    tcgen05 MMA issuer (one thread)
+//      warps 10-11 complete the third warpgroup (no work)
+//    the control warpgroup hands registers to the softmax warpgroups
+//    (setmaxnreg), so the 128 scores of a row stay in registers;
 //  * a work unit is 2 Q tiles of 128 rows of one (batch, head); both share
 //    every K/V tile, which halves K/V shared-memory traffic per FLOP;
 //  * TMEM (512 columns): S_0 | S_1 | O_0 | O_1. The softmax writes P as bf16
@@ -48,7 +51,15 @@ namespace {
 
 constexpr int kBM = 128;  // query rows per Q tile
 constexpr int kBN = 128;  // keys per K/V tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // 3 warpgroups
+// Registers per thread: the kernel launches with 168 (65536 / 384, rounded
+// down to a multiple of 8); the softmax warpgroups then take 208 and the
+// load/MMA warpgroup keeps 88: 2*128*208 + 128*88 = 384*168.
+constexpr int kRegsAtLaunch = 168;
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsControl = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsAtLaunch,
+              "register split exceeds the launch allocation");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when m grows by > 2^8
@@ -59,10 +70,10 @@ enum : int {
   B_Q_FULL = 0,    // +t
   B_Q_EMPTY = 2,   // +t
   B_S_FULL = 4,    // +t
-  B_P_FULL = 6,    // +t
+  B_P_FULL = 12,   // +t: P of tile t is in TMEM
   B_O_FULL = 8,    // +t
   B_O_EMPTY = 10,  // +t
-  B_DRAIN = 12,
+  B_DRAIN = 6,
   B_K_FULL = 16,   // +stage
   B_V_FULL = 20,   // +stage
   B_KV_EMPTY = 24, // +stage
@@ -193,147 +204,160 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_FWD};
 
-  if (warp == kLoadWarp) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int kv_issued = 0, unit_iter = 0;
-      int q_cnt[2] = {0, 0};
-      int k_cnt[L::kStages], v_cnt[L::kStages];
-      for (int s = 0; s < L::kStages; ++s) k_cnt[s] = v_cnt[s] = 0;
-      bool skip_pending = p.debug_skip && blockIdx.x == 0;
-      bool ok = true;
-      int item = blockIdx.x, half = 0, bh, pair;
-      for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
-        const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
-        for (int t = 0; t < 2 && ok; ++t) {
-          ok = wait_bounded(BAR(B_Q_EMPTY + t), (unit_iter & 1) ^ 1, wc, 1);
-          if (!ok) break;
-          mbar_arrive_expect_tx(BAR(B_Q_FULL + t), L::kTileBytes);
-          for (int c = 0; c < L::kSub; ++c)
-            tma_load_3d(sbase + L::kOffQ + t * L::kTileBytes + c * L::kSubBytes, &tmQ,
-                        BAR(B_Q_FULL + t), c * 64, (2 * pair + t) * kBM, bh);
-          ++q_cnt[t];
-        }
-        for (int j = 0; ok && j < n1; ++j, ++kv_issued) {
-          const int s = kv_issued % L::kStages;
-          const uint32_t ph = (kv_issued / L::kStages) & 1;
-          ok = wait_bounded(BAR(B_KV_EMPTY + s), ph ^ 1, wc, 2);
-          if (!ok) break;
-          mbar_arrive_expect_tx(BAR(B_K_FULL + s), L::kTileBytes);
-          for (int c = 0; c < L::kSub; ++c)
-            tma_load_3d(sbase + L::kOffK + s * L::kTileBytes + c * L::kSubBytes, &tmK,
-                        BAR(B_K_FULL + s), c * 64, j * kBN, bh);
-          ++k_cnt[s];
-          if (skip_pending) {
-            skip_pending = false;  // test hook: this V tile never arrives
-          } else {
-            mbar_arrive_expect_tx(BAR(B_V_FULL + s), L::kTileBytes);
+  if (warp >= 8) {
+    regs_decrease<kRegsControl>();
+    if (warp == kLoadWarp) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        int kv_issued = 0, unit_iter = 0;
+        int q_issued0 = 0, q_issued1 = 0;
+        int v_skip_stage = -1;  // stage whose V load the test hook left out
+        bool skip_pending = p.debug_skip && blockIdx.x == 0;
+        bool ok = true;
+        int item = blockIdx.x, half = 0, bh, pair;
+        for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
+          const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
+          for (int t = 0; t < 2 && ok; ++t) {
+            ok = wait_bounded(BAR(B_Q_EMPTY + t), (unit_iter & 1) ^ 1, wc, 1);
+            if (!ok) break;
+            mbar_arrive_expect_tx(BAR(B_Q_FULL + t), L::kTileBytes);
             for (int c = 0; c < L::kSub; ++c)
-              tma_load_3d(sbase + L::kOffV + s * L::kTileBytes + c * L::kSubBytes, &tmV,
-                          BAR(B_V_FULL + s), c * 64, j * kBN, bh);
-            ++v_cnt[s];
+              tma_load_3d(sbase + L::kOffQ + t * L::kTileBytes + c * L::kSubBytes, &tmQ,
+                          BAR(B_Q_FULL + t), c * 64, (2 * pair + t) * kBM, bh);
+            (t ? q_issued1 : q_issued0) += 1;
+          }
+          for (int j = 0; ok && j < n1; ++j, ++kv_issued) {
+            const int s = kv_issued % L::kStages;
+            const uint32_t ph = (kv_issued / L::kStages) & 1;
+            ok = wait_bounded(BAR(B_KV_EMPTY + s), ph ^ 1, wc, 2);
+            if (!ok) break;
+            mbar_arrive_expect_tx(BAR(B_K_FULL + s), L::kTileBytes);
+            for (int c = 0; c < L::kSub; ++c)
+              tma_load_3d(sbase + L::kOffK + s * L::kTileBytes + c * L::kSubBytes, &tmK,
+                          BAR(B_K_FULL + s), c * 64, j * kBN, bh);
+            if (skip_pending) {
+              skip_pending = false;  // test hook: this V tile never arrives
+              v_skip_stage = s;
+            } else {
+              mbar_arrive_expect_tx(BAR(B_V_FULL + s), L::kTileBytes);
+              for (int c = 0; c < L::kSub; ++c)
+                tma_load_3d(sbase + L::kOffV + s * L::kTileBytes + c * L::kSubBytes, &tmV,
+                            BAR(B_V_FULL + s), c * 64, j * kBN, bh);
+            }
+          }
+        }
+        if (*abort_flag) {
+          // let every copy this thread started land before the CTA exits: the
+          // last load into a barrier completes its phase (loads - 1)
+          if (q_issued0) wait_bounded(BAR(B_Q_FULL + 0), (q_issued0 - 1) & 1, wc, 3, true);
+          if (q_issued1) wait_bounded(BAR(B_Q_FULL + 1), (q_issued1 - 1) & 1, wc, 3, true);
+          for (int s = 0; s < L::kStages; ++s) {
+            const int kc = (kv_issued - s + L::kStages - 1) / L::kStages;  // K loads into s
+            const int vc = kc - (s == v_skip_stage ? 1 : 0);
+            if (kc > 0) wait_bounded(BAR(B_K_FULL + s), (kc - 1) & 1, wc, 3, true);
+            if (vc > 0) wait_bounded(BAR(B_V_FULL + s), (vc - 1) & 1, wc, 3, true);
           }
         }
       }
-      if (*abort_flag) {
-        // let every copy this thread started land before the CTA exits
-        for (int t = 0; t < 2; ++t)
-          if (q_cnt[t]) wait_bounded(BAR(B_Q_FULL + t), (q_cnt[t] - 1) & 1, wc, 3, true);
-        for (int s = 0; s < L::kStages; ++s) {
-          if (k_cnt[s]) wait_bounded(BAR(B_K_FULL + s), (k_cnt[s] - 1) & 1, wc, 3, true);
-          if (v_cnt[s]) wait_bounded(BAR(B_V_FULL + s), (v_cnt[s] - 1) & 1, wc, 3, true);
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, false, true);
+        auto colS = [](int t) { return t ? L::kColS1 : L::kColS0; };
+        auto colO = [](int t) { return t ? L::kColO1 : L::kColO0; };
+        auto issue_qk = [&](int t, int stage) {
+          const uint32_t qa = sbase + L::kOffQ + t * L::kTileBytes;
+          const uint32_t kb = sbase + L::kOffK + stage * L::kTileBytes;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
+            mma_ss(tmem + colS(t), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                   idesc_qk, kk > 0 ? 1u : 0u);
+          }
+        };
+        // O_t (+)= P_t V: P (bf16) from the first 64 TMEM columns of S_t
+        auto issue_pv = [&](int t, int stage, bool acc) {
+          const uint32_t vb = sbase + L::kOffV + stage * L::kTileBytes;
+  #pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ts(tmem + colO(t), tmem + colS(t) + kk * 8,
+                   sdesc_sw128(vb + kk * 16 * 128, L::kSubBytes, 1024), idesc_pv,
+                   (acc || kk > 0) ? 1u : 0u);
+        };
+        int kv_used = 0, unit_iter = 0;
+        int p_cnt[2] = {0, 0};
+        bool ok = true;
+        int item = blockIdx.x, half = 0, bh, pair;
+        for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
+          const int n0 = kv_tiles_for<CAUSAL>(2 * pair, p.n_kv);
+          const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
+          for (int t = 0; t < 2 && ok; ++t)
+            ok = wait_bounded(BAR(B_Q_FULL + t), unit_iter & 1, wc, 10);
+          if (!ok) break;
+          {
+            const int s0 = kv_used % L::kStages;
+            ok = wait_bounded(BAR(B_K_FULL + s0), (kv_used / L::kStages) & 1, wc, 11);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(0, s0);
+            tc_commit(BAR(B_S_FULL + 0));
+            issue_qk(1, s0);
+            tc_commit(BAR(B_S_FULL + 1));
+          }
+          int k_ready = 0;
+          for (int j = 0; ok && j < n1; ++j) {
+            const int s = (kv_used + j) % L::kStages;
+            ok = wait_bounded(BAR(B_V_FULL + s), ((kv_used + j) / L::kStages) & 1, wc, 12);
+            if (!ok) break;
+  #pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int nt = t ? n1 : n0;
+              if (j >= nt) continue;
+              if (j == 0) {
+                ok = wait_bounded(BAR(B_O_EMPTY + t), (unit_iter & 1) ^ 1, wc, 13);
+                if (!ok) break;
+              }
+              ok = wait_bounded(BAR(B_P_FULL + t), p_cnt[t] & 1, wc, 14);
+              if (!ok) break;
+              ++p_cnt[t];
+              tc_fence_after();
+              issue_pv(t, s, j > 0);
+              if (j + 1 < nt) {
+                const int s2 = (kv_used + j + 1) % L::kStages;
+                if (k_ready < j + 1) {
+                  ok = wait_bounded(BAR(B_K_FULL + s2), ((kv_used + j + 1) / L::kStages) & 1, wc,
+                                    15);
+                  if (!ok) break;
+                  k_ready = j + 1;
+                  tc_fence_after();
+                }
+                issue_qk(t, s2);
+                tc_commit(BAR(B_S_FULL + t));
+              } else {
+                tc_commit(BAR(B_O_FULL + t));
+                tc_commit(BAR(B_Q_EMPTY + t));
+              }
+            }
+            if (!ok) break;
+            tc_commit(BAR(B_KV_EMPTY + s));
+          }
+          kv_used += n1;
         }
+        // every MMA issued above must be finished before TMEM is released
+        tc_commit(BAR(B_DRAIN));
+        wait_bounded(BAR(B_DRAIN), 0, wc, 16, true);
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, false, true);
-      const uint32_t colS[2] = {L::kColS0, L::kColS1};
-      const uint32_t colO[2] = {L::kColO0, L::kColO1};
-      auto issue_qk = [&](int t, int stage) {
-        const uint32_t qa = sbase + L::kOffQ + t * L::kTileBytes;
-        const uint32_t kb = sbase + L::kOffK + stage * L::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
-          mma_ss(tmem + colS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                 idesc_qk, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int t, int stage, bool acc) {
-        const uint32_t vb = sbase + L::kOffV + stage * L::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8,
-                 sdesc_sw128(vb + kk * 16 * 128, L::kSubBytes, 1024), idesc_pv,
-                 (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      int kv_used = 0, unit_iter = 0;
-      int p_cnt[2] = {0, 0};
-      bool ok = true;
-      int item = blockIdx.x, half = 0, bh, pair;
-      for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
-        const int n[2] = {kv_tiles_for<CAUSAL>(2 * pair, p.n_kv),
-                          kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv)};
-        for (int t = 0; t < 2 && ok; ++t)
-          ok = wait_bounded(BAR(B_Q_FULL + t), unit_iter & 1, wc, 10);
-        if (!ok) break;
-        {
-          const int s0 = kv_used % L::kStages;
-          ok = wait_bounded(BAR(B_K_FULL + s0), (kv_used / L::kStages) & 1, wc, 11);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(0, s0);
-          tc_commit(BAR(B_S_FULL + 0));
-          issue_qk(1, s0);
-          tc_commit(BAR(B_S_FULL + 1));
-        }
-        int k_ready = 0;
-        for (int j = 0; ok && j < n[1]; ++j) {
-          const int s = (kv_used + j) % L::kStages;
-          ok = wait_bounded(BAR(B_V_FULL + s), ((kv_used + j) / L::kStages) & 1, wc, 12);
-          if (!ok) break;
-          for (int t = 0; t < 2; ++t) {
-            if (j >= n[t]) continue;
-            if (j == 0) {
-              ok = wait_bounded(BAR(B_O_EMPTY + t), (unit_iter & 1) ^ 1, wc, 13);
-              if (!ok) break;
-            }
-            ok = wait_bounded(BAR(B_P_FULL + t), p_cnt[t] & 1, wc, 14);
-            if (!ok) break;
-            ++p_cnt[t];
-            tc_fence_after();
-            issue_pv(t, s, j > 0);
-            if (j + 1 < n[t]) {
-              const int s2 = (kv_used + j + 1) % L::kStages;
-              if (k_ready < j + 1) {
-                ok = wait_bounded(BAR(B_K_FULL + s2), ((kv_used + j + 1) / L::kStages) & 1, wc,
-                                  15);
-                if (!ok) break;
-                k_ready = j + 1;
-                tc_fence_after();
-              }
-              issue_qk(t, s2);
-              tc_commit(BAR(B_S_FULL + t));
-            } else {
-              tc_commit(BAR(B_O_FULL + t));
-              tc_commit(BAR(B_Q_EMPTY + t));
-            }
-          }
-          if (!ok) break;
-          tc_commit(BAR(B_KV_EMPTY + s));
-        }
-        kv_used += n[1];
-      }
-      // every MMA issued above must be finished before TMEM is released
-      tc_commit(BAR(B_DRAIN));
-      wait_bounded(BAR(B_DRAIN), 0, wc, 16, true);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
     }
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
+    regs_increase<kRegsSoftmax>();
     const int t = warp >> 2;          // Q tile of this warpgroup
     const int wq = warp & 3;          // TMEM lane quadrant of this warp
     const int r = wq * 32 + lane;     // row inside the Q tile
@@ -367,15 +391,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 128; ++i) s[i] = (i < limit) ? s[i] : -INFINITY;
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]);
+        float mx2 = fmaxf(s[4], s[5]), mx3 = fmaxf(s[6], s[7]);
 #pragma unroll
-        for (int i = 4; i < 128; i += 4) {
-          mx0 = fmaxf(mx0, s[i]);
-          mx1 = fmaxf(mx1, s[i + 1]);
-          mx2 = fmaxf(mx2, s[i + 2]);
-          mx3 = fmaxf(mx3, s[i + 3]);
+        for (int i = 8; i < 128; i += 8) {
+          mx0 = max3f(mx0, s[i], s[i + 1]);
+          mx1 = max3f(mx1, s[i + 2], s[i + 3]);
+          mx2 = max3f(mx2, s[i + 4], s[i + 5]);
+          mx3 = max3f(mx3, s[i + 6], s[i + 7]);
         }
-        const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c);
+        const float m_new = fmaxf(m, fmaxf(max3f(mx0, mx1, mx2), mx3) * c);
         if (j == 0) {
           m = m_new;
         } else if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
@@ -393,23 +418,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(tO + ch * 32, orow);
           }
         }
+        // P = 2^(s c - m): x = s c - m by one paired FMA per two columns, 2^x
+        // on MUFU, row sum by paired adds; P goes to TMEM as bf16 over the
+        // first 64 columns of S.
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_m, neg_m);
+        uint64_t sum_a = f2_pack(0.f, 0.f), sum_b = sum_a;
         uint32_t pk[64];
-        float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2_approx(fmaf(s[2 * i], c, neg_m));
-          const float p1 = ex2_approx(fmaf(s[2 * i + 1], c, neg_m));
-          rs0 += p0;
-          rs1 += p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), c2, nm2), x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (i & 1)
+            sum_b = f2_add(sum_b, f2_pack(p0, p1));
+          else
+            sum_a = f2_add(sum_a, f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st64(tS, pk);  // P (bf16) over the first 64 columns of S
+        tmem_st64(tS, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(B_P_FULL + t));
-        l += rs0 + rs1;
+        {
+          float a0, a1;
+          f2_unpack(f2_add(sum_a, sum_b), a0, a1);
+          l += a0 + a1;
+        }
       }
       if (!ok) break;
       // epilogue: O = O~ / l, LSE = ln2 * (m + log2 l)
@@ -445,13 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_O_EMPTY + t));
     }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tc_fence_before();
+    __syncthreads();
   }
 }
 
@@ -462,6 +493,16 @@ fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
   const int smem = Layout<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fwd)");
+  // the setmaxnreg split is sized for exactly kRegsAtLaunch registers per
+  // thread; with fewer the increase could wait forever, so refuse to launch
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(fwd)");
+  if (attr.numRegs != kRegsAtLaunch) {
+    set_last_error("fwd kernel built with %d registers per thread, expected %d", attr.numRegs,
+                   kRegsAtLaunch);
+    return FA_ERR_UNSUPPORTED;
+  }
   const int grid = p.num_items < ctx.num_sms ? p.num_items : ctx.num_sms;
   {
     ProfileScope prof(KID_FWD, ctx.stream);

@@ -62,28 +62,41 @@ struct WaitCtl {
   unsigned int kernel_id;         // recorded in the status word
 };
 
-// Waits until the phase with the given parity of `bar` has completed.
-// Returns true on completion; false if this CTA is aborting or the time limit
-// ran out (then the abort flag and the device status word are set). Never
-// spins forever. With `drain` set the abort flag is ignored (used to let
-// copies already in flight land before an aborting CTA exits); the time
-// limit still applies.
-static __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCtl& w,
-                                          uint32_t site, bool drain = false) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of wait_bounded: keeps polling, checking the abort flag and the
+// time limit every 16 polls. Inlined (a call cannot cross the register
+// reallocation some kernels do with setmaxnreg).
+__device__ __forceinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity,
+                                                      volatile int* abort_flag,
+                                                      unsigned int* status_word,
+                                                      unsigned long long limit_ns,
+                                                      unsigned int code, bool drain) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0u) {
-      if (!drain && *w.abort_flag) return false;
-      if (global_timer_ns() - t0 > w.limit_ns) {
-        *w.abort_flag = 1;
-        atomicCAS(w.status_word, 0u, (w.kernel_id << 16) | ((site & 0xffu) << 8) | 1u);
+      if (!drain && *abort_flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicCAS(status_word, 0u, code);
         __threadfence();
         return false;
       }
     }
   }
+}
+
+// Waits until the phase with the given parity of `bar` has completed.
+// Returns true on completion; false if this CTA is aborting or the time limit
+// ran out (then the abort flag and the device status word are set). Never
+// spins forever. With `drain` set the abort flag is ignored (used to let
+// copies already in flight land before an aborting CTA exits); the time
+// limit still applies. The first poll is inline; only a phase that is not
+// complete yet pays for the call.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCtl& w,
+                                             uint32_t site, bool drain = false) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bounded_slow(bar, parity, w.abort_flag, w.status_word, w.limit_ns,
+                           (w.kernel_id << 16) | ((site & 0xffu) << 8) | 1u, drain);
 }
 
 // ----------------------------------------------------------------------------
@@ -225,6 +238,45 @@ __device__ __forceinline__ float lg2_approx(float x) {
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// three-input maximum (sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// packed pairs of fp32 (one 64-bit register; .x in the low half) and the
+// sm_100 paired arithmetic on them: one instruction for two lanes of work
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Per-warpgroup register reallocation (all four warps of a warpgroup execute
+// it together). The sum over warpgroups must stay within the registers the
+// block was launched with.
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // two fp32 -> packed bf16x2 (round to nearest even); `lo` in the low half
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

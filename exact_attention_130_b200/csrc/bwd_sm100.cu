@@ -101,37 +101,50 @@ struct Plan {
 };
 
 // --------------------------------------------------------------------------
-// 1. preprocess: one warp per (padded) row
+// 1. preprocess: a row is read by d/8 lanes with 16-byte loads; a warp covers
+//    kPreSteps groups of rows and issues all its loads before using them
 // --------------------------------------------------------------------------
+constexpr int kPreSteps = 4;
+
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
-  constexpr int kPer = D / 32;
-  const long long warp = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  constexpr int kLanesPerRow = D / 8;            // 16 (d = 128) or 8 (d = 64)
+  constexpr int kRowsPerStep = 32 / kLanesPerRow;
+  const long long gwarp = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow, j = lane % kLanesPerRow;
   const long long total = static_cast<long long>(p.BH) * p.Np;
-  if (warp >= total) return;
-  const int bh = int(warp / p.Np);
-  const int row = int(warp % p.Np);
-  float dsum = 0.f;
-  if (row < p.N) {
-    const size_t base = (size_t(bh) * p.N + row) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const uint2 a = *reinterpret_cast<const uint2*>(p.o + base);
-      const uint2 b = *reinterpret_cast<const uint2*>(p.dO + base);
-      dsum = bf16f(a.x & 0xffffu) * bf16f(b.x & 0xffffu) + bf16f(a.x >> 16) * bf16f(b.x >> 16) +
-             bf16f(a.y & 0xffffu) * bf16f(b.y & 0xffffu) + bf16f(a.y >> 16) * bf16f(b.y >> 16);
-    } else {
-      const uint32_t a = *reinterpret_cast<const uint32_t*>(p.o + base);
-      const uint32_t b = *reinterpret_cast<const uint32_t*>(p.dO + base);
-      dsum = bf16f(a & 0xffffu) * bf16f(b & 0xffffu) + bf16f(a >> 16) * bf16f(b >> 16);
-    }
+  const long long row0 = gwarp * kRowsPerStep * kPreSteps;
+  uint4 ov[kPreSteps], gv[kPreSteps];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+  for (int st = 0; st < kPreSteps; ++st) {
+    const long long r = row0 + st * kRowsPerStep + sub;
+    ov[st] = gv[st] = make_uint4(0, 0, 0, 0);
+    if (r < total) {
+      const int bh = int(r / p.Np), row = int(r % p.Np);
+      if (row < p.N) {
+        const size_t off = (size_t(bh) * p.N + row) * D + j * 8;
+        ov[st] = *reinterpret_cast<const uint4*>(p.o + off);
+        gv[st] = *reinterpret_cast<const uint4*>(p.dO + off);
+      }
+    }
   }
-  if (lane == 0) {
-    const size_t o = size_t(bh) * p.Np + row;
-    p.dvec[o] = row < p.N ? dsum : 0.f;
-    p.lse2[o] = row < p.N ? p.lse[size_t(bh) * p.N + row] * kLog2e : INFINITY;
+#pragma unroll
+  for (int st = 0; st < kPreSteps; ++st) {
+    const uint32_t a[4] = {ov[st].x, ov[st].y, ov[st].z, ov[st].w};
+    const uint32_t g[4] = {gv[st].x, gv[st].y, gv[st].z, gv[st].w};
+    float dsum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      dsum += bf16f(a[i] & 0xffffu) * bf16f(g[i] & 0xffffu) + bf16f(a[i] >> 16) * bf16f(g[i] >> 16);
+#pragma unroll
+    for (int off = kLanesPerRow / 2; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+    const long long r = row0 + st * kRowsPerStep + sub;
+    if (j == 0 && r < total) {
+      const int bh = int(r / p.Np), row = int(r % p.Np);
+      p.dvec[r] = row < p.N ? dsum : 0.f;
+      p.lse2[r] = row < p.N ? p.lse[size_t(bh) * p.N + row] * kLog2e : INFINITY;
+    }
   }
 }
 
@@ -609,7 +622,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.limit_ns = ctx.wait_limit_ns;
 
   {
-    const long long warps = (long long)BH * p.Np;
+    const long long rows_per_warp = (32 / (d / 8)) * kPreSteps;
+    const long long warps = ((long long)BH * p.Np + rows_per_warp - 1) / rows_per_warp;
     const long long blocks = (warps * 32 + 255) / 256;
     ProfileScope prof(KID_BWD_PRE, ctx.stream);
     if (d == 128)

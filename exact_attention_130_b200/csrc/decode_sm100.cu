@@ -15,15 +15,15 @@
 // bound is HBM bandwidth, not the tensor cores (a single query row is not a
 // dense contraction). B200 design:
 //  * one CTA per (chunk, head, sequence); a producer warp streams the
-//    chunk's K and V rows into a 4-stage shared-memory ring with plain bulk
-//    copies (cp.async.bulk: the rows of one chunk are contiguous), keeping up
-//    to 64 KB per CTA and ~190 KB per SM in flight;
-//  * four consumer warps take every fourth token of a stage; a lane owns
-//    d/32 consecutive elements of q and of its output accumulator, so a
-//    warp reads one cached row as one contiguous 256-byte line;
-//  * scores of a warp's 8 tokens are formed together and the running
-//    maximum is updated once per 8 tokens, so the exponentials cost about one
-//    per token;
+//    chunk's K and V rows into a 3-stage shared-memory ring with plain bulk
+//    copies (cp.async.bulk: the rows of one chunk are contiguous), up to
+//    96 KB per CTA and two CTAs per SM;
+//  * eight consumer warps; each half-warp owns 4 rows of every 64-row stage
+//    and a lane d/16 elements of q and of the output accumulator, so one
+//    16-byte shared-memory load per lane reads a row;
+//  * the four partial dot products of a half-warp are summed across its 16
+//    lanes together (5 shuffles for 4 rows instead of 4 per row), and the
+//    running maximum moves once per 4 rows;
 //  * positions at or past seqlens[b] are never read;
 //  * all waits are bounded in time (see sm100_ptx.cuh).
 #include <mutex>
@@ -34,23 +34,23 @@
 namespace fa {
 namespace {
 
-constexpr int kTileT = 32;        // cache rows per pipeline stage
-constexpr int kStages = 4;
-constexpr int kConsumerWarps = 4;
+constexpr int kStageTok = 64;     // cache rows per pipeline stage
+constexpr int kStages = 3;
+constexpr int kConsumerWarps = 8;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kTokPerWarp = kTileT / kConsumerWarps;  // 8
+constexpr int kRowsPerHalf = kStageTok / (2 * kConsumerWarps);  // 4
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSmHint = 148;      // B200 SM count, for the automatic split
 
 template <int D>
 struct DecLayout {
-  static constexpr int kTileBytes = kTileT * D * 2;
+  static constexpr int kTileBytes = kStageTok * D * 2;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kStages * kTileBytes;
   static constexpr int kOffBar = 2 * kStages * kTileBytes;       // full[s], empty[s]
   static constexpr int kOffMisc = kOffBar + 8 * 2 * kStages;     // abort flag
-  static constexpr int kOffMerge = kOffMisc + 16;                // per-warp m, l, acc[D]
-  static constexpr int kSmemBytes = kOffMerge + kConsumerWarps * (D + 2) * 4 + 128;
+  static constexpr int kOffMerge = kOffMisc + 16;                // per half-warp m, l, acc[D]
+  static constexpr int kSmemBytes = kOffMerge + 2 * kConsumerWarps * (D + 2) * 4 + 128;
 };
 
 struct DecParams {
@@ -68,13 +68,38 @@ struct DecParams {
   unsigned long long limit_ns;
 };
 
-__device__ __forceinline__ float bf16_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+// kPer bf16 of one cached row (this lane's part) -> fp32
+template <int kPer>
+__device__ __forceinline__ void load_row_part(const uint8_t* row, int j, float (&x)[kPer]) {
+  if constexpr (kPer == 8) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + j * 16);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(ws[i] << 16);
+      x[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+    }
+  } else {
+    const uint2 w = *reinterpret_cast<const uint2*>(row + j * 8);
+    const uint32_t ws[2] = {w.x, w.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      x[2 * i] = __uint_as_float(ws[i] << 16);
+      x[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+    }
+  }
+}
 
+// One CTA per (chunk, head, sequence): a producer warp streams the chunk's
+// K and V rows into a 3-stage ring; each half-warp of the 8 consumer warps
+// owns 4 rows of every 64-row stage. A lane holds d/16 elements of q and of
+// its output accumulator, so one 16-byte shared load per lane reads a whole
+// row per half-warp.
 template <int D>
 __global__ void __launch_bounds__(kThreads)
     decode_split_kernel(const DecParams p) {
   using L = DecLayout<D>;
-  constexpr int kPer = D / 32;  // elements per lane
+  constexpr int kPer = D / 16;  // elements per lane (16 lanes per row)
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
@@ -98,7 +123,7 @@ __global__ void __launch_bounds__(kThreads)
     return;
   }
   const int n_tok = t1 - t0;
-  const int n_tiles = (n_tok + kTileT - 1) / kTileT;
+  const int n_tiles = (n_tok + kStageTok - 1) / kStageTok;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -120,11 +145,11 @@ __global__ void __launch_bounds__(kThreads)
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kStages;
         if (!wait_bounded(EMPTY(s), ((i / kStages) & 1) ^ 1, wc, 1)) break;
-        const int rows = min(kTileT, n_tok - i * kTileT);
+        const int rows = min(kStageTok, n_tok - i * kStageTok);
         const uint32_t bytes = uint32_t(rows) * D * 2;
         mbar_arrive_expect_tx(FULL(s), 2 * bytes);
-        bulk_load(sbase + L::kOffK + s * L::kTileBytes, kb + size_t(i) * kTileT * D, bytes, FULL(s));
-        bulk_load(sbase + L::kOffV + s * L::kTileBytes, vb + size_t(i) * kTileT * D, bytes, FULL(s));
+        bulk_load(sbase + L::kOffK + s * L::kTileBytes, kb + size_t(i) * kStageTok * D, bytes, FULL(s));
+        bulk_load(sbase + L::kOffV + s * L::kTileBytes, vb + size_t(i) * kStageTok * D, bytes, FULL(s));
         ++issued;
       }
       if (*abort_flag)
@@ -135,11 +160,15 @@ __global__ void __launch_bounds__(kThreads)
     }
   } else {
     // ---------------------------------------------------------------- consumers
+    const int half = lane >> 4;   // which of the two rows a step covers
+    const int j = lane & 15;      // this lane's slice of a row
+    // the row whose full score this lane holds after the reduction below
+    const int u_own = 2 * ((j >> 3) & 1) + ((j >> 2) & 1);
     float qv[kPer];
     {
-      const uint16_t* qp = p.q + bh * D + lane * kPer;
+      const uint16_t* qp = p.q + bh * D + j * kPer;
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) qv[i] = bf16_to_f32(qp[i]) * p.scale_log2;
+      for (int i = 0; i < kPer; ++i) qv[i] = __uint_as_float(uint32_t(qp[i]) << 16) * p.scale_log2;
     }
     float m = -INFINITY, l = 0.f, acc[kPer];
 #pragma unroll
@@ -150,92 +179,85 @@ __global__ void __launch_bounds__(kThreads)
       bool ok = wait_bounded(FULL(s), (it / kStages) & 1, wc, 3);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      const int rows = min(kTileT, n_tok - it * kTileT);
+      const int rows = min(kStageTok, n_tok - it * kStageTok);
       const uint8_t* ktile = smem + L::kOffK + s * L::kTileBytes;
       const uint8_t* vtile = smem + L::kOffV + s * L::kTileBytes;
-      float sc[kTokPerWarp];
-      float mx = -INFINITY;
+      // partial q.k of this lane's slice for the half-warp's 4 rows
+      float sc[kRowsPerHalf];
 #pragma unroll
-      for (int u = 0; u < kTokPerWarp; ++u) {
-        const int tt = warp + u * kConsumerWarps;
+      for (int u = 0; u < kRowsPerHalf; ++u) {
+        const int r = warp * 2 * kRowsPerHalf + 2 * u + half;
         float dot = 0.f;
-        if (tt < rows) {
-          const uint16_t* kr = reinterpret_cast<const uint16_t*>(ktile + tt * D * 2) + lane * kPer;
-          if constexpr (kPer == 4) {
-            const uint2 w = *reinterpret_cast<const uint2*>(kr);
-            dot = fmaf(qv[0], bf16_to_f32(w.x & 0xffffu), dot);
-            dot = fmaf(qv[1], bf16_to_f32(w.x >> 16), dot);
-            dot = fmaf(qv[2], bf16_to_f32(w.y & 0xffffu), dot);
-            dot = fmaf(qv[3], bf16_to_f32(w.y >> 16), dot);
-          } else {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(kr);
-            dot = fmaf(qv[0], bf16_to_f32(w & 0xffffu), dot);
-            dot = fmaf(qv[1], bf16_to_f32(w >> 16), dot);
-          }
+        if (r < rows) {
+          float kx[kPer];
+          load_row_part<kPer>(ktile + r * D * 2, j, kx);
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) dot = fmaf(qv[i], kx[i], dot);
         }
         sc[u] = dot;
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-#pragma unroll
-        for (int u = 0; u < kTokPerWarp; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], off);
-      }
-#pragma unroll
-      for (int u = 0; u < kTokPerWarp; ++u) {
-        const int tt = warp + u * kConsumerWarps;
-        if (tt >= rows) sc[u] = -INFINITY;
-        mx = fmaxf(mx, sc[u]);
-      }
-      if (mx != -INFINITY) {
-        const float m_new = fmaxf(m, mx);
+      // sum over the 16 lanes of the half for all 4 rows at once: each
+      // exchange halves the number of rows a lane carries
+      const bool b3 = (j >> 3) & 1, b2 = (j >> 2) & 1;
+      float t0v = b3 ? sc[2] : sc[0], t1v = b3 ? sc[3] : sc[1];
+      t0v += __shfl_xor_sync(0xffffffffu, b3 ? sc[0] : sc[2], 8);
+      t1v += __shfl_xor_sync(0xffffffffu, b3 ? sc[1] : sc[3], 8);
+      float sv = b2 ? t1v : t0v;
+      sv += __shfl_xor_sync(0xffffffffu, b2 ? t0v : t1v, 4);
+      sv += __shfl_xor_sync(0xffffffffu, sv, 2);
+      sv += __shfl_xor_sync(0xffffffffu, sv, 1);
+      const int r_own = warp * 2 * kRowsPerHalf + 2 * u_own + half;
+      const bool valid = r_own < rows;
+      sv = valid ? sv : -INFINITY;
+      float mt = fmaxf(sv, __shfl_xor_sync(0xffffffffu, sv, 4));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+      // warp-uniform (the shuffles below span both halves); a half with no
+      // valid row in this stage keeps its state: alpha = 1 (or 0 before its
+      // first row), p = 0
+      if (__any_sync(0xffffffffu, mt != -INFINITY)) {
+        const float m_new = fmaxf(m, mt);
         const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
         m = m_new;
-        float rs = 0.f;
+        const float pr = valid ? ex2_approx(sv - m) : 0.f;
+        float ps = pr + __shfl_xor_sync(0xffffffffu, pr, 4);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+        l = l * alpha + ps;
 #pragma unroll
         for (int i = 0; i < kPer; ++i) acc[i] *= alpha;
 #pragma unroll
-        for (int u = 0; u < kTokPerWarp; ++u) {
-          const int tt = warp + u * kConsumerWarps;
-          if (tt < rows) {
-            const float pr = ex2_approx(sc[u] - m);
-            rs += pr;
-            const uint16_t* vr =
-                reinterpret_cast<const uint16_t*>(vtile + tt * D * 2) + lane * kPer;
-            if constexpr (kPer == 4) {
-              const uint2 w = *reinterpret_cast<const uint2*>(vr);
-              acc[0] = fmaf(pr, bf16_to_f32(w.x & 0xffffu), acc[0]);
-              acc[1] = fmaf(pr, bf16_to_f32(w.x >> 16), acc[1]);
-              acc[2] = fmaf(pr, bf16_to_f32(w.y & 0xffffu), acc[2]);
-              acc[3] = fmaf(pr, bf16_to_f32(w.y >> 16), acc[3]);
-            } else {
-              const uint32_t w = *reinterpret_cast<const uint32_t*>(vr);
-              acc[0] = fmaf(pr, bf16_to_f32(w & 0xffffu), acc[0]);
-              acc[1] = fmaf(pr, bf16_to_f32(w >> 16), acc[1]);
-            }
+        for (int u = 0; u < kRowsPerHalf; ++u) {
+          // row u's probability sits in lanes with (j>>3, j>>2) = (u>>1, u&1)
+          const float pu = __shfl_sync(0xffffffffu, pr, half * 16 + 8 * (u >> 1) + 4 * (u & 1));
+          const int r = warp * 2 * kRowsPerHalf + 2 * u + half;
+          if (r < rows) {
+            float vx[kPer];
+            load_row_part<kPer>(vtile + r * D * 2, j, vx);
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) acc[i] = fmaf(pu, vx[i], acc[i]);
           }
         }
-        l = l * alpha + rs;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(EMPTY(s));
     }
-    // per-warp state to shared memory for the merge
-    float* mw = merge + warp * (D + 2);
-    if (lane == 0) {
+    // per half-warp state to shared memory for the merge
+    float* mw = merge + (warp * 2 + half) * (D + 2);
+    if (j == 0) {
       mw[0] = m;
       mw[1] = l;
     }
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) mw[2 + lane * kPer + i] = acc[i];
+    for (int i = 0; i < kPer; ++i) mw[2 + j * kPer + i] = acc[i];
   }
   __syncthreads();
   if (*abort_flag) return;
-  // merge the consumer warps (base-2 statistics) into this chunk's partial
+  // merge the 16 half-warp states (base-2 statistics) into this chunk's partial
+  constexpr int kStates = 2 * kConsumerWarps;
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
     float mm = -INFINITY;
-    for (int w = 0; w < kConsumerWarps; ++w) mm = fmaxf(mm, merge[w * (D + 2)]);
+    for (int w = 0; w < kStates; ++w) mm = fmaxf(mm, merge[w * (D + 2)]);
     float ll = 0.f, oo = 0.f;
-    for (int w = 0; w < kConsumerWarps; ++w) {
+    for (int w = 0; w < kStates; ++w) {
       const float mw = merge[w * (D + 2)];
       if (mw == -INFINITY) continue;
       const float f = ex2_approx(mw - mm);

@@ -13,50 +13,59 @@
 //               so their P is exactly 0).
 //  2. bwd_dkdv  one CTA per (batch*head, 128-key tile). K and V of the tile stay
 //               in shared memory; the Q and dO rows of every query that can see
-//               these keys stream past in blocks of 64. Per block:
+//               these keys stream past in blocks of 128. Per block:
 //                 S^T = K Q^T, dP^T = V dO^T          (tcgen05 -> TMEM)
-//                 P^T = 2^(S^T scale log2e - L2),
-//                 dS^T = scale P^T (dP^T - D)        (CUDA cores, one TMEM lane
-//                                                      = one key row)
-//                 dV += P^T dO, dK += dS^T Q          (tcgen05, A from TMEM)
+//                 P^T = 2^(S^T scale log2e - L2)     (phase 1, CUDA cores)
+//                 dV += P^T dO                        (tcgen05, A = P^T in TMEM)
+//                 dS^T = scale P^T (dP^T - D)        (phase 2)
+//                 dK += dS^T Q                        (tcgen05, A = dS^T in TMEM)
 //               dV and dK accumulate in TMEM for the whole key tile.
-//  3. bwd_dq    one CTA per (batch*head, 128-query tile). Q and dO stay in shared
-//               memory; K and V stream past in blocks of 64 keys. Per block:
+//  3. bwd_dq    one CTA per (batch*head, 128-query tile). Q and dO stay in
+//               shared memory; K and V stream past in blocks of 128 keys:
 //                 S = Q K^T, dP = dO V^T; dS = scale P (dP - D); dQ += dS K.
 // The scale is folded into dS before it is rounded to bf16.
 //
 // Splitting dQ from dK/dV recomputes S and dP once more (7 tensor-core GEMMs
-// instead of 5) but needs no atomics and keeps the tensor core busy: in both
-// kernels two compute warpgroups take alternate 64-wide blocks, each with its
-// own S/dP buffer in TMEM, so the exponentials of one block overlap the MMAs of
-// the other (TMEM: buffer 0 | buffer 1 | two 128-column accumulators).
+// instead of 5) but needs no atomics and gives deterministic results. Both
+// kernels use 128-wide blocks, so every MMA is M = 128, N = 128 (the full-rate
+// shape), with one buffer per operand in TMEM; the overlap comes from splitting
+// the per-block CUDA-core work in two phases and issuing each dependent MMA as
+// soon as its phase ends, interleaved with the next block's S and dP MMAs:
+//   dK/dV kernel:  ... dV_i | S^T_i+1 | dK_i | dP^T_i+1 | dV_i+1 ...
+//                  phase 1 of block i+1 (the exponentials) runs during
+//                  dK_i and dP^T_i+1;
+//   dQ kernel:     S_j+1 is issued as soon as S_j has been read into
+//                  registers, so phase 1 of block j+1 starts right after
+//                  phase 2 of block j, during dQ_j and dP_j+1.
 //
-// Warp roles (320 threads): warps 0-3 compute for buffer 0, warps 4-7 for
-// buffer 1, warp 8 TMA producer, warp 9 MMA issuer.
+// Warp roles (192 threads): warps 0-3 compute (one TMEM lane = one row),
+// warp 4 TMA producer, warp 5 MMA issuer. Six warps leave each thread up to 255
+// registers, so a row's 128 probabilities stay in registers between phases.
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace fa {
 namespace {
 
-constexpr int kTile = 128;   // rows of the resident tile (keys or queries)
-constexpr int kSub = 64;     // rows of a streamed block
-constexpr int kThreads = 320;
-constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kStages = 4;
+constexpr int kTile = 128;   // rows of the resident tile and of a streamed block
+constexpr int kThreads = 192;
+constexpr int kLoadWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // barrier slots (shared by both kernels)
 enum : int {
   B_RES_FULL = 0,      // the resident tiles (K,V or Q,dO)
   B_ST_FULL = 1,       // +stage: a streamed block landed
-  B_ST_EMPTY = 5,      // +stage: its MMAs are done
-  B_S_FULL = 9,        // +buffer: S and dP of a block are in TMEM
-  B_P_READY = 11,      // +buffer: P / dS written back to TMEM
-  B_ACC_DONE = 13,
-  B_DRAIN = 14,
-  B_COUNT = 15
+  B_ST_EMPTY = 3,      // +stage: its MMAs are done
+  B_S_FULL = 5,        // S of the current block is in TMEM
+  B_DP_FULL = 6,       // dP of the current block is in TMEM
+  B_PHASE1 = 7,        // dK/dV: P^T written back; dQ: S read into registers
+  B_PHASE2 = 8,        // dS written back to TMEM
+  B_ACC_DONE = 9,
+  B_DRAIN = 10,
+  B_COUNT = 11
 };
 
 struct BwdParams {
@@ -76,28 +85,23 @@ struct BwdParams {
 
 __device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
-// Shared-memory plan. Row-major tiles of bf16 with 128-byte rows, stored as
-// D/64 column groups of rows x 128 bytes, 128-byte swizzled (TMA box 64
-// columns x rows).
+// Shared-memory plan. Row-major bf16 tiles of 128 rows, stored as D/64 column
+// groups of 128 rows x 128 bytes, 128-byte swizzled (TMA box 64 x 128).
 template <int D>
 struct Plan {
   static constexpr int kGroups = D / 64;
-  static constexpr int kResSub = kTile * 128;            // 16 KB per column group
-  static constexpr int kResTile = kGroups * kResSub;      // one resident tile
-  static constexpr int kBlkSub = kSub * 128;              // 8 KB per column group
-  static constexpr int kBlkTile = kGroups * kBlkSub;      // one streamed tile
+  static constexpr int kSubBytes = kTile * 128;        // 16 KB per column group
+  static constexpr int kTileBytes = kGroups * kSubBytes;
   static constexpr int kOffRes0 = 0;
-  static constexpr int kOffRes1 = kResTile;
-  static constexpr int kOffStage = 2 * kResTile;
-  // a stage: two streamed tiles, then (dK/dV kernel) 64 floats of L2 and of D
-  static constexpr int kStageBytes = ((2 * kBlkTile + 512) + 1023) / 1024 * 1024;
+  static constexpr int kOffRes1 = kTileBytes;
+  static constexpr int kOffStage = 2 * kTileBytes;
+  // a stage: two streamed tiles, then (dK/dV kernel) 128 floats of L2 and of D
+  static constexpr int kStageBytes = ((2 * kTileBytes + 1024) + 1023) / 1024 * 1024;
   static constexpr int kOffBar = kOffStage + kStages * kStageBytes;
   static constexpr int kOffMisc = kOffBar + 8 * B_COUNT;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;
-  // TMEM columns: buffer b holds S (64 columns) then dP (64 columns)
-  static constexpr uint32_t kColAcc0 = 256, kColAcc1 = 256 + D;
-  __device__ static constexpr uint32_t col_s(int b) { return b ? 128u : 0u; }
-  __device__ static constexpr uint32_t col_dp(int b) { return b ? 192u : 64u; }
+  // TMEM columns
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
 };
 
 // --------------------------------------------------------------------------
@@ -162,10 +166,10 @@ __device__ __forceinline__ uint32_t setup_cta(uint8_t* smem, int warp, volatile 
       mbar_init(bar(B_ST_FULL + s), 1);
       mbar_init(bar(B_ST_EMPTY + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(B_S_FULL + b), 1);
-      mbar_init(bar(B_P_READY + b), 4);
-    }
+    mbar_init(bar(B_S_FULL), 1);
+    mbar_init(bar(B_DP_FULL), 1);
+    mbar_init(bar(B_PHASE1), 4);  // one arrival per compute warp
+    mbar_init(bar(B_PHASE2), 4);
     mbar_init(bar(B_ACC_DONE), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -181,30 +185,29 @@ __device__ __forceinline__ uint32_t setup_cta(uint8_t* smem, int warp, volatile 
   return *tmem_slot;
 }
 
-// MMA of one streamed block against a resident tile, both K-major operands:
-// D[128 x 64] = R[128 x D] * B[64 x D]^T
+// D[128 x 128] = R[128 x D] * B[128 x D]^T, both K-major in shared memory
 template <int D>
-__device__ __forceinline__ void mma_rows_x_block(uint32_t d_tmem, uint32_t res, uint32_t blk) {
+__device__ __forceinline__ void mma_rows_x_rows(uint32_t d_tmem, uint32_t r, uint32_t b) {
   using L = Plan<D>;
-  constexpr uint32_t idesc = idesc_bf16(kTile, kSub, false, false);
+  constexpr uint32_t idesc = idesc_bf16(kTile, kTile, false, false);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t ra = res + (kk >> 2) * L::kResSub + (kk & 3) * 32;
-    const uint32_t rb = blk + (kk >> 2) * L::kBlkSub + (kk & 3) * 32;
-    mma_ss(d_tmem, sdesc_sw128(ra, 16, 1024), sdesc_sw128(rb, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+    const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
+    mma_ss(d_tmem, sdesc_sw128(r + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), idesc,
+           kk > 0 ? 1u : 0u);
   }
 }
 
-// Accumulating MMA with A (128 x 64, bf16) in TMEM and B a streamed block of
-// 64 rows x D read MN-major: D[128 x D] += A * B
+// D[128 x D] (+)= A[128 x 128] * B[128 x D]: A bf16 in TMEM (K-major, 64
+// columns), B a tile in shared memory read MN-major
 template <int D>
-__device__ __forceinline__ void mma_tmem_x_block(uint32_t d_tmem, uint32_t a_tmem, uint32_t blk,
-                                                 bool accumulate) {
+__device__ __forceinline__ void mma_tmem_x_rows(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
+                                                bool accumulate) {
   using L = Plan<D>;
   constexpr uint32_t idesc = idesc_bf16(kTile, D, false, true);
 #pragma unroll
-  for (int kk = 0; kk < kSub / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(blk + kk * 2048, L::kBlkSub, 1024), idesc,
+  for (int kk = 0; kk < kTile / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b + kk * 2048, L::kSubBytes, 1024), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -229,13 +232,39 @@ __device__ __forceinline__ void store_acc_row(uint32_t t_acc, uint16_t* dst, boo
   }
 }
 
+// dS = scale P (dP - D) for a row of 128, with dP read from TMEM 32 columns at
+// a time and dS written back as bf16 over the first 64 of those columns.
+// dvals(i) gives D for column i (a per-column vector in the dK/dV kernel, one
+// value per row in the dQ kernel).
+template <typename DFn>
+__device__ __forceinline__ void write_ds_row(uint32_t t_dp, const float (&pr)[128], float scale,
+                                             DFn dvals) {
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    uint32_t dr[32];
+    tmem_ld32_wait(t_dp + ch * 32, dr);
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c0 = ch * 32 + 2 * i;
+      const float a = pr[c0] * scale * (__uint_as_float(dr[2 * i]) - dvals(c0));
+      const float b = pr[c0 + 1] * scale * (__uint_as_float(dr[2 * i + 1]) - dvals(c0 + 1));
+      pk[i] = pack_bf16x2(a, b);
+    }
+    // columns ch*16 .. ch*16+15 hold the bf16 pairs of dS columns ch*32 ..
+    // ch*32+31; the dP columns they overwrite were read in earlier chunks or
+    // in this one
+    tmem_st16(t_dp + ch * 16, pk);
+  }
+}
+
 // --------------------------------------------------------------------------
 // 2. dK, dV: key-tile-outer
 // --------------------------------------------------------------------------
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ64, const __grid_constant__ CUtensorMap tmDO64,
-                    const __grid_constant__ CUtensorMap tmK128, const __grid_constant__ CUtensorMap tmV128,
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const BwdParams p) {
   using L = Plan<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -247,34 +276,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   // key tiles that see the most query blocks first, all heads of a level together
   const int jt = blockIdx.x / p.BH;
   const int bh = blockIdx.x % p.BH;
-  const int q_start = CAUSAL ? jt * kTile : 0;
-  const int n_blk = (p.N - q_start + kSub - 1) / kSub;
+  const int i0 = CAUSAL ? jt : 0;       // first query tile that sees these keys
+  const int n_blk = p.n_tiles - i0;
   volatile int* abort_flag;
   const uint32_t tmem = setup_cta<D>(smem, warp, abort_flag);
   const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_BWD};
   const uint32_t sK = sbase + L::kOffRes0, sV = sbase + L::kOffRes1;
+  auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
 
   if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued = 0;
-      mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kResTile);
+      mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
       for (int c = 0; c < L::kGroups; ++c) {
-        tma_load_3d(sK + c * L::kResSub, &tmK128, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
-        tma_load_3d(sV + c * L::kResSub, &tmV128, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
+        tma_load_3d(sK + c * L::kSubBytes, &tmK, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
+        tma_load_3d(sV + c * L::kSubBytes, &tmV, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
       }
       for (int it = 0; it < n_blk; ++it) {
         const int s = it % kStages;
         if (!wait_bounded(BAR(B_ST_EMPTY + s), ((it / kStages) & 1) ^ 1, wc, 1)) break;
-        const int q0 = q_start + it * kSub;
-        const uint32_t st = sbase + L::kOffStage + s * L::kStageBytes;
-        mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kBlkTile + 512);
+        const int q0 = (i0 + it) * kTile;
+        const uint32_t st = stage_addr(it);
+        mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kTileBytes + 1024);
         for (int c = 0; c < L::kGroups; ++c) {
-          tma_load_3d(st + c * L::kBlkSub, &tmQ64, BAR(B_ST_FULL + s), c * 64, q0, bh);
-          tma_load_3d(st + L::kBlkTile + c * L::kBlkSub, &tmDO64, BAR(B_ST_FULL + s), c * 64, q0, bh);
+          tma_load_3d(st + c * L::kSubBytes, &tmQ, BAR(B_ST_FULL + s), c * 64, q0, bh);
+          tma_load_3d(st + L::kTileBytes + c * L::kSubBytes, &tmDO, BAR(B_ST_FULL + s), c * 64, q0, bh);
         }
         const size_t vo = size_t(bh) * p.Np + q0;
-        bulk_load(st + 2 * L::kBlkTile, p.lse2 + vo, 256, BAR(B_ST_FULL + s));
-        bulk_load(st + 2 * L::kBlkTile + 256, p.dvec + vo, 256, BAR(B_ST_FULL + s));
+        bulk_load(st + 2 * L::kTileBytes, p.lse2 + vo, 512, BAR(B_ST_FULL + s));
+        bulk_load(st + 2 * L::kTileBytes + 512, p.dvec + vo, 512, BAR(B_ST_FULL + s));
         ++issued;
       }
       if (*abort_flag) {
@@ -286,109 +317,111 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    // order per block i: dV_i (after phase 1), S^T_i+1, dK_i (after phase 2),
+    // dP^T_i+1; the in-order tensor pipe makes each overwrite of the S or dP
+    // columns wait for the MMA that reads the old contents
     if (lane == 0) {
-      auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
-      auto issue_sdp = [&](int it) {  // S^T and dP^T of block `it` into buffer it&1
-        const int b = it & 1;
-        const uint32_t st = stage_addr(it);
-        mma_rows_x_block<D>(tmem + L::col_s(b), sK, st);
-        mma_rows_x_block<D>(tmem + L::col_dp(b), sV, st + L::kBlkTile);
-        tc_commit(BAR(B_S_FULL + b));
-      };
       bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
-      for (int it = 0; ok && it < 2 && it < n_blk; ++it) {
-        ok = wait_bounded(BAR(B_ST_FULL + it % kStages), (it / kStages) & 1, wc, 11);
-        if (!ok) break;
+      if (ok) ok = wait_bounded(BAR(B_ST_FULL + 0), 0, wc, 11);
+      if (ok) {
         tc_fence_after();
-        issue_sdp(it);
+        mma_rows_x_rows<D>(tmem + L::kColS, sK, stage_addr(0));                    // S^T_0
+        tc_commit(BAR(B_S_FULL));
+        mma_rows_x_rows<D>(tmem + L::kColDP, sV, stage_addr(0) + L::kTileBytes);   // dP^T_0
+        tc_commit(BAR(B_DP_FULL));
       }
       for (int it = 0; ok && it < n_blk; ++it) {
-        const int b = it & 1;
-        ok = wait_bounded(BAR(B_P_READY + b), (it >> 1) & 1, wc, 12);
+        const uint32_t st = stage_addr(it);
+        ok = wait_bounded(BAR(B_PHASE1), it & 1, wc, 12);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t st = stage_addr(it);
-        mma_tmem_x_block<D>(tmem + L::kColAcc0, tmem + L::col_s(b), st + L::kBlkTile, it > 0);  // dV += P^T dO
-        mma_tmem_x_block<D>(tmem + L::kColAcc1, tmem + L::col_dp(b), st, it > 0);               // dK += dS^T Q
-        tc_commit(BAR(B_ST_EMPTY + it % kStages));
-        if (it + 2 < n_blk) {
-          ok = wait_bounded(BAR(B_ST_FULL + (it + 2) % kStages), ((it + 2) / kStages) & 1, wc, 13);
+        mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColS, st + L::kTileBytes, it > 0);  // dV += P^T dO
+        if (it + 1 < n_blk) {
+          ok = wait_bounded(BAR(B_ST_FULL + (it + 1) % kStages), ((it + 1) / kStages) & 1, wc, 13);
           if (!ok) break;
           tc_fence_after();
-          issue_sdp(it + 2);
+          mma_rows_x_rows<D>(tmem + L::kColS, sK, stage_addr(it + 1));             // S^T_i+1
+          tc_commit(BAR(B_S_FULL));
+        }
+        ok = wait_bounded(BAR(B_PHASE2), it & 1, wc, 14);
+        if (!ok) break;
+        tc_fence_after();
+        mma_tmem_x_rows<D>(tmem + L::kColAcc1, tmem + L::kColDP, st, it > 0);  // dK += dS^T Q
+        tc_commit(BAR(B_ST_EMPTY + it % kStages));
+        if (it + 1 < n_blk) {
+          mma_rows_x_rows<D>(tmem + L::kColDP, sV, stage_addr(it + 1) + L::kTileBytes);  // dP^T_i+1
+          tc_commit(BAR(B_DP_FULL));
         }
       }
       tc_commit(BAR(B_ACC_DONE));
       tc_commit(BAR(B_DRAIN));
-      wait_bounded(BAR(B_DRAIN), 0, wc, 14, true);
+      wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
     }
   } else {
-    // ------------------------------------------------------------ compute warpgroups
-    const int b = warp >> 2;          // buffer of this warpgroup
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;   // key row in the tile
+    // ------------------------------------------------------------ compute warps
+    const int r = warp * 32 + lane;   // key row in the tile
     const int key = jt * kTile + r;
     const bool row_valid = key < p.N;
-    const uint32_t lane_base = uint32_t(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_base + L::col_s(b);
-    const uint32_t tDP = tmem + lane_base + L::col_dp(b);
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_base + L::kColS;
+    const uint32_t tDP = tmem + lane_base + L::kColDP;
     const float c = p.scale_log2;
     bool ok = true;
-    for (int it = b; it < n_blk; it += 2) {
-      ok = wait_bounded(BAR(B_S_FULL + b), (it >> 1) & 1, wc, 20);
+    for (int it = 0; it < n_blk; ++it) {
+      ok = wait_bounded(BAR(B_S_FULL), it & 1, wc, 20);
       if (ok) ok = wait_bounded(BAR(B_ST_FULL + it % kStages), (it / kStages) & 1, wc, 21);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int q0 = q_start + it * kSub;
-      const float* l2 = reinterpret_cast<const float*>(smem + L::kOffStage + (it % kStages) * L::kStageBytes +
-                                                       2 * L::kBlkTile);
-      const float* dd = l2 + 64;
+      const int q0 = (i0 + it) * kTile;
+      const float* l2 = reinterpret_cast<const float*>(smem + L::kOffStage +
+                                                       (it % kStages) * L::kStageBytes + 2 * L::kTileBytes);
+      const float* dd = l2 + kTile;
       // queries q0 + i with i < qmask are hidden from this key (causal)
-      const int qmask = CAUSAL ? min(max(key - q0, 0), kSub) : 0;
-      uint32_t sr[64];
-      tmem_ld64_wait(tS, sr);
-      float pr[64];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float x = ex2_approx(fmaf(__uint_as_float(sr[i]), c, -l2[i]));
-        pr[i] = (row_valid && i >= qmask) ? x : 0.f;
-      }
+      const int qmask = CAUSAL ? min(max(key - q0, 0), kTile) : 0;
+      // phase 1: P^T row = 2^(s c - L2_q), written back over S^T as bf16
+      float pr[128];
       {
-        uint32_t pk[32];
+        uint32_t sr[128];
+        tmem_ld128_wait(tS, sr);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
-        tmem_st32(tS, pk);  // P^T over the first 32 columns of S^T
-      }
-      uint32_t dr[64];
-      tmem_ld64_wait(tDP, dr);
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float a = pr[2 * i] * p.scale * (__uint_as_float(dr[2 * i]) - dd[2 * i]);
-          const float e = pr[2 * i + 1] * p.scale * (__uint_as_float(dr[2 * i + 1]) - dd[2 * i + 1]);
-          pk[i] = pack_bf16x2(a, e);
+        for (int i = 0; i < 128; ++i) {
+          const float x = ex2_approx(fmaf(__uint_as_float(sr[i]), c, -l2[i]));
+          pr[i] = (row_valid && i >= qmask) ? x : 0.f;
         }
-        tmem_st32(tDP, pk);  // dS^T over the first 32 columns of dP^T
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[64 * h + 2 * i], pr[64 * h + 2 * i + 1]);
+        tmem_st32(tS + 32 * h, pk);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_P_READY + b));
+      if (lane == 0) mbar_arrive(BAR(B_PHASE1));
+      // phase 2: dS^T row = scale P^T (dP^T - D_q), written back over dP^T
+      ok = wait_bounded(BAR(B_DP_FULL), it & 1, wc, 22);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      write_ds_row(tDP, pr, p.scale, [&](int i) { return dd[i]; });
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_PHASE2));
     }
-    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK
     if (ok) {
-      ok = wait_bounded(BAR(B_ACC_DONE), 0, wc, 22);
+      ok = wait_bounded(BAR(B_ACC_DONE), 0, wc, 23);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
       tc_fence_after();
       const size_t gro = (size_t(bh) * p.N + key) * D;
-      if (b == 0)
-        store_acc_row<D>(tmem + lane_base + L::kColAcc0, p.dv + gro, row_valid);
-      else
-        store_acc_row<D>(tmem + lane_base + L::kColAcc1, p.dk + gro, row_valid);
+      store_acc_row<D>(tmem + lane_base + L::kColAcc0, p.dv + gro, row_valid);
+      store_acc_row<D>(tmem + lane_base + L::kColAcc1, p.dk + gro, row_valid);
     }
   }
 
@@ -405,8 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // --------------------------------------------------------------------------
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ128, const __grid_constant__ CUtensorMap tmDO128,
-                  const __grid_constant__ CUtensorMap tmK64, const __grid_constant__ CUtensorMap tmV64,
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const BwdParams p) {
   using L = Plan<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -419,29 +452,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lvl = blockIdx.x / p.BH;
   const int it_q = CAUSAL ? p.n_tiles - 1 - lvl : lvl;
   const int bh = blockIdx.x % p.BH;
-  const int k_end = CAUSAL ? min(p.N, (it_q + 1) * kTile) : p.N;
-  const int n_blk = (k_end + kSub - 1) / kSub;
+  const int n_blk = CAUSAL ? it_q + 1 : p.n_tiles;  // key tiles this query tile sees
   volatile int* abort_flag;
   const uint32_t tmem = setup_cta<D>(smem, warp, abort_flag);
   const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_BWD_DQ};
   const uint32_t sQ = sbase + L::kOffRes0, sDO = sbase + L::kOffRes1;
+  auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
 
   if (warp == kLoadWarp) {
     if (lane == 0) {
       int issued = 0;
-      mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kResTile);
+      mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
       for (int c = 0; c < L::kGroups; ++c) {
-        tma_load_3d(sQ + c * L::kResSub, &tmQ128, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
-        tma_load_3d(sDO + c * L::kResSub, &tmDO128, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
+        tma_load_3d(sQ + c * L::kSubBytes, &tmQ, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
+        tma_load_3d(sDO + c * L::kSubBytes, &tmDO, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
       }
       for (int it = 0; it < n_blk; ++it) {
         const int s = it % kStages;
         if (!wait_bounded(BAR(B_ST_EMPTY + s), ((it / kStages) & 1) ^ 1, wc, 1)) break;
-        const uint32_t st = sbase + L::kOffStage + s * L::kStageBytes;
-        mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kBlkTile);
+        const uint32_t st = stage_addr(it);
+        mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kTileBytes);
         for (int c = 0; c < L::kGroups; ++c) {
-          tma_load_3d(st + c * L::kBlkSub, &tmK64, BAR(B_ST_FULL + s), c * 64, it * kSub, bh);
-          tma_load_3d(st + L::kBlkTile + c * L::kBlkSub, &tmV64, BAR(B_ST_FULL + s), c * 64, it * kSub, bh);
+          tma_load_3d(st + c * L::kSubBytes, &tmK, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
+          tma_load_3d(st + L::kTileBytes + c * L::kSubBytes, &tmV, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
         }
         ++issued;
       }
@@ -454,86 +487,89 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
+    // order per block j: S_j+1 (once S_j is in registers), dQ_j (after
+    // phase 2), dP_j+1
     if (lane == 0) {
-      auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
-      auto issue_sdp = [&](int it) {  // S and dP of key block `it` into buffer it&1
-        const int b = it & 1;
-        const uint32_t st = stage_addr(it);
-        mma_rows_x_block<D>(tmem + L::col_s(b), sQ, st);
-        mma_rows_x_block<D>(tmem + L::col_dp(b), sDO, st + L::kBlkTile);
-        tc_commit(BAR(B_S_FULL + b));
-      };
       bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
-      for (int it = 0; ok && it < 2 && it < n_blk; ++it) {
-        ok = wait_bounded(BAR(B_ST_FULL + it % kStages), (it / kStages) & 1, wc, 11);
-        if (!ok) break;
+      if (ok) ok = wait_bounded(BAR(B_ST_FULL + 0), 0, wc, 11);
+      if (ok) {
         tc_fence_after();
-        issue_sdp(it);
+        mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(0));                     // S_0
+        tc_commit(BAR(B_S_FULL));
+        mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(0) + L::kTileBytes);   // dP_0
+        tc_commit(BAR(B_DP_FULL));
       }
       for (int it = 0; ok && it < n_blk; ++it) {
-        const int b = it & 1;
-        ok = wait_bounded(BAR(B_P_READY + b), (it >> 1) & 1, wc, 12);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tmem_x_block<D>(tmem + L::kColAcc0, tmem + L::col_dp(b), stage_addr(it), it > 0);  // dQ += dS K
-        tc_commit(BAR(B_ST_EMPTY + it % kStages));
-        if (it + 2 < n_blk) {
-          ok = wait_bounded(BAR(B_ST_FULL + (it + 2) % kStages), ((it + 2) / kStages) & 1, wc, 13);
+        if (it + 1 < n_blk) {
+          ok = wait_bounded(BAR(B_PHASE1), it & 1, wc, 12);
+          if (ok) ok = wait_bounded(BAR(B_ST_FULL + (it + 1) % kStages), ((it + 1) / kStages) & 1, wc, 13);
           if (!ok) break;
           tc_fence_after();
-          issue_sdp(it + 2);
+          mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(it + 1));              // S_j+1
+          tc_commit(BAR(B_S_FULL));
+        }
+        ok = wait_bounded(BAR(B_PHASE2), it & 1, wc, 14);
+        if (!ok) break;
+        tc_fence_after();
+        mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColDP, stage_addr(it), it > 0);  // dQ += dS K
+        tc_commit(BAR(B_ST_EMPTY + it % kStages));
+        if (it + 1 < n_blk) {
+          mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(it + 1) + L::kTileBytes);  // dP_j+1
+          tc_commit(BAR(B_DP_FULL));
         }
       }
       tc_commit(BAR(B_ACC_DONE));
       tc_commit(BAR(B_DRAIN));
-      wait_bounded(BAR(B_DRAIN), 0, wc, 14, true);
+      wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
     }
   } else {
-    const int b = warp >> 2;
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;   // query row in the tile
+    const int r = warp * 32 + lane;   // query row in the tile
     const int q = it_q * kTile + r;
-    const uint32_t lane_base = uint32_t(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_base + L::col_s(b);
-    const uint32_t tDP = tmem + lane_base + L::col_dp(b);
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_base + L::kColS;
+    const uint32_t tDP = tmem + lane_base + L::kColDP;
     const float c = p.scale_log2;
-    const float l2q = p.lse2[size_t(bh) * p.Np + it_q * kTile + r];  // +inf past N
-    const float dq_ = p.dvec[size_t(bh) * p.Np + it_q * kTile + r];
+    const float l2q = p.lse2[size_t(bh) * p.Np + q];  // +inf past N (q < Np always)
+    const float dq_ = p.dvec[size_t(bh) * p.Np + q];
     bool ok = true;
-    for (int it = b; it < n_blk; it += 2) {
-      ok = wait_bounded(BAR(B_S_FULL + b), (it >> 1) & 1, wc, 20);
+    for (int it = 0; it < n_blk; ++it) {
+      ok = wait_bounded(BAR(B_S_FULL), it & 1, wc, 20);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int k0 = it * kSub;
+      const int k0 = it * kTile;
       // keys k0 + i with i >= klim are hidden (causal: key > q; or key >= N)
       int klim = p.N - k0;
       if (CAUSAL) klim = min(klim, q - k0 + 1);
-      klim = max(min(klim, kSub), 0);
-      uint32_t sr[64];
-      tmem_ld64_wait(tS, sr);
-      uint32_t dr[64];
-      tmem_ld64_wait(tDP, dr);
-      uint32_t pk[32];
+      klim = max(min(klim, kTile), 0);
+      // phase 1: read S (then the MMA may overwrite it) and form P
+      uint32_t sr[128];
+      tmem_ld128_wait(tS, sr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_PHASE1));
+      float pr[128];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), c, -l2q));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), c, -l2q));
-        const float a = (2 * i < klim) ? p0 * p.scale * (__uint_as_float(dr[2 * i]) - dq_) : 0.f;
-        const float e = (2 * i + 1 < klim) ? p1 * p.scale * (__uint_as_float(dr[2 * i + 1]) - dq_) : 0.f;
-        pk[i] = pack_bf16x2(a, e);
+      for (int i = 0; i < 128; ++i) {
+        const float x = ex2_approx(fmaf(__uint_as_float(sr[i]), c, -l2q));
+        pr[i] = (i < klim) ? x : 0.f;
       }
-      tmem_st32(tDP, pk);  // dS over the first 32 columns of dP
+      // phase 2: dS = scale P (dP - D_q), written back over dP as bf16
+      ok = wait_bounded(BAR(B_DP_FULL), it & 1, wc, 21);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      write_ds_row(tDP, pr, p.scale, [&](int) { return dq_; });
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_P_READY + b));
+      if (lane == 0) mbar_arrive(BAR(B_PHASE2));
     }
     if (ok) {
       ok = wait_bounded(BAR(B_ACC_DONE), 0, wc, 22);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok && b == 0) {
+    if (ok) {
       tc_fence_after();
       store_acc_row<D>(tmem + lane_base + L::kColAcc0, p.dq + (size_t(bh) * p.N + q) * D, q < p.N);
     }
@@ -569,19 +605,14 @@ fa_status launch_all(const void* q, const void* k, const void* v, const void* dO
   const int smem = Plan<D>::kSmemBytes;
   const unsigned grid = unsigned(p.n_tiles) * unsigned(p.BH);
   CUtensorMap m[4];
-  fa_status st;
-  // dK/dV: queries and dO stream in blocks of 64 rows, K and V tiles of 128
-  if ((st = make_tmap_3d(&m[0], q, true, D, p.N, p.BH, 64, kSub, true)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&m[1], dO, true, D, p.N, p.BH, 64, kSub, true)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&m[2], k, true, D, p.N, p.BH, 64, kTile, true)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&m[3], v, true, D, p.N, p.BH, 64, kTile, true)) != FA_OK) return st;
-  st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid, m, p, ctx, "bwd dK/dV kernel");
+  const void* src[4] = {q, dO, k, v};
+  for (int i = 0; i < 4; ++i) {
+    fa_status st = make_tmap_3d(&m[i], src[i], true, D, p.N, p.BH, 64, kTile, true);
+    if (st != FA_OK) return st;
+  }
+  fa_status st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid, m, p, ctx,
+                             "bwd dK/dV kernel");
   if (st != FA_OK) return st;
-  // dQ: Q and dO tiles of 128 rows, K and V stream in blocks of 64
-  if ((st = make_tmap_3d(&m[0], q, true, D, p.N, p.BH, 64, kTile, true)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&m[1], dO, true, D, p.N, p.BH, 64, kTile, true)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&m[2], k, true, D, p.N, p.BH, 64, kSub, true)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&m[3], v, true, D, p.N, p.BH, 64, kSub, true)) != FA_OK) return st;
   return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid, m, p, ctx, "bwd dQ kernel");
 }
 

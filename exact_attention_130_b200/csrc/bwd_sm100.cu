@@ -8,16 +8,18 @@
 // so neither S nor P (nor dS) is ever stored.
 //
 // Three kernels on the caller's stream:
-//  1. bwd_pre   D_i = sum_c dO_ic O_ic (fp32) and the saved LSE in base 2, both
-//               padded to a multiple of 128 rows (padding rows get LSE = +inf,
-//               so their P is exactly 0).
+//  1. bwd_pre   D_i = sum_c dO_ic O_ic (fp32) and the saved LSE in base 2,
+//               stored negated and D pre-multiplied by -scale (the forms the
+//               paired FMAs of the main kernels add), both padded to a
+//               multiple of 128 rows (padding rows get -L2 = -inf, so their P
+//               is exactly 0, and -scale D = 0).
 //  2. bwd_dkdv  one CTA per (batch*head, 128-key tile). K and V of the tile stay
 //               in shared memory; the Q and dO rows of every query that can see
 //               these keys stream past in blocks of 128. Per block:
 //                 S^T = K Q^T, dP^T = V dO^T          (tcgen05 -> TMEM)
 //                 P^T = 2^(S^T scale log2e - L2)     (phase 1, CUDA cores)
 //                 dV += P^T dO                        (tcgen05, A = P^T in TMEM)
-//                 dS^T = scale P^T (dP^T - D)        (phase 2)
+//                 dS^T = P^T (scale dP^T - scale D)  (phase 2)
 //                 dK += dS^T Q                        (tcgen05, A = dS^T in TMEM)
 //               dV and dK accumulate in TMEM for the whole key tile.
 //  3. bwd_dq    one CTA per (batch*head, 128-query tile). Q and dO stay in
@@ -38,9 +40,13 @@
 //                  registers, so phase 1 of block j+1 starts right after
 //                  phase 2 of block j, during dQ_j and dP_j+1.
 //
-// Warp roles (192 threads): warps 0-3 compute (one TMEM lane = one row),
-// warp 4 TMA producer, warp 5 MMA issuer. Six warps leave each thread up to 255
-// registers, so a row's 128 probabilities stay in registers between phases.
+// Warp roles (320 threads): warps 0-7 compute, warp 8 TMA producer, warp 9 MMA
+// issuer. A row (one TMEM lane) is shared by two compute warps of the same lane
+// quadrant, warp w taking columns 0-63 and warp w+4 columns 64-127, so each
+// thread keeps 64 probabilities in registers between the phases and two warps
+// per SMSP hide each other's latencies. Each half writes its bf16 P or dS
+// inside its own 64 columns, so the A operand of the K-step kk of the next MMA
+// starts at column (kk/4)*64 + (kk%4)*8.
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -48,9 +54,11 @@ namespace fa {
 namespace {
 
 constexpr int kTile = 128;   // rows of the resident tile and of a streamed block
-constexpr int kThreads = 192;
-constexpr int kLoadWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kComputeWarps = 8;
+constexpr int kHalfCols = kTile / 2;  // columns of a row each compute warp owns
 constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -72,8 +80,8 @@ struct BwdParams {
   const uint16_t* o;
   const uint16_t* dO;
   const float* lse;
-  float* lse2;     // [BH, Np] base-2 LSE, +inf in padding rows
-  float* dvec;     // [BH, Np] D, 0 in padding rows
+  float* lse2;     // [BH, Np] minus the base-2 LSE, -inf in padding rows
+  float* dvec;     // [BH, Np] -scale D, 0 in padding rows
   uint16_t* dq;
   uint16_t* dk;
   uint16_t* dv;
@@ -146,8 +154,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     const long long r = row0 + st * kRowsPerStep + sub;
     if (j == 0 && r < total) {
       const int bh = int(r / p.Np), row = int(r % p.Np);
-      p.dvec[r] = row < p.N ? dsum : 0.f;
-      p.lse2[r] = row < p.N ? p.lse[size_t(bh) * p.N + row] * kLog2e : INFINITY;
+      p.dvec[r] = row < p.N ? -p.scale * dsum : 0.f;
+      p.lse2[r] = row < p.N ? -p.lse[size_t(bh) * p.N + row] * kLog2e : -INFINITY;
     }
   }
 }
@@ -168,8 +176,8 @@ __device__ __forceinline__ uint32_t setup_cta(uint8_t* smem, int warp, volatile 
     }
     mbar_init(bar(B_S_FULL), 1);
     mbar_init(bar(B_DP_FULL), 1);
-    mbar_init(bar(B_PHASE1), 4);  // one arrival per compute warp
-    mbar_init(bar(B_PHASE2), 4);
+    mbar_init(bar(B_PHASE1), kComputeWarps);  // one arrival per compute warp
+    mbar_init(bar(B_PHASE2), kComputeWarps);
     mbar_init(bar(B_ACC_DONE), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -198,8 +206,9 @@ __device__ __forceinline__ void mma_rows_x_rows(uint32_t d_tmem, uint32_t r, uin
   }
 }
 
-// D[128 x D] (+)= A[128 x 128] * B[128 x D]: A bf16 in TMEM (K-major, 64
-// columns), B a tile in shared memory read MN-major
+// D[128 x D] (+)= A[128 x 128] * B[128 x D]: A bf16 in TMEM, K-major, its two
+// halves at columns 0-31 and 64-95 of a 128-column region (see the warp roles
+// above); B a tile in shared memory read MN-major
 template <int D>
 __device__ __forceinline__ void mma_tmem_x_rows(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
                                                 bool accumulate) {
@@ -207,15 +216,18 @@ __device__ __forceinline__ void mma_tmem_x_rows(uint32_t d_tmem, uint32_t a_tmem
   constexpr uint32_t idesc = idesc_bf16(kTile, D, false, true);
 #pragma unroll
   for (int kk = 0; kk < kTile / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b + kk * 2048, L::kSubBytes, 1024), idesc,
+    mma_ts(d_tmem, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8, sdesc_sw128(b + kk * 2048, L::kSubBytes, 1024), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// bf16 row of a TMEM accumulator (this thread's lane) -> global
-template <int D>
-__device__ __forceinline__ void store_acc_row(uint32_t t_acc, uint16_t* dst, bool valid) {
+// columns [c0, c0 + NC) of a TMEM accumulator row (this thread's lane) -> bf16
+// in global memory
+template <int NC>
+__device__ __forceinline__ void store_acc_cols(uint32_t t_acc, uint16_t* dst, int c0, bool valid) {
+  t_acc += c0;
+  dst += c0;
 #pragma unroll
-  for (int ch = 0; ch < D / 32; ++ch) {
+  for (int ch = 0; ch < NC / 32; ++ch) {
     uint32_t v[32];
     tmem_ld32_wait(t_acc + ch * 32, v);
     if (valid) {
@@ -232,29 +244,62 @@ __device__ __forceinline__ void store_acc_row(uint32_t t_acc, uint16_t* dst, boo
   }
 }
 
-// dS = scale P (dP - D) for a row of 128, with dP read from TMEM 32 columns at
-// a time and dS written back as bf16 over the first 64 of those columns.
-// dvals(i) gives D for column i (a per-column vector in the dK/dV kernel, one
-// value per row in the dQ kernel).
-template <typename DFn>
-__device__ __forceinline__ void write_ds_row(uint32_t t_dp, const float (&pr)[128], float scale,
-                                             DFn dvals) {
+// dS = P (scale dP - scale D) for this warp's 64 columns of a row, in paired
+// fp32 arithmetic: dP read from TMEM 32 columns at a time, dS written back as
+// bf16 over the first 32 of the 64 (chunk 1 overwrites columns chunk 0 has
+// already read). nsd4(j) gives -scale D for local columns 4j..4j+3 (a
+// per-column vector in the dK/dV kernel, one value per row in the dQ kernel).
+template <typename NsdFn>
+__device__ __forceinline__ void write_ds_half(uint32_t t_dp, const uint64_t (&pr2)[kHalfCols / 2], uint64_t scale2,
+                                              NsdFn nsd4) {
 #pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
+  for (int ch = 0; ch < 2; ++ch) {
     uint32_t dr[32];
     tmem_ld32_wait(t_dp + ch * 32, dr);
     uint32_t pk[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int c0 = ch * 32 + 2 * i;
-      const float a = pr[c0] * scale * (__uint_as_float(dr[2 * i]) - dvals(c0));
-      const float b = pr[c0 + 1] * scale * (__uint_as_float(dr[2 * i + 1]) - dvals(c0 + 1));
-      pk[i] = pack_bf16x2(a, b);
+    for (int j = 0; j < 8; ++j) {
+      const float4 n = nsd4(ch * 8 + j);
+      const uint64_t t0 = f2_fma(f2_pack(__uint_as_float(dr[4 * j]), __uint_as_float(dr[4 * j + 1])), scale2,
+                                 f2_pack(n.x, n.y));
+      const uint64_t t1 = f2_fma(f2_pack(__uint_as_float(dr[4 * j + 2]), __uint_as_float(dr[4 * j + 3])), scale2,
+                                 f2_pack(n.z, n.w));
+      pk[2 * j] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j], t0));
+      pk[2 * j + 1] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j + 1], t1));
     }
-    // columns ch*16 .. ch*16+15 hold the bf16 pairs of dS columns ch*32 ..
-    // ch*32+31; the dP columns they overwrite were read in earlier chunks or
-    // in this one
     tmem_st16(t_dp + ch * 16, pk);
+  }
+}
+
+// P for this warp's 64 columns of a row: 2^(s c + nl2) in pairs, where nl2 is
+// minus the base-2 LSE of the query (the row's one value, or a per-column
+// vector); nl4(j) gives it for local columns 4j..4j+3. Columns with
+// hidden(i) true get P = 0.
+template <bool MASK, typename Nl2Fn, typename HideFn>
+__device__ __forceinline__ void form_p_half(const uint32_t (&sr)[kHalfCols], uint64_t c2, Nl2Fn nl4,
+                                            HideFn hidden, uint64_t (&pr2)[kHalfCols / 2]) {
+#pragma unroll
+  for (int j = 0; j < kHalfCols / 4; ++j) {
+    const float4 n = nl4(j);
+    const uint64_t x0 = f2_fma(f2_pack(__uint_as_float(sr[4 * j]), __uint_as_float(sr[4 * j + 1])), c2,
+                               f2_pack(n.x, n.y));
+    const uint64_t x1 = f2_fma(f2_pack(__uint_as_float(sr[4 * j + 2]), __uint_as_float(sr[4 * j + 3])), c2,
+                               f2_pack(n.z, n.w));
+    float a, b, e, f;
+    f2_unpack(x0, a, b);
+    f2_unpack(x1, e, f);
+    a = ex2_approx(a);
+    b = ex2_approx(b);
+    e = ex2_approx(e);
+    f = ex2_approx(f);
+    if (MASK) {
+      a = hidden(4 * j) ? 0.f : a;
+      b = hidden(4 * j + 1) ? 0.f : b;
+      e = hidden(4 * j + 2) ? 0.f : e;
+      f = hidden(4 * j + 3) ? 0.f : f;
+    }
+    pr2[2 * j] = f2_pack(a, b);
+    pr2[2 * j + 1] = f2_pack(e, f);
   }
 }
 
@@ -360,13 +405,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ compute warps
-    const int r = warp * 32 + lane;   // key row in the tile
+    // warp w: TMEM lanes (key rows) 32 (w % 4) .., columns (queries) 64 (w / 4) ..
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;   // key row in the tile
     const int key = jt * kTile + r;
-    const bool row_valid = key < p.N;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base + L::kColS;
-    const uint32_t tDP = tmem + lane_base + L::kColDP;
-    const float c = p.scale_log2;
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_base + L::kColS + half * kHalfCols;
+    const uint32_t tDP = tmem + lane_base + L::kColDP + half * kHalfCols;
+    const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+    const uint64_t scale2 = f2_pack(p.scale, p.scale);
     bool ok = true;
     for (int it = 0; it < n_blk; ++it) {
       ok = wait_bounded(BAR(B_S_FULL), it & 1, wc, 20);
@@ -375,39 +422,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int q0 = (i0 + it) * kTile;
-      const float* l2 = reinterpret_cast<const float*>(smem + L::kOffStage +
-                                                       (it % kStages) * L::kStageBytes + 2 * L::kTileBytes);
-      const float* dd = l2 + kTile;
-      // queries q0 + i with i < qmask are hidden from this key (causal)
-      const int qmask = CAUSAL ? min(max(key - q0, 0), kTile) : 0;
-      // phase 1: P^T row = 2^(s c - L2_q), written back over S^T as bf16
-      float pr[128];
+      // -L2 and -scale D of this warp's 64 queries (the tail of the stage)
+      const float4* nl2 = reinterpret_cast<const float4*>(smem + L::kOffStage + (it % kStages) * L::kStageBytes +
+                                                          2 * L::kTileBytes) + half * (kHalfCols / 4);
+      const float4* nsd = nl2 + kTile / 4;
+      // phase 1: P^T row = 2^(s c - L2_q), written back over S^T as bf16. Only
+      // the first block under the causal mask hides queries (q < key). Rows
+      // past N are not masked: each row of dV and dK depends on its own row of
+      // P^T and dS^T only, and those rows are never stored.
+      uint64_t pr2[kHalfCols / 2];
       {
-        uint32_t sr[128];
-        tmem_ld128_wait(tS, sr);
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float x = ex2_approx(fmaf(__uint_as_float(sr[i]), c, -l2[i]));
-          pr[i] = (row_valid && i >= qmask) ? x : 0.f;
+        uint32_t sr[kHalfCols];
+        tmem_ld64_wait(tS, sr);
+        auto nl4 = [&](int jj) { return nl2[jj]; };
+        if (CAUSAL && it == 0) {
+          const int qlim = key - q0 - half * kHalfCols;  // local columns below qlim are hidden
+          form_p_half<true>(sr, c2, nl4, [&](int i) { return i < qlim; }, pr2);
+        } else {
+          form_p_half<false>(sr, c2, nl4, [](int) { return false; }, pr2);
         }
       }
+      {
+        uint32_t pk[kHalfCols / 2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[64 * h + 2 * i], pr[64 * h + 2 * i + 1]);
-        tmem_st32(tS + 32 * h, pk);
+        for (int i = 0; i < kHalfCols / 2; ++i) pk[i] = f2_to_bf16x2(pr2[i]);
+        tmem_st32(tS, pk);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_PHASE1));
-      // phase 2: dS^T row = scale P^T (dP^T - D_q), written back over dP^T
+      // phase 2: dS^T row = P^T (scale dP^T - scale D_q), written back over dP^T
       ok = wait_bounded(BAR(B_DP_FULL), it & 1, wc, 22);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      write_ds_row(tDP, pr, p.scale, [&](int i) { return dd[i]; });
+      write_ds_half(tDP, pr2, scale2, [&](int jj) { return nsd[jj]; });
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -420,8 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const size_t gro = (size_t(bh) * p.N + key) * D;
-      store_acc_row<D>(tmem + lane_base + L::kColAcc0, p.dv + gro, row_valid);
-      store_acc_row<D>(tmem + lane_base + L::kColAcc1, p.dk + gro, row_valid);
+      const bool row_valid = key < p.N;
+      store_acc_cols<D / 2>(tmem + lane_base + L::kColAcc0, p.dv + gro, half * (D / 2), row_valid);
+      store_acc_cols<D / 2>(tmem + lane_base + L::kColAcc1, p.dk + gro, half * (D / 2), row_valid);
     }
   }
 
@@ -523,14 +574,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
     }
   } else {
-    const int r = warp * 32 + lane;   // query row in the tile
+    // warp w: TMEM lanes (query rows) 32 (w % 4) .., columns (keys) 64 (w / 4) ..
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;   // query row in the tile
     const int q = it_q * kTile + r;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base + L::kColS;
-    const uint32_t tDP = tmem + lane_base + L::kColDP;
-    const float c = p.scale_log2;
-    const float l2q = p.lse2[size_t(bh) * p.Np + q];  // +inf past N (q < Np always)
-    const float dq_ = p.dvec[size_t(bh) * p.Np + q];
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_base + L::kColS + half * kHalfCols;
+    const uint32_t tDP = tmem + lane_base + L::kColDP + half * kHalfCols;
+    const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+    const uint64_t scale2 = f2_pack(p.scale, p.scale);
+    const float nl2q = p.lse2[size_t(bh) * p.Np + q];  // -inf past N (q < Np always)
+    const float nsdq = p.dvec[size_t(bh) * p.Np + q];
+    const float4 nl2q4 = make_float4(nl2q, nl2q, nl2q, nl2q);
+    const float4 nsdq4 = make_float4(nsdq, nsdq, nsdq, nsdq);
     bool ok = true;
     for (int it = 0; it < n_blk; ++it) {
       ok = wait_bounded(BAR(B_S_FULL), it & 1, wc, 20);
@@ -538,28 +594,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int k0 = it * kTile;
-      // keys k0 + i with i >= klim are hidden (causal: key > q; or key >= N)
-      int klim = p.N - k0;
-      if (CAUSAL) klim = min(klim, q - k0 + 1);
-      klim = max(min(klim, kTile), 0);
       // phase 1: read S (then the MMA may overwrite it) and form P
-      uint32_t sr[128];
-      tmem_ld128_wait(tS, sr);
+      uint32_t sr[kHalfCols];
+      tmem_ld64_wait(tS, sr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_PHASE1));
-      float pr[128];
-#pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        const float x = ex2_approx(fmaf(__uint_as_float(sr[i]), c, -l2q));
-        pr[i] = (i < klim) ? x : 0.f;
+      uint64_t pr2[kHalfCols / 2];
+      auto nl4 = [&](int) { return nl2q4; };
+      // keys past N, or (causal) past q, are hidden: only the last block has any
+      if ((CAUSAL && it == n_blk - 1) || k0 + kTile > p.N) {
+        int klim = p.N - k0;
+        if (CAUSAL) klim = min(klim, q - k0 + 1);
+        klim -= half * kHalfCols;  // local columns at or above klim are hidden
+        form_p_half<true>(sr, c2, nl4, [&](int i) { return i >= klim; }, pr2);
+      } else {
+        form_p_half<false>(sr, c2, nl4, [](int) { return false; }, pr2);
       }
-      // phase 2: dS = scale P (dP - D_q), written back over dP as bf16
+      // phase 2: dS = P (scale dP - scale D_q), written back over dP as bf16
       ok = wait_bounded(BAR(B_DP_FULL), it & 1, wc, 21);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      write_ds_row(tDP, pr, p.scale, [&](int) { return dq_; });
+      write_ds_half(tDP, pr2, scale2, [&](int) { return nsdq4; });
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -571,7 +628,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      store_acc_row<D>(tmem + lane_base + L::kColAcc0, p.dq + (size_t(bh) * p.N + q) * D, q < p.N);
+      store_acc_cols<D / 2>(tmem + lane_base + L::kColAcc0, p.dq + (size_t(bh) * p.N + q) * D, half * (D / 2),
+                            q < p.N);
     }
   }
 

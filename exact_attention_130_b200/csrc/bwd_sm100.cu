@@ -40,8 +40,9 @@
 //                  registers, so phase 1 of block j+1 starts right after
 //                  phase 2 of block j, during dQ_j and dP_j+1.
 //
-// Warp roles (320 threads): warps 0-7 compute, warp 8 TMA producer, warp 9 MMA
-// issuer. A row (one TMEM lane) is shared by two compute warps of the same lane
+// Warp roles (384 threads, three warpgroups): warps 0-7 compute, warp 8 TMA
+// producer, warp 9 MMA issuer, warps 10-11 idle (they only complete the third
+// warpgroup, which setmaxnreg needs whole). A row (one TMEM lane) is shared by two compute warps of the same lane
 // quadrant, warp w taking columns 0-63 and warp w+4 columns 64-127, so each
 // thread keeps 64 probabilities in registers between the phases and two warps
 // per SMSP hide each other's latencies. Each half writes its bf16 P or dS
@@ -54,7 +55,15 @@ namespace fa {
 namespace {
 
 constexpr int kTile = 128;   // rows of the resident tile and of a streamed block
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Registers per thread: the kernels launch with 168 (65536 / 384, rounded down
+// to a multiple of 8); the compute warpgroups then take 208 and the control
+// warpgroup keeps 88: 2*128*208 + 128*88 = 384*168.
+constexpr int kRegsAtLaunch = 168;
+constexpr int kRegsCompute = 208;
+constexpr int kRegsControl = 88;
+static_assert(2 * 128 * kRegsCompute + 128 * kRegsControl <= kThreads * kRegsAtLaunch,
+              "register split exceeds the launch allocation");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kComputeWarps = 8;
@@ -69,11 +78,13 @@ enum : int {
   B_ST_EMPTY = 3,      // +stage: its MMAs are done
   B_S_FULL = 5,        // S of the current block is in TMEM
   B_DP_FULL = 6,       // dP of the current block is in TMEM
-  B_PHASE1 = 7,        // dK/dV: P^T written back; dQ: S read into registers
-  B_PHASE2 = 8,        // dS written back to TMEM
+  B_PHASE1 = 7,        // S of the current block read into registers
+  B_PHASE2 = 8,        // dS (and in the dK/dV kernel P) written back to TMEM
   B_ACC_DONE = 9,
   B_DRAIN = 10,
-  B_COUNT = 11
+  B_DO_FULL = 11,      // +stage, dK/dV kernel: the dO block landed (B_ST_FULL: the Q block)
+  B_DO_EMPTY = 13,     // +stage, dK/dV kernel: dV has read the dO block (B_ST_EMPTY: dK the Q block)
+  B_COUNT = 15
 };
 
 struct BwdParams {
@@ -82,6 +93,8 @@ struct BwdParams {
   const float* lse;
   float* lse2;     // [BH, Np] minus the base-2 LSE, -inf in padding rows
   float* dvec;     // [BH, Np] -scale D, 0 in padding rows
+  uint16_t* qext;  // [BH, Np, 16] bf16: -L/scale split in three (hi, mid, lo), then zeros
+  uint16_t* dext;  // [BH, Np, 16] bf16: -D split in three, then zeros
   uint16_t* dq;
   uint16_t* dk;
   uint16_t* dv;
@@ -93,18 +106,34 @@ struct BwdParams {
 
 __device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
+// v as hi + mid + lo, each rounded to bf16 (round to nearest even): the sum
+// recovers v to about 2^-24 relative, the precision of fp32. Packed as the
+// first three bf16 of 8 (the rest zero).
+__device__ __forceinline__ uint4 split3_bf16(float v) {
+  const uint32_t hi = pack_bf16x2(v, 0.f) & 0xffffu;
+  const float r1 = v - bf16f(hi);
+  const uint32_t mid = pack_bf16x2(r1, 0.f) & 0xffffu;
+  const float r2 = r1 - bf16f(mid);
+  const uint32_t lo = pack_bf16x2(r2, 0.f) & 0xffffu;
+  return make_uint4(hi | (mid << 16), lo, 0u, 0u);
+}
+
 // Shared-memory plan. Row-major bf16 tiles of 128 rows, stored as D/64 column
 // groups of 128 rows x 128 bytes, 128-byte swizzled (TMA box 64 x 128).
+// Extension tiles are 128 rows x 16 bf16 (32 bytes), 32-byte swizzled.
 template <int D>
 struct Plan {
   static constexpr int kGroups = D / 64;
   static constexpr int kSubBytes = kTile * 128;        // 16 KB per column group
   static constexpr int kTileBytes = kGroups * kSubBytes;
+  static constexpr int kExtBytes = kTile * 32;         // 4 KB
   static constexpr int kOffRes0 = 0;
   static constexpr int kOffRes1 = kTileBytes;
-  static constexpr int kOffStage = 2 * kTileBytes;
-  // a stage: two streamed tiles, then (dK/dV kernel) 128 floats of L2 and of D
-  static constexpr int kStageBytes = ((2 * kTileBytes + 1024) + 1023) / 1024 * 1024;
+  static constexpr int kOffOnes = 2 * kTileBytes;      // dK/dV kernel: 128 x 16 ones
+  static constexpr int kOffStage = kOffOnes + kExtBytes;
+  // a stage: two streamed tiles, then (dK/dV kernel) the extension tiles of
+  // the Q block and of the dO block
+  static constexpr int kStageBytes = 2 * kTileBytes + 2 * kExtBytes;
   static constexpr int kOffBar = kOffStage + kStages * kStageBytes;
   static constexpr int kOffMisc = kOffBar + 8 * B_COUNT;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;
@@ -154,8 +183,21 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     const long long r = row0 + st * kRowsPerStep + sub;
     if (j == 0 && r < total) {
       const int bh = int(r / p.Np), row = int(r % p.Np);
-      p.dvec[r] = row < p.N ? -p.scale * dsum : 0.f;
-      p.lse2[r] = row < p.N ? -p.lse[size_t(bh) * p.N + row] * kLog2e : -INFINITY;
+      const bool valid = row < p.N;
+      const float lse = valid ? p.lse[size_t(bh) * p.N + row] : 0.f;
+      p.dvec[r] = valid ? -p.scale * dsum : 0.f;
+      p.lse2[r] = valid ? -lse * kLog2e : -INFINITY;
+      // extension rows: -L/scale (added to S by the MMA, so that scale log2e
+      // times the sum is the exponent of P) and -D (added to dP); a padding
+      // query gets a hugely negative S, so its P is exactly 0
+      const uint4 qx = valid ? split3_bf16(-lse / p.scale) : make_uint4(0xF149u, 0, 0, 0);  // bf16, about -1e30
+      const uint4 dx = valid ? split3_bf16(-dsum) : make_uint4(0, 0, 0, 0);
+      uint4* qo = reinterpret_cast<uint4*>(p.qext + size_t(r) * 16);
+      uint4* dout = reinterpret_cast<uint4*>(p.dext + size_t(r) * 16);
+      qo[0] = qx;
+      qo[1] = make_uint4(0, 0, 0, 0);
+      dout[0] = dx;
+      dout[1] = make_uint4(0, 0, 0, 0);
     }
   }
 }
@@ -173,6 +215,8 @@ __device__ __forceinline__ uint32_t setup_cta(uint8_t* smem, int warp, volatile 
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(B_ST_FULL + s), 1);
       mbar_init(bar(B_ST_EMPTY + s), 1);
+      mbar_init(bar(B_DO_FULL + s), 1);
+      mbar_init(bar(B_DO_EMPTY + s), 1);
     }
     mbar_init(bar(B_S_FULL), 1);
     mbar_init(bar(B_DP_FULL), 1);
@@ -204,6 +248,13 @@ __device__ __forceinline__ void mma_rows_x_rows(uint32_t d_tmem, uint32_t r, uin
     mma_ss(d_tmem, sdesc_sw128(r + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), idesc,
            kk > 0 ? 1u : 0u);
   }
+}
+
+// D[128 x 128] += ONES[128 x 16] * X[128 x 16]^T: adds sum_j X[n][j] to every
+// row of column n (one more K step, both operands 32-byte-swizzled K-major)
+__device__ __forceinline__ void mma_ext(uint32_t d_tmem, uint32_t ones, uint32_t x) {
+  constexpr uint32_t idesc = idesc_bf16(kTile, kTile, false, false);
+  mma_ss(d_tmem, sdesc_sw32_kmajor(ones), sdesc_sw32_kmajor(x), idesc, 1u);
 }
 
 // D[128 x D] (+)= A[128 x 128] * B[128 x D]: A bf16 in TMEM, K-major, its two
@@ -310,6 +361,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmQX, const __grid_constant__ CUtensorMap tmDX,
                     const BwdParams p) {
   using L = Plan<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -323,87 +375,122 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = blockIdx.x % p.BH;
   const int i0 = CAUSAL ? jt : 0;       // first query tile that sees these keys
   const int n_blk = p.n_tiles - i0;
+  // the all-ones tile that multiplies the extension columns (uniform, so its
+  // swizzle does not matter); visible to the tensor core after the fence and
+  // the barrier in setup_cta
+  for (int i = threadIdx.x; i < L::kExtBytes / 16; i += kThreads)
+    reinterpret_cast<uint4*>(smem + L::kOffOnes)[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  fence_proxy_async_smem();
   volatile int* abort_flag;
   const uint32_t tmem = setup_cta<D>(smem, warp, abort_flag);
   const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_BWD};
   const uint32_t sK = sbase + L::kOffRes0, sV = sbase + L::kOffRes1;
-  auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
+  // stage slot s: the Q block (+ its -L2 and -scale D) and the dO block, each
+  // with its own full / empty barriers (Q is released after dK, dO after dV)
+  auto q_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
+  auto do_addr = [&](int it) { return q_addr(it) + L::kTileBytes; };
+  auto qx_addr = [&](int it) { return q_addr(it) + 2 * L::kTileBytes; };
+  auto dx_addr = [&](int it) { return qx_addr(it) + L::kExtBytes; };
+  const uint32_t sOnes = sbase + L::kOffOnes;
+  const uint32_t tP = tmem + L::kColDP;        // P^T as bf16: columns 0-31 and 64-95 of the dP region
+  const uint32_t tDS = tmem + L::kColDP + 32;  // dS^T as bf16: columns 32-63 and 96-127
 
-  if (warp == kLoadWarp) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int issued = 0;
-      mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
-      for (int c = 0; c < L::kGroups; ++c) {
-        tma_load_3d(sK + c * L::kSubBytes, &tmK, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
-        tma_load_3d(sV + c * L::kSubBytes, &tmV, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
-      }
-      for (int it = 0; it < n_blk; ++it) {
-        const int s = it % kStages;
-        if (!wait_bounded(BAR(B_ST_EMPTY + s), ((it / kStages) & 1) ^ 1, wc, 1)) break;
-        const int q0 = (i0 + it) * kTile;
-        const uint32_t st = stage_addr(it);
-        mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kTileBytes + 1024);
+  if (warp >= 8) {
+    regs_decrease<kRegsControl>();
+    if (warp == kLoadWarp) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        int q_issued = 0, do_issued = 0;
+        mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
         for (int c = 0; c < L::kGroups; ++c) {
-          tma_load_3d(st + c * L::kSubBytes, &tmQ, BAR(B_ST_FULL + s), c * 64, q0, bh);
-          tma_load_3d(st + L::kTileBytes + c * L::kSubBytes, &tmDO, BAR(B_ST_FULL + s), c * 64, q0, bh);
+          tma_load_3d(sK + c * L::kSubBytes, &tmK, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
+          tma_load_3d(sV + c * L::kSubBytes, &tmV, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
         }
-        const size_t vo = size_t(bh) * p.Np + q0;
-        bulk_load(st + 2 * L::kTileBytes, p.lse2 + vo, 512, BAR(B_ST_FULL + s));
-        bulk_load(st + 2 * L::kTileBytes + 512, p.dvec + vo, 512, BAR(B_ST_FULL + s));
-        ++issued;
-      }
-      if (*abort_flag) {
-        wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
-        for (int s = 0; s < kStages; ++s) {
-          const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
-          if (cnt > 0) wait_bounded(BAR(B_ST_FULL + s), (cnt - 1) & 1, wc, 2, true);
+        for (int it = 0; it < n_blk; ++it) {
+          const int s = it % kStages, ph = ((it / kStages) & 1) ^ 1;
+          const int q0 = (i0 + it) * kTile;
+          if (!wait_bounded(BAR(B_ST_EMPTY + s), ph, wc, 1)) break;
+          const uint32_t sq = q_addr(it);
+          mbar_arrive_expect_tx(BAR(B_ST_FULL + s), L::kTileBytes + L::kExtBytes);
+          for (int c = 0; c < L::kGroups; ++c)
+            tma_load_3d(sq + c * L::kSubBytes, &tmQ, BAR(B_ST_FULL + s), c * 64, q0, bh);
+          tma_load_3d(qx_addr(it), &tmQX, BAR(B_ST_FULL + s), 0, q0, bh);
+          ++q_issued;
+          if (!wait_bounded(BAR(B_DO_EMPTY + s), ph, wc, 3)) break;
+          mbar_arrive_expect_tx(BAR(B_DO_FULL + s), L::kTileBytes + L::kExtBytes);
+          for (int c = 0; c < L::kGroups; ++c)
+            tma_load_3d(do_addr(it) + c * L::kSubBytes, &tmDO, BAR(B_DO_FULL + s), c * 64, q0, bh);
+          tma_load_3d(dx_addr(it), &tmDX, BAR(B_DO_FULL + s), 0, q0, bh);
+          ++do_issued;
+        }
+        if (*abort_flag) {
+          wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
+          for (int s = 0; s < kStages; ++s) {
+            const int cq = (q_issued - s + kStages - 1) / kStages;  // loads into slot s
+            if (cq > 0) wait_bounded(BAR(B_ST_FULL + s), (cq - 1) & 1, wc, 2, true);
+            const int cd = (do_issued - s + kStages - 1) / kStages;
+            if (cd > 0) wait_bounded(BAR(B_DO_FULL + s), (cd - 1) & 1, wc, 2, true);
+          }
         }
       }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    // order per block i: dV_i (after phase 1), S^T_i+1, dK_i (after phase 2),
-    // dP^T_i+1; the in-order tensor pipe makes each overwrite of the S or dP
-    // columns wait for the MMA that reads the old contents
-    if (lane == 0) {
-      bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
-      if (ok) ok = wait_bounded(BAR(B_ST_FULL + 0), 0, wc, 11);
-      if (ok) {
-        tc_fence_after();
-        mma_rows_x_rows<D>(tmem + L::kColS, sK, stage_addr(0));                    // S^T_0
-        tc_commit(BAR(B_S_FULL));
-        mma_rows_x_rows<D>(tmem + L::kColDP, sV, stage_addr(0) + L::kTileBytes);   // dP^T_0
-        tc_commit(BAR(B_DP_FULL));
-      }
-      for (int it = 0; ok && it < n_blk; ++it) {
-        const uint32_t st = stage_addr(it);
-        ok = wait_bounded(BAR(B_PHASE1), it & 1, wc, 12);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColS, st + L::kTileBytes, it > 0);  // dV += P^T dO
-        if (it + 1 < n_blk) {
-          ok = wait_bounded(BAR(B_ST_FULL + (it + 1) % kStages), ((it + 1) / kStages) & 1, wc, 13);
-          if (!ok) break;
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------ MMA issuer
+      // per block i: S^T_i+1 as soon as S^T_i is in registers; then, once P^T
+      // and dS^T are in TMEM, dK_i, dV_i and dP^T_i+1 (the in-order tensor
+      // pipe makes dP^T_i+1 overwrite the dP region only after dK_i and dV_i
+      // have read it)
+      if (lane == 0) {
+        bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
+        if (ok) ok = wait_bounded(BAR(B_ST_FULL + 0), 0, wc, 11);
+        if (ok) {
           tc_fence_after();
-          mma_rows_x_rows<D>(tmem + L::kColS, sK, stage_addr(it + 1));             // S^T_i+1
+          mma_rows_x_rows<D>(tmem + L::kColS, sK, q_addr(0));            // S^T_0 - L/scale
+          mma_ext(tmem + L::kColS, sOnes, qx_addr(0));
           tc_commit(BAR(B_S_FULL));
         }
-        ok = wait_bounded(BAR(B_PHASE2), it & 1, wc, 14);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tmem_x_rows<D>(tmem + L::kColAcc1, tmem + L::kColDP, st, it > 0);  // dK += dS^T Q
-        tc_commit(BAR(B_ST_EMPTY + it % kStages));
-        if (it + 1 < n_blk) {
-          mma_rows_x_rows<D>(tmem + L::kColDP, sV, stage_addr(it + 1) + L::kTileBytes);  // dP^T_i+1
+        if (ok) ok = wait_bounded(BAR(B_DO_FULL + 0), 0, wc, 16);
+        if (ok) {
+          tc_fence_after();
+          mma_rows_x_rows<D>(tmem + L::kColDP, sV, do_addr(0));          // dP^T_0 - D
+          mma_ext(tmem + L::kColDP, sOnes, dx_addr(0));
           tc_commit(BAR(B_DP_FULL));
         }
+        for (int it = 0; ok && it < n_blk; ++it) {
+          const int s = it % kStages;
+          if (it + 1 < n_blk) {
+            const int s1 = (it + 1) % kStages, ph1 = ((it + 1) / kStages) & 1;
+            ok = wait_bounded(BAR(B_PHASE1), it & 1, wc, 12);
+            if (ok) ok = wait_bounded(BAR(B_ST_FULL + s1), ph1, wc, 13);
+            if (!ok) break;
+            tc_fence_after();
+            mma_rows_x_rows<D>(tmem + L::kColS, sK, q_addr(it + 1));     // S^T_i+1 - L/scale
+            mma_ext(tmem + L::kColS, sOnes, qx_addr(it + 1));
+            tc_commit(BAR(B_S_FULL));
+          }
+          ok = wait_bounded(BAR(B_PHASE2), it & 1, wc, 14);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tmem_x_rows<D>(tmem + L::kColAcc1, tDS, q_addr(it), it > 0);   // dK += dS^T Q
+          tc_commit(BAR(B_ST_EMPTY + s));
+          mma_tmem_x_rows<D>(tmem + L::kColAcc0, tP, do_addr(it), it > 0);   // dV += P^T dO
+          tc_commit(BAR(B_DO_EMPTY + s));
+          if (it + 1 < n_blk) {
+            const int s1 = (it + 1) % kStages, ph1 = ((it + 1) / kStages) & 1;
+            ok = wait_bounded(BAR(B_DO_FULL + s1), ph1, wc, 17);
+            if (!ok) break;
+            tc_fence_after();
+            mma_rows_x_rows<D>(tmem + L::kColDP, sV, do_addr(it + 1));   // dP^T_i+1 - D
+            mma_ext(tmem + L::kColDP, sOnes, dx_addr(it + 1));
+            tc_commit(BAR(B_DP_FULL));
+          }
+        }
+        tc_commit(BAR(B_ACC_DONE));
+        tc_commit(BAR(B_DRAIN));
+        wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
       }
-      tc_commit(BAR(B_ACC_DONE));
-      tc_commit(BAR(B_DRAIN));
-      wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
     }
   } else {
+    regs_increase<kRegsCompute>();
     // ------------------------------------------------------------ compute warps
     // warp w: TMEM lanes (key rows) 32 (w % 4) .., columns (queries) 64 (w / 4) ..
     const int quad = warp & 3, half = warp >> 2;
@@ -415,26 +502,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     const uint64_t scale2 = f2_pack(p.scale, p.scale);
     bool ok = true;
+    // the per-query terms -L/scale and -D arrive inside S^T and dP^T (the
+    // extension K step of their MMAs), so these warps read no shared memory:
+    // while the tensor core streams its operands, shared-memory reads queue for
+    // hundreds of cycles and would stall the exponentials and the barrier
+    // arrivals behind them
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int it = 0; it < n_blk; ++it) {
       ok = wait_bounded(BAR(B_S_FULL), it & 1, wc, 20);
-      if (ok) ok = wait_bounded(BAR(B_ST_FULL + it % kStages), (it / kStages) & 1, wc, 21);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const int q0 = (i0 + it) * kTile;
-      // -L2 and -scale D of this warp's 64 queries (the tail of the stage)
-      const float4* nl2 = reinterpret_cast<const float4*>(smem + L::kOffStage + (it % kStages) * L::kStageBytes +
-                                                          2 * L::kTileBytes) + half * (kHalfCols / 4);
-      const float4* nsd = nl2 + kTile / 4;
-      // phase 1: P^T row = 2^(s c - L2_q), written back over S^T as bf16. Only
-      // the first block under the causal mask hides queries (q < key). Rows
-      // past N are not masked: each row of dV and dK depends on its own row of
-      // P^T and dS^T only, and those rows are never stored.
+      // phase 1: read S^T - L/scale (after which the next S^T may overwrite
+      // it) and form P^T = 2^(scale log2e (s - L_q/scale)) in registers. Only the first block under the
+      // causal mask hides queries (q < key). Rows past N are not masked: each
+      // row of dV and dK depends on its own row of P^T and dS^T only, and those
+      // rows are never stored.
       uint64_t pr2[kHalfCols / 2];
       {
         uint32_t sr[kHalfCols];
         tmem_ld64_wait(tS, sr);
-        auto nl4 = [&](int jj) { return nl2[jj]; };
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_PHASE1));
+        auto nl4 = [&](int) { return zero4; };
         if (CAUSAL && it == 0) {
           const int qlim = key - q0 - half * kHalfCols;  // local columns below qlim are hidden
           form_p_half<true>(sr, c2, nl4, [&](int i) { return i < qlim; }, pr2);
@@ -442,22 +534,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           form_p_half<false>(sr, c2, nl4, [](int) { return false; }, pr2);
         }
       }
-      {
-        uint32_t pk[kHalfCols / 2];
-#pragma unroll
-        for (int i = 0; i < kHalfCols / 2; ++i) pk[i] = f2_to_bf16x2(pr2[i]);
-        tmem_st32(tS, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_PHASE1));
-      // phase 2: dS^T row = P^T (scale dP^T - scale D_q), written back over dP^T
+      // phase 2: dS^T = P^T scale (dP^T - D_q); P^T and dS^T (bf16) then
+      // replace this warp's 64 dP^T columns: P^T in the first 32, dS^T in the
+      // last 32. Both chunks of dP^T are read before either store.
       ok = wait_bounded(BAR(B_DP_FULL), it & 1, wc, 22);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      write_ds_half(tDP, pr2, scale2, [&](int jj) { return nsd[jj]; });
+      {
+        uint32_t pk_ds[kHalfCols / 2];
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t dr[32];
+          tmem_ld32_wait(tDP + ch * 32, dr);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint64_t t0 = f2_mul(f2_pack(__uint_as_float(dr[4 * j]), __uint_as_float(dr[4 * j + 1])), scale2);
+            const uint64_t t1 = f2_mul(f2_pack(__uint_as_float(dr[4 * j + 2]), __uint_as_float(dr[4 * j + 3])), scale2);
+            pk_ds[ch * 16 + 2 * j] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j], t0));
+            pk_ds[ch * 16 + 2 * j + 1] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j + 1], t1));
+          }
+        }
+        uint32_t pk_p[kHalfCols / 2];
+#pragma unroll
+        for (int i = 0; i < kHalfCols / 2; ++i) pk_p[i] = f2_to_bf16x2(pr2[i]);
+        tmem_st32(tDP, pk_p);
+        tmem_st32(tDP + 32, pk_ds);
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -491,6 +594,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
                   const BwdParams p) {
   using L = Plan<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -510,70 +614,74 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = sbase + L::kOffRes0, sDO = sbase + L::kOffRes1;
   auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
 
-  if (warp == kLoadWarp) {
-    if (lane == 0) {
-      int issued = 0;
-      mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
-      for (int c = 0; c < L::kGroups; ++c) {
-        tma_load_3d(sQ + c * L::kSubBytes, &tmQ, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
-        tma_load_3d(sDO + c * L::kSubBytes, &tmDO, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
-      }
-      for (int it = 0; it < n_blk; ++it) {
-        const int s = it % kStages;
-        if (!wait_bounded(BAR(B_ST_EMPTY + s), ((it / kStages) & 1) ^ 1, wc, 1)) break;
-        const uint32_t st = stage_addr(it);
-        mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kTileBytes);
+  if (warp >= 8) {
+    regs_decrease<kRegsControl>();
+    if (warp == kLoadWarp) {
+      if (lane == 0) {
+        int issued = 0;
+        mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
         for (int c = 0; c < L::kGroups; ++c) {
-          tma_load_3d(st + c * L::kSubBytes, &tmK, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
-          tma_load_3d(st + L::kTileBytes + c * L::kSubBytes, &tmV, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
+          tma_load_3d(sQ + c * L::kSubBytes, &tmQ, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
+          tma_load_3d(sDO + c * L::kSubBytes, &tmDO, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
         }
-        ++issued;
-      }
-      if (*abort_flag) {
-        wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
-        for (int s = 0; s < kStages; ++s) {
-          const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
-          if (cnt > 0) wait_bounded(BAR(B_ST_FULL + s), (cnt - 1) & 1, wc, 2, true);
+        for (int it = 0; it < n_blk; ++it) {
+          const int s = it % kStages;
+          if (!wait_bounded(BAR(B_ST_EMPTY + s), ((it / kStages) & 1) ^ 1, wc, 1)) break;
+          const uint32_t st = stage_addr(it);
+          mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kTileBytes);
+          for (int c = 0; c < L::kGroups; ++c) {
+            tma_load_3d(st + c * L::kSubBytes, &tmK, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
+            tma_load_3d(st + L::kTileBytes + c * L::kSubBytes, &tmV, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
+          }
+          ++issued;
+        }
+        if (*abort_flag) {
+          wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
+          for (int s = 0; s < kStages; ++s) {
+            const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
+            if (cnt > 0) wait_bounded(BAR(B_ST_FULL + s), (cnt - 1) & 1, wc, 2, true);
+          }
         }
       }
-    }
-  } else if (warp == kMmaWarp) {
-    // order per block j: S_j+1 (once S_j is in registers), dQ_j (after
-    // phase 2), dP_j+1
-    if (lane == 0) {
-      bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
-      if (ok) ok = wait_bounded(BAR(B_ST_FULL + 0), 0, wc, 11);
-      if (ok) {
-        tc_fence_after();
-        mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(0));                     // S_0
-        tc_commit(BAR(B_S_FULL));
-        mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(0) + L::kTileBytes);   // dP_0
-        tc_commit(BAR(B_DP_FULL));
-      }
-      for (int it = 0; ok && it < n_blk; ++it) {
-        if (it + 1 < n_blk) {
-          ok = wait_bounded(BAR(B_PHASE1), it & 1, wc, 12);
-          if (ok) ok = wait_bounded(BAR(B_ST_FULL + (it + 1) % kStages), ((it + 1) / kStages) & 1, wc, 13);
-          if (!ok) break;
+    } else if (warp == kMmaWarp) {
+      // order per block j: S_j+1 (once S_j is in registers), dQ_j (after
+      // phase 2), dP_j+1
+      if (lane == 0) {
+        bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
+        if (ok) ok = wait_bounded(BAR(B_ST_FULL + 0), 0, wc, 11);
+        if (ok) {
           tc_fence_after();
-          mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(it + 1));              // S_j+1
+          mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(0));                     // S_0
           tc_commit(BAR(B_S_FULL));
-        }
-        ok = wait_bounded(BAR(B_PHASE2), it & 1, wc, 14);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColDP, stage_addr(it), it > 0);  // dQ += dS K
-        tc_commit(BAR(B_ST_EMPTY + it % kStages));
-        if (it + 1 < n_blk) {
-          mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(it + 1) + L::kTileBytes);  // dP_j+1
+          mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(0) + L::kTileBytes);   // dP_0
           tc_commit(BAR(B_DP_FULL));
         }
+        for (int it = 0; ok && it < n_blk; ++it) {
+          if (it + 1 < n_blk) {
+            ok = wait_bounded(BAR(B_PHASE1), it & 1, wc, 12);
+            if (ok) ok = wait_bounded(BAR(B_ST_FULL + (it + 1) % kStages), ((it + 1) / kStages) & 1, wc, 13);
+            if (!ok) break;
+            tc_fence_after();
+            mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(it + 1));              // S_j+1
+            tc_commit(BAR(B_S_FULL));
+          }
+          ok = wait_bounded(BAR(B_PHASE2), it & 1, wc, 14);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColDP, stage_addr(it), it > 0);  // dQ += dS K
+          tc_commit(BAR(B_ST_EMPTY + it % kStages));
+          if (it + 1 < n_blk) {
+            mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(it + 1) + L::kTileBytes);  // dP_j+1
+            tc_commit(BAR(B_DP_FULL));
+          }
+        }
+        tc_commit(BAR(B_ACC_DONE));
+        tc_commit(BAR(B_DRAIN));
+        wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
       }
-      tc_commit(BAR(B_ACC_DONE));
-      tc_commit(BAR(B_DRAIN));
-      wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
     }
   } else {
+    regs_increase<kRegsCompute>();
     // warp w: TMEM lanes (query rows) 32 (w % 4) .., columns (keys) 64 (w / 4) ..
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;   // query row in the tile
@@ -648,9 +756,18 @@ fa_status launch_main(Kern kern, unsigned kid, int smem, unsigned grid, const CU
                       const BwdParams& p, const LaunchCtx& ctx, const char* what) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, what);
+  // the setmaxnreg split is sized for exactly kRegsAtLaunch registers per
+  // thread; with fewer the increase could wait forever, so refuse to launch
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  if (attr.numRegs != kRegsAtLaunch) {
+    set_last_error("%s built with %d registers per thread, expected %d", what, attr.numRegs, kRegsAtLaunch);
+    return FA_ERR_UNSUPPORTED;
+  }
   {
     ProfileScope prof(kid, ctx.stream);
-    kern<<<grid, kThreads, smem, ctx.stream>>>(m[0], m[1], m[2], m[3], p);
+    kern<<<grid, kThreads, smem, ctx.stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
@@ -662,13 +779,16 @@ fa_status launch_all(const void* q, const void* k, const void* v, const void* dO
                      const LaunchCtx& ctx) {
   const int smem = Plan<D>::kSmemBytes;
   const unsigned grid = unsigned(p.n_tiles) * unsigned(p.BH);
-  CUtensorMap m[4];
+  CUtensorMap m[6];
   const void* src[4] = {q, dO, k, v};
   for (int i = 0; i < 4; ++i) {
-    fa_status st = make_tmap_3d(&m[i], src[i], true, D, p.N, p.BH, 64, kTile, true);
+    fa_status st = make_tmap_3d(&m[i], src[i], true, D, p.N, p.BH, 64, kTile, 128);
     if (st != FA_OK) return st;
   }
-  fa_status st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid, m, p, ctx,
+  fa_status st = make_tmap_3d(&m[4], p.qext, true, 16, p.Np, p.BH, 16, kTile, 32);
+  if (st == FA_OK) st = make_tmap_3d(&m[5], p.dext, true, 16, p.Np, p.BH, 16, kTile, 32);
+  if (st != FA_OK) return st;
+  st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid, m, p, ctx,
                              "bwd dK/dV kernel");
   if (st != FA_OK) return st;
   return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid, m, p, ctx, "bwd dQ kernel");
@@ -680,7 +800,7 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d) {
   (void)d;
   const size_t bh = size_t(B) * H;
   const size_t np = (size_t(N) + kTile - 1) / kTile * kTile;
-  return 2 * align256(bh * np * 4);
+  return 2 * align256(bh * np * 4) + 2 * align256(bh * np * 32);
 }
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -700,8 +820,11 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     return FA_ERR_UNSUPPORTED;
   }
   char* ws = static_cast<char*>(workspace);
+  const size_t vec_bytes = align256(size_t(BH) * p.Np * 4), ext_bytes = align256(size_t(BH) * p.Np * 32);
   p.lse2 = reinterpret_cast<float*>(ws);
-  p.dvec = reinterpret_cast<float*>(ws + align256(size_t(BH) * p.Np * 4));
+  p.dvec = reinterpret_cast<float*>(ws + vec_bytes);
+  p.qext = reinterpret_cast<uint16_t*>(ws + 2 * vec_bytes);
+  p.dext = reinterpret_cast<uint16_t*>(ws + 2 * vec_bytes + ext_bytes);
   p.dq = static_cast<uint16_t*>(dq);
   p.dk = static_cast<uint16_t*>(dk);
   p.dv = static_cast<uint16_t*>(dv);

@@ -174,7 +174,7 @@ fa_status current_launch_ctx(cudaStream_t stream, LaunchCtx* ctx) {
 
 fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t inner,
                        uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows,
-                       bool swizzle128) {
+                       int swizzle_bytes) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -192,7 +192,9 @@ fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_
   CUresult r = g_encode(map, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                         3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                              : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return invalid(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));

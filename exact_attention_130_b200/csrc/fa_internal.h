@@ -54,12 +54,11 @@ void set_last_error(const char* fmt, ...);
 fa_status cuda_fail(cudaError_t e, const char* what);
 
 // 3-D tiled tensor map over a [outer, rows, inner] bf16 or fp32 tensor
-// (inner contiguous), box = box_inner x box_rows x 1, 128-byte swizzle when
-// `swizzle128` (box_inner * elem must then be 128 bytes), zero fill out of
-// bounds.
+// (inner contiguous), box = box_inner x box_rows x 1, zero fill out of bounds.
+// swizzle_bytes: 128 or 32 (box_inner * elem must then equal it) or 0.
 fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t inner,
                        uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows,
-                       bool swizzle128);
+                       int swizzle_bytes);
 
 fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int N, int d, float scale, bool causal,

@@ -521,9 +521,9 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   const uint64_t BH = uint64_t(B) * uint64_t(H);
   CUtensorMap mq, mk, mv;
   fa_status st;
-  if ((st = make_tmap_3d(&mq, q, true, d, N, BH, 64, 128, true)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&mk, k, true, d, N, BH, 64, 128, true)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&mv, v, true, d, N, BH, 64, 128, true)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mq, q, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mk, k, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mv, v, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
   FwdParams p;
   p.o = o;
   p.lse = lse;

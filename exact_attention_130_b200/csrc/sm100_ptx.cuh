@@ -211,6 +211,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= uint64_t(2) << 61;
   return d;
 }
+// The same for a K-major operand in the 32-byte swizzle (rows of 16 bf16 =
+// 32 bytes, 8-row groups 256 bytes apart): one K step of 16 per row. Layout
+// code 6 in bits 61-63.
+__device__ __forceinline__ uint64_t sdesc_sw32_kmajor(uint32_t saddr) {
+  uint64_t d = uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t(1) << 16;                    // leading offset unused (one swizzle atom in K)
+  d |= uint64_t((256u >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(6) << 61;
+  return d;
+}
 
 // ----------------------------------------------------------------------------
 // tensor memory <-> registers, shape 32x32b: thread i of warp w touches lane

@@ -100,9 +100,11 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o,
 
 /*
  * fa_bwd_workspace_size -- bytes of scratch fa_bwd needs: two fp32 vectors
- * [B, H, Np] (the saved LSE in base 2, and D = rowsum(dO * O)), Np = N
- * rounded up to a multiple of 128, each starting on a 256-byte boundary.
- * Returns 0 for invalid sizes.
+ * [B, H, Np] (the saved LSE in base 2, and D = rowsum(dO * O), in the forms
+ * the kernels add) and two bf16 arrays [B, H, Np, 16] (-L/scale and -D, each
+ * split into three bf16 terms, which the tensor cores add to S and dP), Np =
+ * N rounded up to a multiple of 128, each part starting on a 256-byte
+ * boundary. Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 

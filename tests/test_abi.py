@@ -80,8 +80,9 @@ def test_bwd_and_decode_argument_errors(lib):
 def test_workspace_sizes(lib):
     # base-2 LSE and D (fp32 [B,H,Np], Np = N rounded up to 128), each
     # 256-aligned
-    assert fa.fa_bwd_workspace_size(2, 16, 4096, 128) == 2 * (2 * 16 * 4096 * 4)
-    assert fa.fa_bwd_workspace_size(1, 1, 130, 64) == 2 * 1024
+    # two fp32 vectors and two rows of 16 bf16 per (batch, head, padded row)
+    assert fa.fa_bwd_workspace_size(2, 16, 4096, 128) == 2 * (2 * 16 * 4096 * 4) + 2 * (2 * 16 * 4096 * 32)
+    assert fa.fa_bwd_workspace_size(1, 1, 130, 64) == 2 * 1024 + 2 * 256 * 32
     assert fa.fa_bwd_workspace_size(1, 1, 0, 64) == 0
     # decode: C chunks of partial outputs and LSEs
     ws = fa.fa_decode_workspace_size(8, 32, 32768, 128, 16)

@@ -77,7 +77,9 @@ enum : int {
   B_K_FULL = 16,   // +stage
   B_V_FULL = 20,   // +stage
   B_KV_EMPTY = 24, // +stage
-  B_COUNT = 28
+  B_STG_FREE = 28, // the O staging buffer may be rewritten (one arrival per epilogue)
+  B_STG_READY = 29, // +t: the 4 warps of softmax group t have written the staging buffer
+  B_COUNT = 31
 };
 
 template <int D>
@@ -89,7 +91,8 @@ struct Layout {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kOffStg = kOffV + kStages * kTileBytes;  // O tile staging for the TMA store
+  static constexpr int kOffBar = kOffStg + kTileBytes;
   static constexpr int kOffMisc = kOffBar + 8 * B_COUNT;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
@@ -157,7 +160,8 @@ __device__ __forceinline__ int kv_tiles_for(int qtile, int n_kv) {
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const FwdParams p) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -181,6 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(BAR(B_O_EMPTY + t), 4);
     }
     mbar_init(BAR(B_DRAIN), 1);
+    mbar_init(BAR(B_STG_FREE), 1);
+    mbar_init(BAR(B_STG_READY + 0), 4);
+    mbar_init(BAR(B_STG_READY + 1), 4);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(BAR(B_K_FULL + s), 1);
       mbar_init(BAR(B_V_FULL + s), 1);
@@ -300,10 +307,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = wait_bounded(BAR(B_K_FULL + s0), (kv_used / L::kStages) & 1, wc, 11);
             if (!ok) break;
             tc_fence_after();
+            // a Q tile is released after its last QK^T (not its last PV), so
+            // the next unit's Q loads while this unit's last steps run
             issue_qk(0, s0);
             tc_commit(BAR(B_S_FULL + 0));
+            if (n0 == 1) tc_commit(BAR(B_Q_EMPTY + 0));
             issue_qk(1, s0);
             tc_commit(BAR(B_S_FULL + 1));
+            if (n1 == 1) tc_commit(BAR(B_Q_EMPTY + 1));
           }
           int k_ready = 0;
           for (int j = 0; ok && j < n1; ++j) {
@@ -334,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 issue_qk(t, s2);
                 tc_commit(BAR(B_S_FULL + t));
+                if (j + 2 == nt) tc_commit(BAR(B_Q_EMPTY + t));
               } else {
                 tc_commit(BAR(B_O_FULL + t));
-                tc_commit(BAR(B_Q_EMPTY + t));
               }
             }
             if (!ok) break;
@@ -448,39 +459,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      // epilogue: O = O~ / l, LSE = ln2 * (m + log2 l)
+      // epilogue: O = O~ / l as bf16, staged in shared memory (128-byte
+      // swizzle, the layout of the tensor map) and written by TMA stores of
+      // 64-column groups, so the rows need no strided global stores; LSE =
+      // ln2 * (m + log2 l). One staging buffer serves both groups: the
+      // epilogues of a CTA happen in the order their O_FULL commits (tile 0,
+      // tile 1, next unit ...), and epilogue e waits until the store of
+      // epilogue e-1 has read the buffer.
+      const int e = 2 * unit_iter + t;
       ok = wait_bounded(BAR(B_O_FULL + t), unit_iter & 1, wc, 21);
+      if (ok && e > 0) ok = wait_bounded(BAR(B_STG_FREE), (e - 1) & 1, wc, 22);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.0f / l;
-      uint16_t* orow_g = reinterpret_cast<uint16_t*>(p.o) + (size_t(bh) * p.N + size_t(row)) * D;
+      uint8_t* stg = smem + L::kOffStg + r * 128;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t orow[32];
         tmem_ld32_wait(tO + ch * 32, orow);
-        if (row < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow_g + ch * 32);
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(orow[8 * v4 + 0]) * inv_l,
-                              __uint_as_float(orow[8 * v4 + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(orow[8 * v4 + 2]) * inv_l,
-                              __uint_as_float(orow[8 * v4 + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(orow[8 * v4 + 4]) * inv_l,
-                              __uint_as_float(orow[8 * v4 + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(orow[8 * v4 + 6]) * inv_l,
-                              __uint_as_float(orow[8 * v4 + 7]) * inv_l);
-            dst[v4] = w;
-          }
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(orow[8 * v4 + 0]) * inv_l,
+                            __uint_as_float(orow[8 * v4 + 1]) * inv_l);
+          w.y = pack_bf16x2(__uint_as_float(orow[8 * v4 + 2]) * inv_l,
+                            __uint_as_float(orow[8 * v4 + 3]) * inv_l);
+          w.z = pack_bf16x2(__uint_as_float(orow[8 * v4 + 4]) * inv_l,
+                            __uint_as_float(orow[8 * v4 + 5]) * inv_l);
+          w.w = pack_bf16x2(__uint_as_float(orow[8 * v4 + 6]) * inv_l,
+                            __uint_as_float(orow[8 * v4 + 7]) * inv_l);
+          const int k16 = ch * 4 + v4;           // 16-byte chunk of the row (8 columns)
+          const int g = k16 >> 3, cc = k16 & 7;  // 64-column group, chunk in its 128-byte row
+          *reinterpret_cast<uint4*>(stg + g * L::kSubBytes + ((cc ^ (r & 7)) << 4)) = w;
         }
       }
-      if (row < p.N) p.lse[size_t(bh) * p.N + row] = (m + lg2_approx(l)) * kLn2;
       tc_fence_before();
+      fence_proxy_async_smem();  // the staging writes, for the TMA store
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_O_EMPTY + t));
+      if (lane == 0) {
+        mbar_arrive(BAR(B_O_EMPTY + t));
+        mbar_arrive(BAR(B_STG_READY + t));
+      }
+      if (row < p.N) p.lse[size_t(bh) * p.N + row] = (m + lg2_approx(l)) * kLn2;
+      if (r == 0) {
+        // rows past N fall outside the tensor and are not written
+        if (wait_bounded(BAR(B_STG_READY + t), unit_iter & 1, wc, 23)) {
+          for (int g = 0; g < L::kSub; ++g)
+            tma_store_3d(&tmO, sbase + L::kOffStg + g * L::kSubBytes, g * 64, qt * kBM, bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(BAR(B_STG_FREE));
+        }
+      }
     }
+    // the last stores must be complete before the CTA exits
+    if (r == 0) bulk_wait_group0();
     tc_fence_before();
     __syncthreads();
   }
@@ -488,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool CAUSAL>
 fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                 const FwdParams& p, const LaunchCtx& ctx) {
+                 const CUtensorMap& mo, const FwdParams& p, const LaunchCtx& ctx) {
   auto kern = fwd_kernel<D, CAUSAL>;
   const int smem = Layout<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -506,7 +540,7 @@ fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
   const int grid = p.num_items < ctx.num_sms ? p.num_items : ctx.num_sms;
   {
     ProfileScope prof(KID_FWD, ctx.stream);
-    kern<<<grid, kThreads, smem, ctx.stream>>>(mq, mk, mv, p);
+    kern<<<grid, kThreads, smem, ctx.stream>>>(mq, mk, mv, mo, p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
@@ -519,11 +553,12 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
                           int B, int H, int N, int d, float scale, bool causal,
                           const LaunchCtx& ctx) {
   const uint64_t BH = uint64_t(B) * uint64_t(H);
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   fa_status st;
   if ((st = make_tmap_3d(&mq, q, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
   if ((st = make_tmap_3d(&mk, k, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
   if ((st = make_tmap_3d(&mv, v, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mo, o, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
   FwdParams p;
   p.o = o;
   p.lse = lse;
@@ -537,9 +572,9 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load;
-  if (d == 128) return causal ? launch<128, true>(mq, mk, mv, p, ctx)
-                              : launch<128, false>(mq, mk, mv, p, ctx);
-  return causal ? launch<64, true>(mq, mk, mv, p, ctx) : launch<64, false>(mq, mk, mv, p, ctx);
+  if (d == 128) return causal ? launch<128, true>(mq, mk, mv, mo, p, ctx)
+                              : launch<128, false>(mq, mk, mv, mo, p, ctx);
+  return causal ? launch<64, true>(mq, mk, mv, mo, p, ctx) : launch<64, false>(mq, mk, mv, mo, p, ctx);
 }
 
 }  // namespace fa

@@ -106,26 +106,43 @@ struct FwdParams {
   int n_kv;       // K/V tiles per head
   int n_pairs;    // Q-tile pairs per head
   int cpp;        // causal: couples of pairs per head, ceil(n_pairs / 2)
-  int num_items;  // work items handed out round-robin to the CTAs
+  int num_items;  // work items handed out to the CTAs
   float scale_log2;
   unsigned int* status;
   unsigned long long limit_ns;
   int debug_skip;
 };
 
-// Work list. A unit is one (head, Q-tile pair). CTA c takes items c, c + G,
-// c + 2G, ... (G = grid size), so all three roles walk the same sequence.
-//  * no mask: item = unit, head-major, so the ~G units in flight share few
-//    heads and their K/V tiles stay in L2;
-//  * causal: item = a couple of pairs (n_pairs-1-k, k) of one head, the
-//    heavier first; a couple always costs 2 n_pairs + 1 K/V tile steps, so
-//    equal item counts mean equal work, and the couples of one head run
-//    side by side (L2 reuse again). With n_pairs odd the middle pair is a
-//    couple on its own.
-// Advances (item, half) and returns the unit, or false at the end.
-template <bool CAUSAL>
+// Work list. A unit is one (head, Q-tile pair); every role of a CTA walks the
+// same sequence (G = grid size).
+//  * no mask: CTA c takes items c, c + G, c + 2G, ...; item = unit,
+//    head-major, so the ~G units in flight share few heads and their K/V
+//    tiles stay in L2;
+//  * causal, couples: item = a couple of pairs (n_pairs-1-k, k) of one head,
+//    the heavier first, taken as above; a couple always costs 2 n_pairs + 1 or
+//    + 2 K/V tile steps, so equal item counts mean equal work, and the couples
+//    of one head run side by side (L2 reuse again). With n_pairs odd the
+//    middle pair is a couple on its own.
+//  * causal, snake (a separate instantiation, chosen by the host when the couples leave the last round
+//    of CTAs much emptier than the others, as with few heads and short
+//    sequences): item = one pair, sorted by level from the heaviest down
+//    (item i: level n_pairs-1-i/BH, head i%BH); round r gives CTA c item
+//    r G + c for even r and r G + G-1-c for odd r, which evens out the sums.
+// Advances the state and returns the unit, or false at the end.
+template <bool CAUSAL, bool SNAKE>
 __device__ __forceinline__ bool next_unit(const FwdParams& p, int& item, int& half, int& bh,
                                           int& pair) {
+  if (SNAKE) {
+    // `item` counts the rounds here (it starts at 0)
+    const int G = int(gridDim.x), c = int(blockIdx.x);
+    const int idx = item * G + ((item & 1) ? G - 1 - c : c);
+    if (idx >= p.num_items) return false;
+    pair = p.n_pairs - 1 - idx / p.BH;
+    bh = idx % p.BH;
+    ++item;
+    return true;
+  }
+  // `item` is the item index (it starts at blockIdx.x)
   if (item >= p.num_items) return false;
   if (!CAUSAL) {
     bh = item / p.n_pairs;
@@ -157,7 +174,7 @@ __device__ __forceinline__ int kv_tiles_for(int qtile, int n_kv) {
   return n_kv;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SNAKE>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -221,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int v_skip_stage = -1;  // stage whose V load the test hook left out
         bool skip_pending = p.debug_skip && blockIdx.x == 0;
         bool ok = true;
-        int item = blockIdx.x, half = 0, bh, pair;
-        for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
+        int item = SNAKE ? 0 : int(blockIdx.x), half = 0, bh, pair;
+        for (; ok && next_unit<CAUSAL, SNAKE>(p, item, half, bh, pair); ++unit_iter) {
           const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
           for (int t = 0; t < 2 && ok; ++t) {
             ok = wait_bounded(BAR(B_Q_EMPTY + t), (unit_iter & 1) ^ 1, wc, 1);
@@ -295,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int kv_used = 0, unit_iter = 0;
         int p_cnt[2] = {0, 0};
         bool ok = true;
-        int item = blockIdx.x, half = 0, bh, pair;
-        for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
+        int item = SNAKE ? 0 : int(blockIdx.x), half = 0, bh, pair;
+        for (; ok && next_unit<CAUSAL, SNAKE>(p, item, half, bh, pair); ++unit_iter) {
           const int n0 = kv_tiles_for<CAUSAL>(2 * pair, p.n_kv);
           const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
           for (int t = 0; t < 2 && ok; ++t)
@@ -378,8 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     int s_cnt = 0, unit_iter = 0;
     bool ok = true;
-    int item = blockIdx.x, half = 0, bh, pair;
-    for (; ok && next_unit<CAUSAL>(p, item, half, bh, pair); ++unit_iter) {
+    int item = SNAKE ? 0 : int(blockIdx.x), half = 0, bh, pair;
+    for (; ok && next_unit<CAUSAL, SNAKE>(p, item, half, bh, pair); ++unit_iter) {
       const int qt = 2 * pair + t;
       const int nt = kv_tiles_for<CAUSAL>(qt, p.n_kv);
       const int row = qt * kBM + r;
@@ -520,10 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SNAKE = false>
 fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                  const CUtensorMap& mo, const FwdParams& p, const LaunchCtx& ctx) {
-  auto kern = fwd_kernel<D, CAUSAL>;
+  auto kern = fwd_kernel<D, CAUSAL, SNAKE>;
   const int smem = Layout<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fwd)");
@@ -567,14 +584,29 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   p.n_kv = (N + kBN - 1) / kBN;
   p.n_pairs = (p.n_kv + 1) / 2;
   p.cpp = (p.n_pairs + 1) / 2;
+  bool snake = false;
   p.num_items = causal ? p.BH * p.cpp : p.BH * p.n_pairs;
+  if (causal) {
+    // couples carry equal work; if the last round of them leaves many CTAs
+    // idle (fraction of a full round below 95%), deal single pairs instead,
+    // heaviest first in snake order
+    const int G = p.num_items < ctx.num_sms ? p.num_items : ctx.num_sms;
+    const long long rounds = (p.num_items + G - 1) / G;
+    if (double(p.num_items) / double(G) < 0.95 * double(rounds)) {
+      snake = true;
+      p.num_items = p.BH * p.n_pairs;
+    }
+  }
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load;
-  if (d == 128) return causal ? launch<128, true>(mq, mk, mv, mo, p, ctx)
-                              : launch<128, false>(mq, mk, mv, mo, p, ctx);
-  return causal ? launch<64, true>(mq, mk, mv, mo, p, ctx) : launch<64, false>(mq, mk, mv, mo, p, ctx);
+  if (d == 128) {
+    if (!causal) return launch<128, false>(mq, mk, mv, mo, p, ctx);
+    return snake ? launch<128, true, true>(mq, mk, mv, mo, p, ctx) : launch<128, true>(mq, mk, mv, mo, p, ctx);
+  }
+  if (!causal) return launch<64, false>(mq, mk, mv, mo, p, ctx);
+  return snake ? launch<64, true, true>(mq, mk, mv, mo, p, ctx) : launch<64, true>(mq, mk, mv, mo, p, ctx);
 }
 
 }  // namespace fa

@@ -156,13 +156,18 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   const int sub = lane / kLanesPerRow, j = lane % kLanesPerRow;
   const long long total = static_cast<long long>(p.BH) * p.Np;
   const long long row0 = gwarp * kRowsPerStep * kPreSteps;
+  // a warp's rows never cross a (batch, head): Np is a multiple of 128 and a
+  // warp covers kRowsPerStep * kPreSteps rows (8 or 16), a divisor of 128, so
+  // one division per thread
+  static_assert(kTile % (kRowsPerStep * kPreSteps) == 0, "a warp's rows must stay in one head");
+  const int bh0 = int(row0 / p.Np), rowb = int(row0 - static_cast<long long>(bh0) * p.Np);
   uint4 ov[kPreSteps], gv[kPreSteps];
 #pragma unroll
   for (int st = 0; st < kPreSteps; ++st) {
     const long long r = row0 + st * kRowsPerStep + sub;
     ov[st] = gv[st] = make_uint4(0, 0, 0, 0);
     if (r < total) {
-      const int bh = int(r / p.Np), row = int(r % p.Np);
+      const int bh = bh0, row = rowb + st * kRowsPerStep + sub;
       if (row < p.N) {
         const size_t off = (size_t(bh) * p.N + row) * D + j * 8;
         ov[st] = *reinterpret_cast<const uint4*>(p.o + off);
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     for (int off = kLanesPerRow / 2; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
     const long long r = row0 + st * kRowsPerStep + sub;
     if (j == 0 && r < total) {
-      const int bh = int(r / p.Np), row = int(r % p.Np);
+      const int bh = bh0, row = rowb + st * kRowsPerStep + sub;
       const bool valid = row < p.N;
       const float lse = valid ? p.lse[size_t(bh) * p.N + row] : 0.f;
       p.dvec[r] = valid ? -p.scale * dsum : 0.f;

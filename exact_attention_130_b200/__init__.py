@@ -72,7 +72,7 @@ _SIGNATURES = {
 }
 
 KERNEL_NAMES = {1: "fwd", 2: "fwd_f32", 3: "bwd_pre", 4: "bwd_dkdv", 5: "bwd_dq",
-                6: "decode_split", 7: "decode_merge"}
+                6: "decode_split", 7: "decode_merge", 8: "fwd_merge"}
 
 
 def load_library():
@@ -279,9 +279,9 @@ def fa_profile_begin():
 def fa_profile_end():
     """Stop per-kernel timing; return {kernel name: (launches, total ms)}."""
     lib = load_library()
-    launches = (ctypes.c_int * 8)()
-    total = (ctypes.c_double * 8)()
-    rc = lib.fa_profile_end(launches, total, 8)
+    launches = (ctypes.c_int * 16)()
+    total = (ctypes.c_double * 16)()
+    rc = lib.fa_profile_end(launches, total, 16)
     if rc < 0:
         raise FAError(5, "fa_profile_end: a CUDA event call failed")
     return {KERNEL_NAMES[k]: (launches[k], total[k]) for k in KERNEL_NAMES if launches[k]}

@@ -107,6 +107,10 @@ struct FwdParams {
   int n_pairs;    // Q-tile pairs per head
   int cpp;        // causal: couples of pairs per head, ceil(n_pairs / 2)
   int num_items;  // work items handed out to the CTAs
+  int full_items; // split mode: items before this index are whole units
+  int split_s;    // split mode: parts per split unit (along the keys)
+  float* part_o;  // split mode: [slot][2 tiles][128 rows][d] fp32, O of each part normalised by its l
+  float* part_lse;  // split mode: [slot][2 tiles][128 rows] base-2 LSE of each part
   float scale_log2;
   unsigned int* status;
   unsigned long long limit_ns;
@@ -123,16 +127,30 @@ struct FwdParams {
 //    + 2 K/V tile steps, so equal item counts mean equal work, and the couples
 //    of one head run side by side (L2 reuse again). With n_pairs odd the
 //    middle pair is a couple on its own.
+//  * no mask, split (a separate instantiation, chosen by the host when the
+//    units leave the last round of CTAs short): items below full_items are
+//    whole units as above; the remaining units are split along the keys into
+//    split_s parts each (item full_items + k is part k % split_s of unit
+//    full_items + k / split_s), whose partial O and LSE go to slot k and are
+//    merged afterwards;
 //  * causal, snake (a separate instantiation, chosen by the host when the couples leave the last round
 //    of CTAs much emptier than the others, as with few heads and short
 //    sequences): item = one pair, sorted by level from the heaviest down
 //    (item i: level n_pairs-1-i/BH, head i%BH); round r gives CTA c item
 //    r G + c for even r and r G + G-1-c for odd r, which evens out the sums.
 // Advances the state and returns the unit, or false at the end.
-template <bool CAUSAL, bool SNAKE>
+// Work modes (a template parameter of the kernel).
+constexpr int kModePlain = 0, kModeSnake = 1, kModeSplit = 2;
+
+// kv0: first K/V tile of the item; cnt: its K/V tile count, or -1 for "as
+// the mask allows"; slot: partial-result slot, or -1 for a whole unit.
+template <bool CAUSAL, int MODE>
 __device__ __forceinline__ bool next_unit(const FwdParams& p, int& item, int& half, int& bh,
-                                          int& pair) {
-  if (SNAKE) {
+                                          int& pair, int& kv0, int& cnt, int& slot) {
+  kv0 = 0;
+  cnt = -1;
+  slot = -1;
+  if (MODE == kModeSnake) {
     // `item` counts the rounds here (it starts at 0)
     const int G = int(gridDim.x), c = int(blockIdx.x);
     const int idx = item * G + ((item & 1) ? G - 1 - c : c);
@@ -145,8 +163,17 @@ __device__ __forceinline__ bool next_unit(const FwdParams& p, int& item, int& ha
   // `item` is the item index (it starts at blockIdx.x)
   if (item >= p.num_items) return false;
   if (!CAUSAL) {
-    bh = item / p.n_pairs;
-    pair = item % p.n_pairs;
+    int u = item;
+    if (MODE == kModeSplit && item >= p.full_items) {
+      const int k = item - p.full_items;
+      const int part = k % p.split_s;
+      u = p.full_items + k / p.split_s;
+      kv0 = part * p.n_kv / p.split_s;
+      cnt = (part + 1) * p.n_kv / p.split_s - kv0;
+      slot = k;
+    }
+    bh = u / p.n_pairs;
+    pair = u % p.n_pairs;
     item += gridDim.x;
     return true;
   }
@@ -174,7 +201,7 @@ __device__ __forceinline__ int kv_tiles_for(int qtile, int n_kv) {
   return n_kv;
 }
 
-template <int D, bool CAUSAL, bool SNAKE>
+template <int D, bool CAUSAL, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -238,9 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int v_skip_stage = -1;  // stage whose V load the test hook left out
         bool skip_pending = p.debug_skip && blockIdx.x == 0;
         bool ok = true;
-        int item = SNAKE ? 0 : int(blockIdx.x), half = 0, bh, pair;
-        for (; ok && next_unit<CAUSAL, SNAKE>(p, item, half, bh, pair); ++unit_iter) {
-          const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
+        int item = MODE == kModeSnake ? 0 : int(blockIdx.x), half = 0, bh, pair, kv0, cnt, slot;
+        for (; ok && next_unit<CAUSAL, MODE>(p, item, half, bh, pair, kv0, cnt, slot); ++unit_iter) {
+          const int n1 = cnt >= 0 ? cnt : kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
           for (int t = 0; t < 2 && ok; ++t) {
             ok = wait_bounded(BAR(B_Q_EMPTY + t), (unit_iter & 1) ^ 1, wc, 1);
             if (!ok) break;
@@ -258,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(BAR(B_K_FULL + s), L::kTileBytes);
             for (int c = 0; c < L::kSub; ++c)
               tma_load_3d(sbase + L::kOffK + s * L::kTileBytes + c * L::kSubBytes, &tmK,
-                          BAR(B_K_FULL + s), c * 64, j * kBN, bh);
+                          BAR(B_K_FULL + s), c * 64, (kv0 + j) * kBN, bh);
             if (skip_pending) {
               skip_pending = false;  // test hook: this V tile never arrives
               v_skip_stage = s;
@@ -266,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(BAR(B_V_FULL + s), L::kTileBytes);
               for (int c = 0; c < L::kSub; ++c)
                 tma_load_3d(sbase + L::kOffV + s * L::kTileBytes + c * L::kSubBytes, &tmV,
-                            BAR(B_V_FULL + s), c * 64, j * kBN, bh);
+                            BAR(B_V_FULL + s), c * 64, (kv0 + j) * kBN, bh);
             }
           }
         }
@@ -312,10 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int kv_used = 0, unit_iter = 0;
         int p_cnt[2] = {0, 0};
         bool ok = true;
-        int item = SNAKE ? 0 : int(blockIdx.x), half = 0, bh, pair;
-        for (; ok && next_unit<CAUSAL, SNAKE>(p, item, half, bh, pair); ++unit_iter) {
-          const int n0 = kv_tiles_for<CAUSAL>(2 * pair, p.n_kv);
-          const int n1 = kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
+        int item = MODE == kModeSnake ? 0 : int(blockIdx.x), half = 0, bh, pair, kv0, cnt, slot;
+        for (; ok && next_unit<CAUSAL, MODE>(p, item, half, bh, pair, kv0, cnt, slot); ++unit_iter) {
+          const int n0 = cnt >= 0 ? cnt : kv_tiles_for<CAUSAL>(2 * pair, p.n_kv);
+          const int n1 = cnt >= 0 ? cnt : kv_tiles_for<CAUSAL>(2 * pair + 1, p.n_kv);
           for (int t = 0; t < 2 && ok; ++t)
             ok = wait_bounded(BAR(B_Q_FULL + t), unit_iter & 1, wc, 10);
           if (!ok) break;
@@ -395,10 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     int s_cnt = 0, unit_iter = 0;
     bool ok = true;
-    int item = SNAKE ? 0 : int(blockIdx.x), half = 0, bh, pair;
-    for (; ok && next_unit<CAUSAL, SNAKE>(p, item, half, bh, pair); ++unit_iter) {
+    int item = MODE == kModeSnake ? 0 : int(blockIdx.x), half = 0, bh, pair, kv0, cnt, slot;
+    for (; ok && next_unit<CAUSAL, MODE>(p, item, half, bh, pair, kv0, cnt, slot); ++unit_iter) {
       const int qt = 2 * pair + t;
-      const int nt = kv_tiles_for<CAUSAL>(qt, p.n_kv);
+      const int nt = cnt >= 0 ? cnt : kv_tiles_for<CAUSAL>(qt, p.n_kv);
       const int row = qt * kBM + r;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nt; ++j) {
@@ -413,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
         // mask: the diagonal tile under the causal mask, and keys >= N
-        int limit = p.N - j * kBN;
+        int limit = p.N - (kv0 + j) * kBN;
         if (CAUSAL && j == qt) limit = min(limit, r + 1);
         if (limit < kBN) {
 #pragma unroll
@@ -490,6 +517,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.0f / l;
+      if (MODE == kModeSplit && slot >= 0) {
+        // a part of a split unit: O of this part (normalised by its own l)
+        // and its base-2 LSE go to the slot, for the merge kernel. It keeps
+        // the staging barriers' sequence (one phase of each per epilogue)
+        // without using the buffer.
+        float* po = p.part_o + ((size_t(slot) * 2 + t) * kBM + r) * D;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t orow[32];
+          tmem_ld32_wait(tO + ch * 32, orow);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            reinterpret_cast<float4*>(po + ch * 32)[v4] =
+                make_float4(__uint_as_float(orow[4 * v4 + 0]) * inv_l, __uint_as_float(orow[4 * v4 + 1]) * inv_l,
+                            __uint_as_float(orow[4 * v4 + 2]) * inv_l, __uint_as_float(orow[4 * v4 + 3]) * inv_l);
+        }
+        p.part_lse[(size_t(slot) * 2 + t) * kBM + r] = m + lg2_approx(l);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(BAR(B_O_EMPTY + t));
+          mbar_arrive(BAR(B_STG_READY + t));
+        }
+        if (r == 0 && wait_bounded(BAR(B_STG_READY + t), unit_iter & 1, wc, 24))
+          mbar_arrive(BAR(B_STG_FREE));
+        continue;
+      }
       uint8_t* stg = smem + L::kOffStg + r * 128;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -537,10 +591,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool SNAKE = false>
+// O and LSE of the split units from their parts ("Online Softmax": two
+// softmax partials over disjoint key sets combine exactly): with the parts'
+// base-2 LSEs L_i and normalised O_i, M = max L_i, w_i = 2^(L_i - M),
+// O = sum w_i O_i / sum w_i and LSE = ln2 (M + log2 sum w_i). One warp per
+// row, lanes striding the d columns.
+template <int D>
+__global__ void __launch_bounds__(256) fwd_merge_kernel(const FwdParams p, int n_units) {
+  const long long gw = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= static_cast<long long>(n_units) * 2 * kBM) return;
+  const int k = int(gw / (2 * kBM)), tr = int(gw % (2 * kBM));
+  const int t = tr / kBM, r = tr % kBM;
+  const int u = p.full_items + k;
+  const int bh = u / p.n_pairs, pair = u % p.n_pairs;
+  const int row = (2 * pair + t) * kBM + r;
+  if (row >= p.N) return;
+  const int S = p.split_s;  // 2..4
+  auto at = [&](int i) { return (size_t(k) * S + i) * 2 * kBM + size_t(t) * kBM + r; };
+  // every load of every part first (S <= 4), then the arithmetic
+  constexpr int kMaxParts = 4;
+  float L[kMaxParts], v[kMaxParts][D / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxParts; ++i) {
+    L[i] = -INFINITY;
+    if (i < S) {
+      L[i] = p.part_lse[at(i)];
+      const float* po = p.part_o + at(i) * D;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) v[i][q] = po[q * 32 + lane];
+    } else {
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) v[i][q] = 0.f;
+    }
+  }
+  const float M = fmaxf(fmaxf(L[0], L[1]), fmaxf(L[2], L[3]));
+  float acc[D / 32];
+#pragma unroll
+  for (int q = 0; q < D / 32; ++q) acc[q] = 0.f;
+  float wsum = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxParts; ++i) {
+    const float w = i < S ? ex2_approx(L[i] - M) : 0.f;
+    wsum += w;
+#pragma unroll
+    for (int q = 0; q < D / 32; ++q) acc[q] = fmaf(w, v[i][q], acc[q]);
+  }
+  const float inv = 1.0f / wsum;
+  uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + (size_t(bh) * p.N + row) * D;
+#pragma unroll
+  for (int q = 0; q < D / 32; ++q) orow[q * 32 + lane] = uint16_t(pack_bf16x2(acc[q] * inv, 0.f) & 0xffffu);
+  if (lane == 0) p.lse[size_t(bh) * p.N + row] = (M + lg2_approx(wsum)) * kLn2;
+}
+
+template <int D, bool CAUSAL, int MODE = kModePlain>
 fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                  const CUtensorMap& mo, const FwdParams& p, const LaunchCtx& ctx) {
-  auto kern = fwd_kernel<D, CAUSAL, SNAKE>;
+  auto kern = fwd_kernel<D, CAUSAL, MODE>;
   const int smem = Layout<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fwd)");
@@ -585,6 +692,10 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   p.n_pairs = (p.n_kv + 1) / 2;
   p.cpp = (p.n_pairs + 1) / 2;
   bool snake = false;
+  p.full_items = 0;
+  p.split_s = 1;
+  p.part_o = nullptr;
+  p.part_lse = nullptr;
   p.num_items = causal ? p.BH * p.cpp : p.BH * p.n_pairs;
   if (causal) {
     // couples carry equal work; if the last round of them leaves many CTAs
@@ -601,12 +712,49 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load;
-  if (d == 128) {
-    if (!causal) return launch<128, false>(mq, mk, mv, mo, p, ctx);
-    return snake ? launch<128, true, true>(mq, mk, mv, mo, p, ctx) : launch<128, true>(mq, mk, mv, mo, p, ctx);
+  if (causal) {
+    if (d == 128)
+      return snake ? launch<128, true, kModeSnake>(mq, mk, mv, mo, p, ctx) : launch<128, true>(mq, mk, mv, mo, p, ctx);
+    return snake ? launch<64, true, kModeSnake>(mq, mk, mv, mo, p, ctx) : launch<64, true>(mq, mk, mv, mo, p, ctx);
   }
-  if (!causal) return launch<64, false>(mq, mk, mv, mo, p, ctx);
-  return snake ? launch<64, true, true>(mq, mk, mv, mo, p, ctx) : launch<64, true>(mq, mk, mv, mo, p, ctx);
+  // no mask: if the last round of units fills at most half the CTAs, split
+  // its units along the keys (2-4 parts, each at least one K/V tile) and
+  // merge the parts afterwards
+  {
+    const int U = p.num_items;
+    const int G = U < ctx.num_sms ? U : ctx.num_sms;
+    const int full = U / G, rem = U - full * G;
+    int S = rem > 0 ? G / rem : 1;
+    S = S < 4 ? S : 4;
+    S = S < p.n_kv ? S : p.n_kv;
+    if (S >= 2) {
+      p.full_items = full * G;
+      p.split_s = S;
+      p.num_items = p.full_items + rem * S;
+      const size_t slots = size_t(rem) * S;
+      const size_t o_bytes = slots * 2 * kBM * size_t(d) * 4, l_bytes = slots * 2 * kBM * 4;
+      void* scratch = nullptr;
+      if ((st = scratch_alloc(o_bytes + l_bytes, ctx, &scratch)) != FA_OK) return st;
+      p.part_o = static_cast<float*>(scratch);
+      p.part_lse = reinterpret_cast<float*>(static_cast<char*>(scratch) + o_bytes);
+      st = d == 128 ? launch<128, false, kModeSplit>(mq, mk, mv, mo, p, ctx)
+                    : launch<64, false, kModeSplit>(mq, mk, mv, mo, p, ctx);
+      if (st == FA_OK) {
+        const long long threads = static_cast<long long>(rem) * 2 * kBM * 32;
+        const unsigned blocks = unsigned((threads + 255) / 256);
+        ProfileScope prof(KID_FWD_MERGE, ctx.stream);
+        if (d == 128)
+          fwd_merge_kernel<128><<<blocks, 256, 0, ctx.stream>>>(p, rem);
+        else
+          fwd_merge_kernel<64><<<blocks, 256, 0, ctx.stream>>>(p, rem);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) st = cuda_fail(e, "fwd merge kernel launch");
+      }
+      scratch_free(scratch, ctx);
+      return st;
+    }
+  }
+  return d == 128 ? launch<128, false>(mq, mk, mv, mo, p, ctx) : launch<64, false>(mq, mk, mv, mo, p, ctx);
 }
 
 }  // namespace fa

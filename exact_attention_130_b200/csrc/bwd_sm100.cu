@@ -84,7 +84,8 @@ enum : int {
   B_DRAIN = 10,
   B_DO_FULL = 11,      // +stage, dK/dV kernel: the dO block landed (B_ST_FULL: the Q block)
   B_DO_EMPTY = 13,     // +stage, dK/dV kernel: dV has read the dO block (B_ST_EMPTY: dK the Q block)
-  B_COUNT = 15
+  B_OUT_READY = 15,    // the compute warps have staged the output tiles (one arrival per warp)
+  B_COUNT = 16
 };
 
 struct BwdParams {
@@ -229,6 +230,7 @@ __device__ __forceinline__ uint32_t setup_cta(uint8_t* smem, int warp, volatile 
     mbar_init(bar(B_PHASE2), kComputeWarps);
     mbar_init(bar(B_ACC_DONE), 1);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_OUT_READY), kComputeWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -276,26 +278,28 @@ __device__ __forceinline__ void mma_tmem_x_rows(uint32_t d_tmem, uint32_t a_tmem
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// columns [c0, c0 + NC) of a TMEM accumulator row (this thread's lane) -> bf16
-// in global memory
-template <int NC>
-__device__ __forceinline__ void store_acc_cols(uint32_t t_acc, uint16_t* dst, int c0, bool valid) {
-  t_acc += c0;
-  dst += c0;
+// This thread's half of an accumulator row (TMEM lane r, columns half*D/2 ..)
+// as bf16 into a staged output tile: D/64 column groups of 128 rows x 128
+// bytes with the 128-byte swizzle of the tensor maps (16-byte chunk c of row
+// r at chunk c ^ (r % 8)), ready for TMA stores.
+template <int D>
+__device__ __forceinline__ void stage_acc_half(uint32_t t_acc, uint8_t* stg, int r, int half) {
+  constexpr int kSubBytes = kTile * 128;
 #pragma unroll
-  for (int ch = 0; ch < NC / 32; ++ch) {
+  for (int ch = 0; ch < D / 64; ++ch) {
+    const int c0 = half * (D / 2) + ch * 32;
     uint32_t v[32];
-    tmem_ld32_wait(t_acc + ch * 32, v);
-    if (valid) {
+    tmem_ld32_wait(t_acc + c0, v);
 #pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(v[8 * v4 + 0]), __uint_as_float(v[8 * v4 + 1]));
-        w.y = pack_bf16x2(__uint_as_float(v[8 * v4 + 2]), __uint_as_float(v[8 * v4 + 3]));
-        w.z = pack_bf16x2(__uint_as_float(v[8 * v4 + 4]), __uint_as_float(v[8 * v4 + 5]));
-        w.w = pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7]));
-        *reinterpret_cast<uint4*>(dst + ch * 32 + 8 * v4) = w;
-      }
+    for (int v4 = 0; v4 < 4; ++v4) {
+      uint4 w;
+      w.x = pack_bf16x2(__uint_as_float(v[8 * v4 + 0]), __uint_as_float(v[8 * v4 + 1]));
+      w.y = pack_bf16x2(__uint_as_float(v[8 * v4 + 2]), __uint_as_float(v[8 * v4 + 3]));
+      w.z = pack_bf16x2(__uint_as_float(v[8 * v4 + 4]), __uint_as_float(v[8 * v4 + 5]));
+      w.w = pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7]));
+      const int k16 = c0 / 8 + v4;          // 16-byte chunk of the row
+      const int g = k16 >> 3, cc = k16 & 7;  // column group, chunk in its 128-byte row
+      *reinterpret_cast<uint4*>(stg + g * kSubBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
     }
   }
 }
@@ -367,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmQX, const __grid_constant__ CUtensorMap tmDX,
+                    const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                     const BwdParams p) {
   using L = Plan<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -576,11 +581,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      // dV and dK as bf16 into the first Q/dO slot (idle once every MMA is
+      // done), then TMA stores; key rows past N fall outside the tensor
       tc_fence_after();
-      const size_t gro = (size_t(bh) * p.N + key) * D;
-      const bool row_valid = key < p.N;
-      store_acc_cols<D / 2>(tmem + lane_base + L::kColAcc0, p.dv + gro, half * (D / 2), row_valid);
-      store_acc_cols<D / 2>(tmem + lane_base + L::kColAcc1, p.dk + gro, half * (D / 2), row_valid);
+      uint8_t* stg = smem + L::kOffStage;
+      stage_acc_half<D>(tmem + lane_base + L::kColAcc0, stg, r, half);
+      stage_acc_half<D>(tmem + lane_base + L::kColAcc1, stg + L::kTileBytes, r, half);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_OUT_READY));
+      if (warp == 0 && lane == 0 && wait_bounded(BAR(B_OUT_READY), 0, wc, 24)) {
+        for (int c = 0; c < L::kGroups; ++c) {
+          tma_store_3d(&tmDV, sbase + L::kOffStage + c * L::kSubBytes, c * 64, jt * kTile, bh);
+          tma_store_3d(&tmDK, sbase + L::kOffStage + L::kTileBytes + c * L::kSubBytes, c * 64, jt * kTile, bh);
+        }
+        bulk_commit_group();
+        bulk_wait_group0();
+      }
     }
   }
 
@@ -600,6 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
+                  const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap,
                   const BwdParams p) {
   using L = Plan<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -740,9 +758,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      // dQ as bf16 into the first K/V slot, then TMA stores (rows past N are
+      // clipped)
       tc_fence_after();
-      store_acc_cols<D / 2>(tmem + lane_base + L::kColAcc0, p.dq + (size_t(bh) * p.N + q) * D, half * (D / 2),
-                            q < p.N);
+      stage_acc_half<D>(tmem + lane_base + L::kColAcc0, smem + L::kOffStage, r, half);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_OUT_READY));
+      if (warp == 0 && lane == 0 && wait_bounded(BAR(B_OUT_READY), 0, wc, 23)) {
+        for (int c = 0; c < L::kGroups; ++c)
+          tma_store_3d(&tmDQ, sbase + L::kOffStage + c * L::kSubBytes, c * 64, it_q * kTile, bh);
+        bulk_commit_group();
+        bulk_wait_group0();
+      }
     }
   }
 
@@ -772,7 +800,7 @@ fa_status launch_main(Kern kern, unsigned kid, int smem, unsigned grid, const CU
   }
   {
     ProfileScope prof(kid, ctx.stream);
-    kern<<<grid, kThreads, smem, ctx.stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
+    kern<<<grid, kThreads, smem, ctx.stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
@@ -782,9 +810,11 @@ fa_status launch_main(Kern kern, unsigned kid, int smem, unsigned grid, const CU
 template <int D, bool CAUSAL>
 fa_status launch_all(const void* q, const void* k, const void* v, const void* dO, const BwdParams& p,
                      const LaunchCtx& ctx) {
+  // maps 0-3: Q, dO, K, V; 4-5: extension rows; 6-7: outputs (dK, dV for the
+  // key-tile kernel, dQ for the query-tile kernel)
   const int smem = Plan<D>::kSmemBytes;
   const unsigned grid = unsigned(p.n_tiles) * unsigned(p.BH);
-  CUtensorMap m[6];
+  CUtensorMap m[8], mq[8];
   const void* src[4] = {q, dO, k, v};
   for (int i = 0; i < 4; ++i) {
     fa_status st = make_tmap_3d(&m[i], src[i], true, D, p.N, p.BH, 64, kTile, 128);
@@ -792,11 +822,16 @@ fa_status launch_all(const void* q, const void* k, const void* v, const void* dO
   }
   fa_status st = make_tmap_3d(&m[4], p.qext, true, 16, p.Np, p.BH, 16, kTile, 32);
   if (st == FA_OK) st = make_tmap_3d(&m[5], p.dext, true, 16, p.Np, p.BH, 16, kTile, 32);
+  if (st == FA_OK) st = make_tmap_3d(&m[6], p.dk, true, D, p.N, p.BH, 64, kTile, 128);
+  if (st == FA_OK) st = make_tmap_3d(&m[7], p.dv, true, D, p.N, p.BH, 64, kTile, 128);
   if (st != FA_OK) return st;
-  st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid, m, p, ctx,
-                             "bwd dK/dV kernel");
+  for (int i = 0; i < 6; ++i) mq[i] = m[i];
+  st = make_tmap_3d(&mq[6], p.dq, true, D, p.N, p.BH, 64, kTile, 128);
   if (st != FA_OK) return st;
-  return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid, m, p, ctx, "bwd dQ kernel");
+  mq[7] = mq[6];
+  st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid, m, p, ctx, "bwd dK/dV kernel");
+  if (st != FA_OK) return st;
+  return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid, mq, p, ctx, "bwd dQ kernel");
 }
 
 }  // namespace

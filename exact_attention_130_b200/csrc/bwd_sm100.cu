@@ -84,8 +84,11 @@ enum : int {
   B_DRAIN = 10,
   B_DO_FULL = 11,      // +stage, dK/dV kernel: the dO block landed (B_ST_FULL: the Q block)
   B_DO_EMPTY = 13,     // +stage, dK/dV kernel: dV has read the dO block (B_ST_EMPTY: dK the Q block)
-  B_OUT_READY = 15,    // the compute warps have staged the output tiles (one arrival per warp)
-  B_COUNT = 16
+  B_OUT_READY = 15,    // +stage (dK/dV kernel), else 15: the compute warps have staged output tiles
+                       // (one arrival per warp)
+  B_RES_EMPTY = 17,    // dK/dV kernel: the item's last S^T and dP^T have read K, V
+  B_ACC_EMPTY = 18,    // dK/dV kernel: the compute warps have read the accumulators (one per warp)
+  B_COUNT = 19
 };
 
 struct BwdParams {
@@ -231,6 +234,9 @@ __device__ __forceinline__ uint32_t setup_cta(uint8_t* smem, int warp, volatile 
     mbar_init(bar(B_ACC_DONE), 1);
     mbar_init(bar(B_DRAIN), 1);
     mbar_init(bar(B_OUT_READY), kComputeWarps);
+    mbar_init(bar(B_OUT_READY + 1), kComputeWarps);
+    mbar_init(bar(B_RES_EMPTY), 1);
+    mbar_init(bar(B_ACC_EMPTY), kComputeWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -366,6 +372,20 @@ __device__ __forceinline__ void form_p_half(const uint32_t (&sr)[kHalfCols], uin
 // --------------------------------------------------------------------------
 // 2. dK, dV: key-tile-outer
 // --------------------------------------------------------------------------
+// Persistent work list of both main kernels: item = (b*h, tile), heaviest
+// level first (under the causal mask the key tiles that see the most query
+// blocks, and the query tiles that see the most key blocks); round r gives
+// CTA c item r G + c for even r and r G + G-1-c for odd r (G = grid size),
+// which evens out the sums.
+__device__ __forceinline__ bool bwd_item(const BwdParams& p, int round, int& bh, int& level) {
+  const int G = int(gridDim.x), c = int(blockIdx.x);
+  const int idx = round * G + ((round & 1) ? G - 1 - c : c);
+  if (idx >= p.n_tiles * p.BH) return false;
+  level = idx / p.BH;
+  bh = idx % p.BH;
+  return true;
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
@@ -380,11 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   auto BAR = [&](int i) -> uint32_t { return sbase + L::kOffBar + 8u * uint32_t(i); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // key tiles that see the most query blocks first, all heads of a level together
-  const int jt = blockIdx.x / p.BH;
-  const int bh = blockIdx.x % p.BH;
-  const int i0 = CAUSAL ? jt : 0;       // first query tile that sees these keys
-  const int n_blk = p.n_tiles - i0;
+  // items: (b*h, key tile jt); an item streams the query blocks i0 + it,
+  // it = 0 .. n_blk-1, that can see its keys
+  auto blocks_of = [&](int jt) { return CAUSAL ? p.n_tiles - jt : p.n_tiles; };
   // the all-ones tile that multiplies the extension columns (uniform, so its
   // swizzle does not matter); visible to the tensor core after the fence and
   // the barrier in setup_cta
@@ -395,12 +413,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = setup_cta<D>(smem, warp, abort_flag);
   const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_BWD};
   const uint32_t sK = sbase + L::kOffRes0, sV = sbase + L::kOffRes1;
-  // stage slot s: the Q block (+ its -L2 and -scale D) and the dO block, each
-  // with its own full / empty barriers (Q is released after dK, dO after dV)
-  auto q_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
-  auto do_addr = [&](int it) { return q_addr(it) + L::kTileBytes; };
-  auto qx_addr = [&](int it) { return q_addr(it) + 2 * L::kTileBytes; };
-  auto dx_addr = [&](int it) { return qx_addr(it) + L::kExtBytes; };
+  // stage slot s (global block g of this CTA uses slot g % 2): the Q block
+  // (+ its extension rows) and the dO block (+ its own), each with full /
+  // empty barriers (Q is released by dK, dO by dV). After an item's last
+  // block the slot of that block stages the item's dV and dK tiles for the
+  // TMA stores, which the producer issues before its next load into it.
+  auto q_addr = [&](int g) { return sbase + L::kOffStage + (g % kStages) * L::kStageBytes; };
+  auto do_addr = [&](int g) { return q_addr(g) + L::kTileBytes; };
+  auto qx_addr = [&](int g) { return q_addr(g) + 2 * L::kTileBytes; };
+  auto dx_addr = [&](int g) { return qx_addr(g) + L::kExtBytes; };
   const uint32_t sOnes = sbase + L::kOffOnes;
   const uint32_t tP = tmem + L::kColDP;        // P^T as bf16: columns 0-31 and 64-95 of the dP region
   const uint32_t tDS = tmem + L::kColDP + 32;  // dS^T as bf16: columns 32-63 and 96-127
@@ -410,31 +431,66 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kLoadWarp) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
-        int q_issued = 0, do_issued = 0;
-        mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
-        for (int c = 0; c < L::kGroups; ++c) {
-          tma_load_3d(sK + c * L::kSubBytes, &tmK, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
-          tma_load_3d(sV + c * L::kSubBytes, &tmV, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
+        int q_issued = 0, do_issued = 0, res_issued = 0;
+        // the item whose output is staged in slot s and not yet stored (-1:
+        // none), with its coordinates, and how many stagings slot s has seen
+        int pend_jt[kStages] = {-1, -1}, pend_bh[kStages] = {0, 0}, staged[kStages] = {0, 0};
+        auto flush = [&](int s) -> bool {
+          if (pend_jt[s] < 0) return true;
+          if (!wait_bounded(BAR(B_OUT_READY + s), staged[s] & 1, wc, 4)) return false;
+          ++staged[s];
+          const uint32_t stg = sbase + L::kOffStage + s * L::kStageBytes;
+          for (int c = 0; c < L::kGroups; ++c) {
+            tma_store_3d(&tmDV, stg + c * L::kSubBytes, c * 64, pend_jt[s] * kTile, pend_bh[s]);
+            tma_store_3d(&tmDK, stg + L::kTileBytes + c * L::kSubBytes, c * 64, pend_jt[s] * kTile,
+                         pend_bh[s]);
+          }
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          pend_jt[s] = -1;
+          return true;
+        };
+        bool ok = true;
+        int g = 0, bh, jt;
+        for (int round = 0; ok && bwd_item(p, round, bh, jt); ++round) {
+          const int i0 = CAUSAL ? jt : 0, n_blk = blocks_of(jt);
+          // resident K, V: the previous item's last S^T and dP^T have read them
+          if (!wait_bounded(BAR(B_RES_EMPTY), (round & 1) ^ 1, wc, 5)) break;
+          mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
+          for (int c = 0; c < L::kGroups; ++c) {
+            tma_load_3d(sK + c * L::kSubBytes, &tmK, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
+            tma_load_3d(sV + c * L::kSubBytes, &tmV, BAR(B_RES_FULL), c * 64, jt * kTile, bh);
+          }
+          ++res_issued;
+          for (int it = 0; it < n_blk; ++it, ++g) {
+            const int s = g % kStages, ph = ((g / kStages) & 1) ^ 1;
+            const int q0 = (i0 + it) * kTile;
+            if (!(ok = wait_bounded(BAR(B_ST_EMPTY + s), ph, wc, 1))) break;
+            if (!(ok = flush(s))) break;
+            const uint32_t sq = q_addr(g);
+            mbar_arrive_expect_tx(BAR(B_ST_FULL + s), L::kTileBytes + L::kExtBytes);
+            for (int c = 0; c < L::kGroups; ++c)
+              tma_load_3d(sq + c * L::kSubBytes, &tmQ, BAR(B_ST_FULL + s), c * 64, q0, bh);
+            tma_load_3d(qx_addr(g), &tmQX, BAR(B_ST_FULL + s), 0, q0, bh);
+            ++q_issued;
+            if (!(ok = wait_bounded(BAR(B_DO_EMPTY + s), ph, wc, 3))) break;
+            mbar_arrive_expect_tx(BAR(B_DO_FULL + s), L::kTileBytes + L::kExtBytes);
+            for (int c = 0; c < L::kGroups; ++c)
+              tma_load_3d(do_addr(g) + c * L::kSubBytes, &tmDO, BAR(B_DO_FULL + s), c * 64, q0, bh);
+            tma_load_3d(dx_addr(g), &tmDX, BAR(B_DO_FULL + s), 0, q0, bh);
+            ++do_issued;
+            if (it == n_blk - 1) {  // this slot will stage the item's output
+              pend_jt[s] = jt;
+              pend_bh[s] = bh;
+            }
+          }
         }
-        for (int it = 0; it < n_blk; ++it) {
-          const int s = it % kStages, ph = ((it / kStages) & 1) ^ 1;
-          const int q0 = (i0 + it) * kTile;
-          if (!wait_bounded(BAR(B_ST_EMPTY + s), ph, wc, 1)) break;
-          const uint32_t sq = q_addr(it);
-          mbar_arrive_expect_tx(BAR(B_ST_FULL + s), L::kTileBytes + L::kExtBytes);
-          for (int c = 0; c < L::kGroups; ++c)
-            tma_load_3d(sq + c * L::kSubBytes, &tmQ, BAR(B_ST_FULL + s), c * 64, q0, bh);
-          tma_load_3d(qx_addr(it), &tmQX, BAR(B_ST_FULL + s), 0, q0, bh);
-          ++q_issued;
-          if (!wait_bounded(BAR(B_DO_EMPTY + s), ph, wc, 3)) break;
-          mbar_arrive_expect_tx(BAR(B_DO_FULL + s), L::kTileBytes + L::kExtBytes);
-          for (int c = 0; c < L::kGroups; ++c)
-            tma_load_3d(do_addr(it) + c * L::kSubBytes, &tmDO, BAR(B_DO_FULL + s), c * 64, q0, bh);
-          tma_load_3d(dx_addr(it), &tmDX, BAR(B_DO_FULL + s), 0, q0, bh);
-          ++do_issued;
-        }
+        // the outputs still staged, oldest first
+        if (ok) ok = flush(g % kStages);
+        if (ok) ok = flush((g + 1) % kStages);
+        bulk_wait_group0();
         if (*abort_flag) {
-          wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
+          if (res_issued) wait_bounded(BAR(B_RES_FULL), (res_issued - 1) & 1, wc, 2, true);
           for (int s = 0; s < kStages; ++s) {
             const int cq = (q_issued - s + kStages - 1) / kStages;  // loads into slot s
             if (cq > 0) wait_bounded(BAR(B_ST_FULL + s), (cq - 1) & 1, wc, 2, true);
@@ -445,56 +501,78 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == kMmaWarp) {
       // ------------------------------------------------------------ MMA issuer
-      // per block i: S^T_i+1 as soon as S^T_i is in registers; then, once P^T
-      // and dS^T are in TMEM, dK_i, dV_i and dP^T_i+1 (the in-order tensor
-      // pipe makes dP^T_i+1 overwrite the dP region only after dK_i and dV_i
-      // have read it)
+      // per block g: S^T of the next block (which may open the next item) as
+      // soon as S^T_g is in registers; then, once P^T and dS^T are in TMEM,
+      // dK_g, dV_g and dP^T of the next block (the in-order tensor pipe makes
+      // it overwrite the dP region only after dK_g and dV_g have read it).
+      // An item's resident K, V are released after its last S^T and dP^T; a
+      // new item's first dK, dV (which overwrite the accumulators) wait until
+      // the compute warps have read the previous item's.
       if (lane == 0) {
-        bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
-        if (ok) ok = wait_bounded(BAR(B_ST_FULL + 0), 0, wc, 11);
-        if (ok) {
+        int round = 0, bh, jt;
+        bool ok = bwd_item(p, 0, bh, jt);
+        int n_blk = ok ? blocks_of(jt) : 0;
+        // the block after (round, it): (nround, nit), valid if has_next
+        int nround = 0, nit = 0, nbh = bh, njt = jt, nn_blk = n_blk;
+        auto issue_s = [&](int g, int r, int it_, int nb) -> bool {
+          if (it_ == 0 && !wait_bounded(BAR(B_RES_FULL), r & 1, wc, 10)) return false;
+          if (!wait_bounded(BAR(B_ST_FULL + g % kStages), (g / kStages) & 1, wc, 11)) return false;
           tc_fence_after();
-          mma_rows_x_rows<D>(tmem + L::kColS, sK, q_addr(0));            // S^T_0 - L/scale
-          mma_ext(tmem + L::kColS, sOnes, qx_addr(0));
+          mma_rows_x_rows<D>(tmem + L::kColS, sK, q_addr(g));  // S^T - L/scale
+          mma_ext(tmem + L::kColS, sOnes, qx_addr(g));
           tc_commit(BAR(B_S_FULL));
-        }
-        if (ok) ok = wait_bounded(BAR(B_DO_FULL + 0), 0, wc, 16);
-        if (ok) {
+          (void)nb;
+          return true;
+        };
+        auto issue_dp = [&](int g, int it_, int nb) -> bool {
+          if (!wait_bounded(BAR(B_DO_FULL + g % kStages), (g / kStages) & 1, wc, 16)) return false;
           tc_fence_after();
-          mma_rows_x_rows<D>(tmem + L::kColDP, sV, do_addr(0));          // dP^T_0 - D
-          mma_ext(tmem + L::kColDP, sOnes, dx_addr(0));
+          mma_rows_x_rows<D>(tmem + L::kColDP, sV, do_addr(g));  // dP^T - D
+          mma_ext(tmem + L::kColDP, sOnes, dx_addr(g));
           tc_commit(BAR(B_DP_FULL));
-        }
-        for (int it = 0; ok && it < n_blk; ++it) {
-          const int s = it % kStages;
+          if (it_ == nb - 1) tc_commit(BAR(B_RES_EMPTY));  // the item's last reads of K, V
+          return true;
+        };
+        if (ok) ok = issue_s(0, 0, 0, n_blk) && issue_dp(0, 0, n_blk);
+        for (int g = 0, it = 0; ok; ++g) {
+          // the next block
+          bool has_next = true;
           if (it + 1 < n_blk) {
-            const int s1 = (it + 1) % kStages, ph1 = ((it + 1) / kStages) & 1;
-            ok = wait_bounded(BAR(B_PHASE1), it & 1, wc, 12);
-            if (ok) ok = wait_bounded(BAR(B_ST_FULL + s1), ph1, wc, 13);
-            if (!ok) break;
-            tc_fence_after();
-            mma_rows_x_rows<D>(tmem + L::kColS, sK, q_addr(it + 1));     // S^T_i+1 - L/scale
-            mma_ext(tmem + L::kColS, sOnes, qx_addr(it + 1));
-            tc_commit(BAR(B_S_FULL));
+            nround = round, nit = it + 1, nbh = bh, njt = jt, nn_blk = n_blk;
+          } else {
+            nround = round + 1, nit = 0;
+            has_next = bwd_item(p, nround, nbh, njt);
+            nn_blk = has_next ? blocks_of(njt) : 0;
           }
-          ok = wait_bounded(BAR(B_PHASE2), it & 1, wc, 14);
+          const int s = g % kStages;
+          // within an item the next S^T goes first; across items it goes after
+          // this block's dK, dV, since it waits for the next item's K and V
+          // (loaded only once this item's last S^T and dP^T have read the
+          // resident tiles) and must not hold back the item's ACC_DONE
+          const bool next_same_item = has_next && nit != 0;
+          if (next_same_item) {
+            ok = wait_bounded(BAR(B_PHASE1), g & 1, wc, 12);
+            if (ok) ok = issue_s(g + 1, nround, nit, nn_blk);
+            if (!ok) break;
+          }
+          ok = wait_bounded(BAR(B_PHASE2), g & 1, wc, 14);
+          if (ok && it == 0 && round > 0) ok = wait_bounded(BAR(B_ACC_EMPTY), (round - 1) & 1, wc, 17);
           if (!ok) break;
           tc_fence_after();
-          mma_tmem_x_rows<D>(tmem + L::kColAcc1, tDS, q_addr(it), it > 0);   // dK += dS^T Q
+          mma_tmem_x_rows<D>(tmem + L::kColAcc1, tDS, q_addr(g), it > 0);   // dK += dS^T Q
           tc_commit(BAR(B_ST_EMPTY + s));
-          mma_tmem_x_rows<D>(tmem + L::kColAcc0, tP, do_addr(it), it > 0);   // dV += P^T dO
+          mma_tmem_x_rows<D>(tmem + L::kColAcc0, tP, do_addr(g), it > 0);   // dV += P^T dO
           tc_commit(BAR(B_DO_EMPTY + s));
-          if (it + 1 < n_blk) {
-            const int s1 = (it + 1) % kStages, ph1 = ((it + 1) / kStages) & 1;
-            ok = wait_bounded(BAR(B_DO_FULL + s1), ph1, wc, 17);
+          if (it == n_blk - 1) tc_commit(BAR(B_ACC_DONE));
+          if (!has_next) break;
+          if (!next_same_item) {
+            ok = wait_bounded(BAR(B_PHASE1), g & 1, wc, 12);
+            if (ok) ok = issue_s(g + 1, nround, nit, nn_blk);
             if (!ok) break;
-            tc_fence_after();
-            mma_rows_x_rows<D>(tmem + L::kColDP, sV, do_addr(it + 1));   // dP^T_i+1 - D
-            mma_ext(tmem + L::kColDP, sOnes, dx_addr(it + 1));
-            tc_commit(BAR(B_DP_FULL));
           }
+          if (!(ok = issue_dp(g + 1, nit, nn_blk))) break;
+          round = nround, it = nit, bh = nbh, jt = njt, n_blk = nn_blk;
         }
-        tc_commit(BAR(B_ACC_DONE));
         tc_commit(BAR(B_DRAIN));
         wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
       }
@@ -505,98 +583,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp w: TMEM lanes (key rows) 32 (w % 4) .., columns (queries) 64 (w / 4) ..
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;   // key row in the tile
-    const int key = jt * kTile + r;
     const uint32_t lane_base = uint32_t(quad * 32) << 16;
     const uint32_t tS = tmem + lane_base + L::kColS + half * kHalfCols;
     const uint32_t tDP = tmem + lane_base + L::kColDP + half * kHalfCols;
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     const uint64_t scale2 = f2_pack(p.scale, p.scale);
-    bool ok = true;
     // the per-query terms -L/scale and -D arrive inside S^T and dP^T (the
     // extension K step of their MMAs), so these warps read no shared memory:
     // while the tensor core streams its operands, shared-memory reads queue for
     // hundreds of cycles and would stall the exponentials and the barrier
     // arrivals behind them
     const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int it = 0; it < n_blk; ++it) {
-      ok = wait_bounded(BAR(B_S_FULL), it & 1, wc, 20);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const int q0 = (i0 + it) * kTile;
-      // phase 1: read S^T - L/scale (after which the next S^T may overwrite
-      // it) and form P^T = 2^(scale log2e (s - L_q/scale)) in registers. Only the first block under the
-      // causal mask hides queries (q < key). Rows past N are not masked: each
-      // row of dV and dK depends on its own row of P^T and dS^T only, and those
-      // rows are never stored.
-      uint64_t pr2[kHalfCols / 2];
-      {
-        uint32_t sr[kHalfCols];
-        tmem_ld64_wait(tS, sr);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(B_PHASE1));
-        auto nl4 = [&](int) { return zero4; };
-        if (CAUSAL && it == 0) {
-          const int qlim = key - q0 - half * kHalfCols;  // local columns below qlim are hidden
-          form_p_half<true>(sr, c2, nl4, [&](int i) { return i < qlim; }, pr2);
-        } else {
-          form_p_half<false>(sr, c2, nl4, [](int) { return false; }, pr2);
-        }
-      }
-      // phase 2: dS^T = P^T scale (dP^T - D_q); P^T and dS^T (bf16) then
-      // replace this warp's 64 dP^T columns: P^T in the first 32, dS^T in the
-      // last 32. Both chunks of dP^T are read before either store.
-      ok = wait_bounded(BAR(B_DP_FULL), it & 1, wc, 22);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      {
-        uint32_t pk_ds[kHalfCols / 2];
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t dr[32];
-          tmem_ld32_wait(tDP + ch * 32, dr);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint64_t t0 = f2_mul(f2_pack(__uint_as_float(dr[4 * j]), __uint_as_float(dr[4 * j + 1])), scale2);
-            const uint64_t t1 = f2_mul(f2_pack(__uint_as_float(dr[4 * j + 2]), __uint_as_float(dr[4 * j + 3])), scale2);
-            pk_ds[ch * 16 + 2 * j] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j], t0));
-            pk_ds[ch * 16 + 2 * j + 1] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j + 1], t1));
+    bool ok = true;
+    int g = 0, bh, jt;
+    for (int round = 0; ok && bwd_item(p, round, bh, jt); ++round) {
+      const int i0 = CAUSAL ? jt : 0, n_blk = blocks_of(jt);
+      const int key = jt * kTile + r;
+      for (int it = 0; it < n_blk; ++it, ++g) {
+        ok = wait_bounded(BAR(B_S_FULL), g & 1, wc, 20);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const int q0 = (i0 + it) * kTile;
+        // phase 1: read S^T - L/scale (after which the next S^T may overwrite
+        // it) and form P^T = 2^(scale log2e (s - L_q/scale)) in registers. Only
+        // the first block under the causal mask hides queries (q < key). Rows
+        // past N are not masked: each row of dV and dK depends on its own row
+        // of P^T and dS^T only, and those rows are never stored.
+        uint64_t pr2[kHalfCols / 2];
+        {
+          uint32_t sr[kHalfCols];
+          tmem_ld64_wait(tS, sr);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(B_PHASE1));
+          auto nl4 = [&](int) { return zero4; };
+          if (CAUSAL && it == 0) {
+            const int qlim = key - q0 - half * kHalfCols;  // local columns below qlim are hidden
+            form_p_half<true>(sr, c2, nl4, [&](int i) { return i < qlim; }, pr2);
+          } else {
+            form_p_half<false>(sr, c2, nl4, [](int) { return false; }, pr2);
           }
         }
-        uint32_t pk_p[kHalfCols / 2];
+        // phase 2: dS^T = P^T scale (dP^T - D_q); P^T and dS^T (bf16) then
+        // replace this warp's 64 dP^T columns: P^T in the first 32, dS^T in the
+        // last 32. Both chunks of dP^T are read before either store.
+        ok = wait_bounded(BAR(B_DP_FULL), g & 1, wc, 22);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        {
+          uint32_t pk_ds[kHalfCols / 2];
 #pragma unroll
-        for (int i = 0; i < kHalfCols / 2; ++i) pk_p[i] = f2_to_bf16x2(pr2[i]);
-        tmem_st32(tDP, pk_p);
-        tmem_st32(tDP + 32, pk_ds);
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t dr[32];
+            tmem_ld32_wait(tDP + ch * 32, dr);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint64_t t0 = f2_mul(f2_pack(__uint_as_float(dr[4 * j]), __uint_as_float(dr[4 * j + 1])), scale2);
+              const uint64_t t1 = f2_mul(f2_pack(__uint_as_float(dr[4 * j + 2]), __uint_as_float(dr[4 * j + 3])), scale2);
+              pk_ds[ch * 16 + 2 * j] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j], t0));
+              pk_ds[ch * 16 + 2 * j + 1] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j + 1], t1));
+            }
+          }
+          uint32_t pk_p[kHalfCols / 2];
+#pragma unroll
+          for (int i = 0; i < kHalfCols / 2; ++i) pk_p[i] = f2_to_bf16x2(pr2[i]);
+          tmem_st32(tDP, pk_p);
+          tmem_st32(tDP + 32, pk_ds);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_PHASE2));
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_PHASE2));
-    }
-    if (ok) {
-      ok = wait_bounded(BAR(B_ACC_DONE), 0, wc, 23);
+      if (!ok) break;
+      // epilogue of the item: dV and dK as bf16 into the slot of its last
+      // block (idle once every MMA of the item is done); the producer stores
+      // them with TMA before it loads into that slot again. Key rows past N
+      // fall outside the tensor.
+      ok = wait_bounded(BAR(B_ACC_DONE), round & 1, wc, 23);
       ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      // dV and dK as bf16 into the first Q/dO slot (idle once every MMA is
-      // done), then TMA stores; key rows past N fall outside the tensor
+      if (!ok) break;
       tc_fence_after();
-      uint8_t* stg = smem + L::kOffStage;
+      const int s = (g - 1) % kStages;
+      uint8_t* stg = smem + L::kOffStage + s * L::kStageBytes;
       stage_acc_half<D>(tmem + lane_base + L::kColAcc0, stg, r, half);
       stage_acc_half<D>(tmem + lane_base + L::kColAcc1, stg + L::kTileBytes, r, half);
+      tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_OUT_READY));
-      if (warp == 0 && lane == 0 && wait_bounded(BAR(B_OUT_READY), 0, wc, 24)) {
-        for (int c = 0; c < L::kGroups; ++c) {
-          tma_store_3d(&tmDV, sbase + L::kOffStage + c * L::kSubBytes, c * 64, jt * kTile, bh);
-          tma_store_3d(&tmDK, sbase + L::kOffStage + L::kTileBytes + c * L::kSubBytes, c * 64, jt * kTile, bh);
-        }
-        bulk_commit_group();
-        bulk_wait_group0();
+      if (lane == 0) {
+        mbar_arrive(BAR(B_ACC_EMPTY));
+        mbar_arrive(BAR(B_OUT_READY + s));
       }
     }
   }
@@ -829,7 +908,9 @@ fa_status launch_all(const void* q, const void* k, const void* v, const void* dO
   st = make_tmap_3d(&mq[6], p.dq, true, D, p.N, p.BH, 64, kTile, 128);
   if (st != FA_OK) return st;
   mq[7] = mq[6];
-  st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid, m, p, ctx, "bwd dK/dV kernel");
+  // the dK/dV kernel is persistent: one CTA per SM walks its items
+  const unsigned grid_kv = grid < unsigned(ctx.num_sms) ? grid : unsigned(ctx.num_sms);
+  st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid_kv, m, p, ctx, "bwd dK/dV kernel");
   if (st != FA_OK) return st;
   return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid, mq, p, ctx, "bwd dQ kernel");
 }

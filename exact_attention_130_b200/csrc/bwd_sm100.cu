@@ -84,10 +84,10 @@ enum : int {
   B_DRAIN = 10,
   B_DO_FULL = 11,      // +stage, dK/dV kernel: the dO block landed (B_ST_FULL: the Q block)
   B_DO_EMPTY = 13,     // +stage, dK/dV kernel: dV has read the dO block (B_ST_EMPTY: dK the Q block)
-  B_OUT_READY = 15,    // +stage (dK/dV kernel), else 15: the compute warps have staged output tiles
+  B_OUT_READY = 15,    // +stage: the compute warps have staged an item's output tiles in that slot
                        // (one arrival per warp)
-  B_RES_EMPTY = 17,    // dK/dV kernel: the item's last S^T and dP^T have read K, V
-  B_ACC_EMPTY = 18,    // dK/dV kernel: the compute warps have read the accumulators (one per warp)
+  B_RES_EMPTY = 17,    // the item's last S and dP MMAs have read the resident tiles
+  B_ACC_EMPTY = 18,    // the compute warps have read the accumulators (one arrival per warp)
   B_COUNT = 19
 };
 
@@ -705,40 +705,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   auto BAR = [&](int i) -> uint32_t { return sbase + L::kOffBar + 8u * uint32_t(i); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // query tiles that see the most key blocks first (causal: the last ones)
-  const int lvl = blockIdx.x / p.BH;
-  const int it_q = CAUSAL ? p.n_tiles - 1 - lvl : lvl;
-  const int bh = blockIdx.x % p.BH;
-  const int n_blk = CAUSAL ? it_q + 1 : p.n_tiles;  // key tiles this query tile sees
+  // items: (b*h, query tile it_q), the tiles that see the most key blocks
+  // first (causal: the last ones); an item streams key blocks 0 .. n_blk-1
+  auto tile_of = [&](int level) { return CAUSAL ? p.n_tiles - 1 - level : level; };
+  auto blocks_of = [&](int it_q) { return CAUSAL ? it_q + 1 : p.n_tiles; };
   volatile int* abort_flag;
   const uint32_t tmem = setup_cta<D>(smem, warp, abort_flag);
   const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_BWD_DQ};
   const uint32_t sQ = sbase + L::kOffRes0, sDO = sbase + L::kOffRes1;
-  auto stage_addr = [&](int it) { return sbase + L::kOffStage + (it % kStages) * L::kStageBytes; };
+  // global block g of this CTA uses slot g % 2 (K then V); after an item's
+  // last block the K part of its slot stages the item's dQ tile, which the
+  // producer stores with TMA before its next load into that slot
+  auto stage_addr = [&](int g) { return sbase + L::kOffStage + (g % kStages) * L::kStageBytes; };
 
   if (warp >= 8) {
     regs_decrease<kRegsControl>();
     if (warp == kLoadWarp) {
       if (lane == 0) {
-        int issued = 0;
-        mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
-        for (int c = 0; c < L::kGroups; ++c) {
-          tma_load_3d(sQ + c * L::kSubBytes, &tmQ, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
-          tma_load_3d(sDO + c * L::kSubBytes, &tmDO, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
-        }
-        for (int it = 0; it < n_blk; ++it) {
-          const int s = it % kStages;
-          if (!wait_bounded(BAR(B_ST_EMPTY + s), ((it / kStages) & 1) ^ 1, wc, 1)) break;
-          const uint32_t st = stage_addr(it);
-          mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kTileBytes);
+        int issued = 0, res_issued = 0;
+        int pend_q[kStages] = {-1, -1}, pend_bh[kStages] = {0, 0}, staged[kStages] = {0, 0};
+        auto flush = [&](int s) -> bool {
+          if (pend_q[s] < 0) return true;
+          if (!wait_bounded(BAR(B_OUT_READY + s), staged[s] & 1, wc, 4)) return false;
+          ++staged[s];
+          for (int c = 0; c < L::kGroups; ++c)
+            tma_store_3d(&tmDQ, sbase + L::kOffStage + s * L::kStageBytes + c * L::kSubBytes, c * 64,
+                         pend_q[s] * kTile, pend_bh[s]);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          pend_q[s] = -1;
+          return true;
+        };
+        bool ok = true;
+        int g = 0, bh, lvl;
+        for (int round = 0; ok && bwd_item(p, round, bh, lvl); ++round) {
+          const int it_q = tile_of(lvl), n_blk = blocks_of(it_q);
+          if (!wait_bounded(BAR(B_RES_EMPTY), (round & 1) ^ 1, wc, 5)) break;
+          mbar_arrive_expect_tx(BAR(B_RES_FULL), 2 * L::kTileBytes);
           for (int c = 0; c < L::kGroups; ++c) {
-            tma_load_3d(st + c * L::kSubBytes, &tmK, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
-            tma_load_3d(st + L::kTileBytes + c * L::kSubBytes, &tmV, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
+            tma_load_3d(sQ + c * L::kSubBytes, &tmQ, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
+            tma_load_3d(sDO + c * L::kSubBytes, &tmDO, BAR(B_RES_FULL), c * 64, it_q * kTile, bh);
           }
-          ++issued;
+          ++res_issued;
+          for (int it = 0; it < n_blk; ++it, ++g) {
+            const int s = g % kStages;
+            if (!(ok = wait_bounded(BAR(B_ST_EMPTY + s), ((g / kStages) & 1) ^ 1, wc, 1))) break;
+            if (!(ok = flush(s))) break;
+            const uint32_t st = stage_addr(g);
+            mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kTileBytes);
+            for (int c = 0; c < L::kGroups; ++c) {
+              tma_load_3d(st + c * L::kSubBytes, &tmK, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
+              tma_load_3d(st + L::kTileBytes + c * L::kSubBytes, &tmV, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
+            }
+            ++issued;
+            if (it == n_blk - 1) {
+              pend_q[s] = it_q;
+              pend_bh[s] = bh;
+            }
+          }
         }
+        if (ok) ok = flush(g % kStages);
+        if (ok) ok = flush((g + 1) % kStages);
+        bulk_wait_group0();
         if (*abort_flag) {
-          wait_bounded(BAR(B_RES_FULL), 0, wc, 2, true);
+          if (res_issued) wait_bounded(BAR(B_RES_FULL), (res_issued - 1) & 1, wc, 2, true);
           for (int s = 0; s < kStages; ++s) {
             const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
             if (cnt > 0) wait_bounded(BAR(B_ST_FULL + s), (cnt - 1) & 1, wc, 2, true);
@@ -746,38 +776,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else if (warp == kMmaWarp) {
-      // order per block j: S_j+1 (once S_j is in registers), dQ_j (after
-      // phase 2), dP_j+1
+      // per block g: S of the next block of the same item once S_g is in
+      // registers; dQ_g after phase 2; then (for a new item, after dQ_g, since
+      // it waits for the item's resident Q and dO) S of the next block, and
+      // dP of the next block. An item's resident Q, dO are released after its
+      // last S and dP; a new item's first dQ (which overwrites the
+      // accumulator) waits until the compute warps have read the previous one.
       if (lane == 0) {
-        bool ok = wait_bounded(BAR(B_RES_FULL), 0, wc, 10);
-        if (ok) ok = wait_bounded(BAR(B_ST_FULL + 0), 0, wc, 11);
-        if (ok) {
+        int round = 0, bh, lvl;
+        bool ok = bwd_item(p, 0, bh, lvl);
+        int n_blk = ok ? blocks_of(tile_of(lvl)) : 0;
+        int nround = 0, nit = 0, nbh = bh, nlvl = lvl, nn_blk = n_blk;
+        auto issue_s = [&](int g, int r, int it_) -> bool {
+          if (it_ == 0 && !wait_bounded(BAR(B_RES_FULL), r & 1, wc, 10)) return false;
+          if (!wait_bounded(BAR(B_ST_FULL + g % kStages), (g / kStages) & 1, wc, 11)) return false;
           tc_fence_after();
-          mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(0));                     // S_0
+          mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(g));  // S = Q K^T
           tc_commit(BAR(B_S_FULL));
-          mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(0) + L::kTileBytes);   // dP_0
+          return true;
+        };
+        auto issue_dp = [&](int g, int it_, int nb) {
+          mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(g) + L::kTileBytes);  // dP = dO V^T
           tc_commit(BAR(B_DP_FULL));
-        }
-        for (int it = 0; ok && it < n_blk; ++it) {
+          if (it_ == nb - 1) tc_commit(BAR(B_RES_EMPTY));  // the item's last reads of Q, dO
+        };
+        if (ok && (ok = issue_s(0, 0, 0))) issue_dp(0, 0, n_blk);
+        for (int g = 0, it = 0; ok; ++g) {
+          bool has_next = true;
           if (it + 1 < n_blk) {
-            ok = wait_bounded(BAR(B_PHASE1), it & 1, wc, 12);
-            if (ok) ok = wait_bounded(BAR(B_ST_FULL + (it + 1) % kStages), ((it + 1) / kStages) & 1, wc, 13);
-            if (!ok) break;
-            tc_fence_after();
-            mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(it + 1));              // S_j+1
-            tc_commit(BAR(B_S_FULL));
+            nround = round, nit = it + 1, nbh = bh, nlvl = lvl, nn_blk = n_blk;
+          } else {
+            nround = round + 1, nit = 0;
+            has_next = bwd_item(p, nround, nbh, nlvl);
+            nn_blk = has_next ? blocks_of(tile_of(nlvl)) : 0;
           }
-          ok = wait_bounded(BAR(B_PHASE2), it & 1, wc, 14);
+          const bool next_same_item = has_next && nit != 0;
+          if (next_same_item) {
+            ok = wait_bounded(BAR(B_PHASE1), g & 1, wc, 12);
+            if (ok) ok = issue_s(g + 1, nround, nit);
+            if (!ok) break;
+          }
+          ok = wait_bounded(BAR(B_PHASE2), g & 1, wc, 14);
+          if (ok && it == 0 && round > 0) ok = wait_bounded(BAR(B_ACC_EMPTY), (round - 1) & 1, wc, 17);
           if (!ok) break;
           tc_fence_after();
-          mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColDP, stage_addr(it), it > 0);  // dQ += dS K
-          tc_commit(BAR(B_ST_EMPTY + it % kStages));
-          if (it + 1 < n_blk) {
-            mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(it + 1) + L::kTileBytes);  // dP_j+1
-            tc_commit(BAR(B_DP_FULL));
+          mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColDP, stage_addr(g), it > 0);  // dQ += dS K
+          tc_commit(BAR(B_ST_EMPTY + g % kStages));
+          if (it == n_blk - 1) tc_commit(BAR(B_ACC_DONE));
+          if (!has_next) break;
+          if (!next_same_item) {
+            ok = wait_bounded(BAR(B_PHASE1), g & 1, wc, 12);
+            if (ok) ok = issue_s(g + 1, nround, nit);
+            if (!ok) break;
           }
+          issue_dp(g + 1, nit, nn_blk);
+          round = nround, it = nit, bh = nbh, lvl = nlvl, n_blk = nn_blk;
         }
-        tc_commit(BAR(B_ACC_DONE));
         tc_commit(BAR(B_DRAIN));
         wait_bounded(BAR(B_DRAIN), 0, wc, 15, true);
       }
@@ -787,68 +841,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp w: TMEM lanes (query rows) 32 (w % 4) .., columns (keys) 64 (w / 4) ..
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;   // query row in the tile
-    const int q = it_q * kTile + r;
     const uint32_t lane_base = uint32_t(quad * 32) << 16;
     const uint32_t tS = tmem + lane_base + L::kColS + half * kHalfCols;
     const uint32_t tDP = tmem + lane_base + L::kColDP + half * kHalfCols;
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     const uint64_t scale2 = f2_pack(p.scale, p.scale);
-    const float nl2q = p.lse2[size_t(bh) * p.Np + q];  // -inf past N (q < Np always)
-    const float nsdq = p.dvec[size_t(bh) * p.Np + q];
-    const float4 nl2q4 = make_float4(nl2q, nl2q, nl2q, nl2q);
-    const float4 nsdq4 = make_float4(nsdq, nsdq, nsdq, nsdq);
     bool ok = true;
-    for (int it = 0; it < n_blk; ++it) {
-      ok = wait_bounded(BAR(B_S_FULL), it & 1, wc, 20);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const int k0 = it * kTile;
-      // phase 1: read S (then the MMA may overwrite it) and form P
-      uint32_t sr[kHalfCols];
-      tmem_ld64_wait(tS, sr);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_PHASE1));
-      uint64_t pr2[kHalfCols / 2];
-      auto nl4 = [&](int) { return nl2q4; };
-      // keys past N, or (causal) past q, are hidden: only the last block has any
-      if ((CAUSAL && it == n_blk - 1) || k0 + kTile > p.N) {
-        int klim = p.N - k0;
-        if (CAUSAL) klim = min(klim, q - k0 + 1);
-        klim -= half * kHalfCols;  // local columns at or above klim are hidden
-        form_p_half<true>(sr, c2, nl4, [&](int i) { return i >= klim; }, pr2);
-      } else {
-        form_p_half<false>(sr, c2, nl4, [](int) { return false; }, pr2);
+    int g = 0, bh, lvl;
+    // this row's -L2 and -scale D (-inf and 0 past N; q < Np always), read one
+    // item ahead so the load hides behind the previous item's epilogue
+    bool have = bwd_item(p, 0, bh, lvl);
+    float nl2q = 0.f, nsdq = 0.f;
+    if (have) {
+      const size_t at = size_t(bh) * p.Np + tile_of(lvl) * kTile + r;
+      nl2q = p.lse2[at];
+      nsdq = p.dvec[at];
+    }
+    for (int round = 0; ok && have; ++round) {
+      const int it_q = tile_of(lvl), n_blk = blocks_of(it_q);
+      const int q = it_q * kTile + r;
+      const float4 nl2q4 = make_float4(nl2q, nl2q, nl2q, nl2q);
+      const float4 nsdq4 = make_float4(nsdq, nsdq, nsdq, nsdq);
+      for (int it = 0; it < n_blk; ++it, ++g) {
+        ok = wait_bounded(BAR(B_S_FULL), g & 1, wc, 20);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const int k0 = it * kTile;
+        // phase 1: read S (then the MMA may overwrite it) and form P
+        uint32_t sr[kHalfCols];
+        tmem_ld64_wait(tS, sr);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_PHASE1));
+        uint64_t pr2[kHalfCols / 2];
+        auto nl4 = [&](int) { return nl2q4; };
+        // keys past N, or (causal) past q, are hidden: only the last block has any
+        if ((CAUSAL && it == n_blk - 1) || k0 + kTile > p.N) {
+          int klim = p.N - k0;
+          if (CAUSAL) klim = min(klim, q - k0 + 1);
+          klim -= half * kHalfCols;  // local columns at or above klim are hidden
+          form_p_half<true>(sr, c2, nl4, [&](int i) { return i >= klim; }, pr2);
+        } else {
+          form_p_half<false>(sr, c2, nl4, [](int) { return false; }, pr2);
+        }
+        // phase 2: dS = P (scale dP - scale D_q), written back over dP as bf16
+        ok = wait_bounded(BAR(B_DP_FULL), g & 1, wc, 21);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        write_ds_half(tDP, pr2, scale2, [&](int) { return nsdq4; });
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_PHASE2));
       }
-      // phase 2: dS = P (scale dP - scale D_q), written back over dP as bf16
-      ok = wait_bounded(BAR(B_DP_FULL), it & 1, wc, 21);
+      if (!ok) break;
+      // the next item's row terms, then the epilogue of this one: dQ as bf16
+      // into the K part of the last block's slot (idle once every MMA of the
+      // item is done); the producer stores it with TMA (rows past N clipped)
+      have = bwd_item(p, round + 1, bh, lvl);
+      if (have) {
+        const size_t at = size_t(bh) * p.Np + tile_of(lvl) * kTile + r;
+        nl2q = p.lse2[at];
+        nsdq = p.dvec[at];
+      }
+      ok = wait_bounded(BAR(B_ACC_DONE), round & 1, wc, 22);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      write_ds_half(tDP, pr2, scale2, [&](int) { return nsdq4; });
-      tmem_st_wait();
+      const int s = (g - 1) % kStages;
+      stage_acc_half<D>(tmem + lane_base + L::kColAcc0, smem + L::kOffStage + s * L::kStageBytes, r, half);
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_PHASE2));
-    }
-    if (ok) {
-      ok = wait_bounded(BAR(B_ACC_DONE), 0, wc, 22);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      // dQ as bf16 into the first K/V slot, then TMA stores (rows past N are
-      // clipped)
-      tc_fence_after();
-      stage_acc_half<D>(tmem + lane_base + L::kColAcc0, smem + L::kOffStage, r, half);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_OUT_READY));
-      if (warp == 0 && lane == 0 && wait_bounded(BAR(B_OUT_READY), 0, wc, 23)) {
-        for (int c = 0; c < L::kGroups; ++c)
-          tma_store_3d(&tmDQ, sbase + L::kOffStage + c * L::kSubBytes, c * 64, it_q * kTile, bh);
-        bulk_commit_group();
-        bulk_wait_group0();
+      if (lane == 0) {
+        mbar_arrive(BAR(B_ACC_EMPTY));
+        mbar_arrive(BAR(B_OUT_READY + s));
       }
     }
   }
@@ -908,11 +977,11 @@ fa_status launch_all(const void* q, const void* k, const void* v, const void* dO
   st = make_tmap_3d(&mq[6], p.dq, true, D, p.N, p.BH, 64, kTile, 128);
   if (st != FA_OK) return st;
   mq[7] = mq[6];
-  // the dK/dV kernel is persistent: one CTA per SM walks its items
+  // both kernels are persistent: one CTA per SM walks its items
   const unsigned grid_kv = grid < unsigned(ctx.num_sms) ? grid : unsigned(ctx.num_sms);
   st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid_kv, m, p, ctx, "bwd dK/dV kernel");
   if (st != FA_OK) return st;
-  return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid, mq, p, ctx, "bwd dQ kernel");
+  return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid_kv, mq, p, ctx, "bwd dQ kernel");
 }
 
 }  // namespace

@@ -479,9 +479,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
         const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_m, neg_m);
         uint64_t sum_a = f2_pack(0.f, 0.f), sum_b = sum_a;
+        // P goes to TMEM in 32-column chunks as they are formed, so the stores
+        // overlap the remaining exponentials (S is already in registers)
         uint32_t pk[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
+          if (i > 0 && (i & 15) == 0) tmem_st16(tS + (i - 16), *reinterpret_cast<uint32_t(*)[16]>(pk + i - 16));
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), c2, nm2), x0, x1);
           const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
@@ -491,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sum_a = f2_add(sum_a, f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st64(tS, pk);
+        tmem_st16(tS + 48, *reinterpret_cast<uint32_t(*)[16]>(pk + 48));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

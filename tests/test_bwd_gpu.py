@@ -64,6 +64,21 @@ def test_bwd_small(shape, causal):
     check(x, causal)
 
 
+# more (head, tile) items than SMs, so every CTA of the persistent kernels
+# walks several items: d = 64, a ragged last tile, and N = 256 (two tiles:
+# under the mask half the items are a single block, so consecutive items
+# stage their outputs in both slots before the producer stores them)
+MULTI = [(2, 40, 512, 64), (1, 30, 700, 128), (4, 40, 256, 64)]
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("shape", MULTI, ids=lambda s: "x".join(map(str, s)))
+def test_bwd_persistent_multi_item(shape, causal):
+    B, H, N, d = shape
+    x = inputgen.make_small_inputs(3000 + N + H, B, H, N, d, with_grad=True)
+    check(x, causal)
+
+
 def test_bwd_workload_every_head():
     """B=2, H=16, N=4096, d=128, causal; compared in full for every head."""
     w = inputgen.WORKLOADS["backward"]

@@ -69,6 +69,7 @@ constexpr int kMmaWarp = 9;
 constexpr int kComputeWarps = 8;
 constexpr int kHalfCols = kTile / 2;  // columns of a row each compute warp owns
 constexpr int kStages = 2;
+constexpr int kKSlots = 3;   // dQ kernel: K ring depth (its V ring has kStages slots)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // barrier slots (shared by both kernels)
@@ -88,7 +89,10 @@ enum : int {
                        // (one arrival per warp)
   B_RES_EMPTY = 17,    // the item's last S and dP MMAs have read the resident tiles
   B_ACC_EMPTY = 18,    // the compute warps have read the accumulators (one arrival per warp)
-  B_COUNT = 19
+  B_K_FULL = 19,       // +slot (3), dQ kernel: a K block landed (B_DO_FULL: a V block)
+  B_K_EMPTY = 22,      // +slot (3), dQ kernel: dQ has read the K block (B_DO_EMPTY: dP the V block)
+  B_KOUT_READY = 25,   // +slot (3), dQ kernel: dQ staged in that K slot (one arrival per warp)
+  B_COUNT = 28
 };
 
 struct BwdParams {
@@ -138,7 +142,13 @@ struct Plan {
   // a stage: two streamed tiles, then (dK/dV kernel) the extension tiles of
   // the Q block and of the dO block
   static constexpr int kStageBytes = 2 * kTileBytes + 2 * kExtBytes;
-  static constexpr int kOffBar = kOffStage + kStages * kStageBytes;
+  // dQ kernel: resident Q, dO at kOffRes0/1, then a ring of kKSlots K tiles
+  // and a ring of kStages V tiles (no extension tiles, no ones tile)
+  static constexpr int kOffKRing = 2 * kTileBytes;
+  static constexpr int kOffVRing = kOffKRing + kKSlots * kTileBytes;
+  static constexpr int kDqEnd = kOffVRing + kStages * kTileBytes;
+  static constexpr int kStageEnd = kOffStage + kStages * kStageBytes;
+  static constexpr int kOffBar = kStageEnd > kDqEnd ? kStageEnd : kDqEnd;
   static constexpr int kOffMisc = kOffBar + 8 * B_COUNT;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;
   // TMEM columns
@@ -237,6 +247,11 @@ __device__ __forceinline__ uint32_t setup_cta(uint8_t* smem, int warp, volatile 
     mbar_init(bar(B_OUT_READY + 1), kComputeWarps);
     mbar_init(bar(B_RES_EMPTY), 1);
     mbar_init(bar(B_ACC_EMPTY), kComputeWarps);
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(bar(B_K_FULL + s), 1);
+      mbar_init(bar(B_K_EMPTY + s), 1);
+      mbar_init(bar(B_KOUT_READY + s), kComputeWarps);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -713,23 +728,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = setup_cta<D>(smem, warp, abort_flag);
   const WaitCtl wc{abort_flag, p.status, p.limit_ns, KID_BWD_DQ};
   const uint32_t sQ = sbase + L::kOffRes0, sDO = sbase + L::kOffRes1;
-  // global block g of this CTA uses slot g % 2 (K then V); after an item's
-  // last block the K part of its slot stages the item's dQ tile, which the
-  // producer stores with TMA before its next load into that slot
-  auto stage_addr = [&](int g) { return sbase + L::kOffStage + (g % kStages) * L::kStageBytes; };
+  // global block g of this CTA takes K slot g % 3 and V slot g % 2: K (read
+  // by S and, last, by dQ) gets one more block of prefetch than V (last read
+  // by dP). After an item's last block its K slot stages the item's dQ tile,
+  // which the producer stores with TMA before its next load into that slot.
+  auto k_addr = [&](int g) { return sbase + L::kOffKRing + (g % kKSlots) * L::kTileBytes; };
+  auto v_addr = [&](int g) { return sbase + L::kOffVRing + (g % kStages) * L::kTileBytes; };
 
   if (warp >= 8) {
     regs_decrease<kRegsControl>();
     if (warp == kLoadWarp) {
       if (lane == 0) {
-        int issued = 0, res_issued = 0;
-        int pend_q[kStages] = {-1, -1}, pend_bh[kStages] = {0, 0}, staged[kStages] = {0, 0};
+        int k_issued = 0, v_issued = 0, res_issued = 0;
+        int pend_q[kKSlots] = {-1, -1, -1}, pend_bh[kKSlots] = {0, 0, 0}, staged[kKSlots] = {0, 0, 0};
         auto flush = [&](int s) -> bool {
           if (pend_q[s] < 0) return true;
-          if (!wait_bounded(BAR(B_OUT_READY + s), staged[s] & 1, wc, 4)) return false;
+          if (!wait_bounded(BAR(B_KOUT_READY + s), staged[s] & 1, wc, 4)) return false;
           ++staged[s];
           for (int c = 0; c < L::kGroups; ++c)
-            tma_store_3d(&tmDQ, sbase + L::kOffStage + s * L::kStageBytes + c * L::kSubBytes, c * 64,
+            tma_store_3d(&tmDQ, sbase + L::kOffKRing + s * L::kTileBytes + c * L::kSubBytes, c * 64,
                          pend_q[s] * kTile, pend_bh[s]);
           bulk_commit_group();
           bulk_wait_group_read0();
@@ -748,30 +765,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++res_issued;
           for (int it = 0; it < n_blk; ++it, ++g) {
-            const int s = g % kStages;
-            if (!(ok = wait_bounded(BAR(B_ST_EMPTY + s), ((g / kStages) & 1) ^ 1, wc, 1))) break;
-            if (!(ok = flush(s))) break;
-            const uint32_t st = stage_addr(g);
-            mbar_arrive_expect_tx(BAR(B_ST_FULL + s), 2 * L::kTileBytes);
-            for (int c = 0; c < L::kGroups; ++c) {
-              tma_load_3d(st + c * L::kSubBytes, &tmK, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
-              tma_load_3d(st + L::kTileBytes + c * L::kSubBytes, &tmV, BAR(B_ST_FULL + s), c * 64, it * kTile, bh);
-            }
-            ++issued;
+            const int ks = g % kKSlots, vs = g % kStages;
+            if (!(ok = wait_bounded(BAR(B_K_EMPTY + ks), ((g / kKSlots) & 1) ^ 1, wc, 1))) break;
+            if (!(ok = flush(ks))) break;
+            mbar_arrive_expect_tx(BAR(B_K_FULL + ks), L::kTileBytes);
+            for (int c = 0; c < L::kGroups; ++c)
+              tma_load_3d(k_addr(g) + c * L::kSubBytes, &tmK, BAR(B_K_FULL + ks), c * 64, it * kTile, bh);
+            ++k_issued;
+            if (!(ok = wait_bounded(BAR(B_DO_EMPTY + vs), ((g / kStages) & 1) ^ 1, wc, 3))) break;
+            mbar_arrive_expect_tx(BAR(B_DO_FULL + vs), L::kTileBytes);
+            for (int c = 0; c < L::kGroups; ++c)
+              tma_load_3d(v_addr(g) + c * L::kSubBytes, &tmV, BAR(B_DO_FULL + vs), c * 64, it * kTile, bh);
+            ++v_issued;
             if (it == n_blk - 1) {
-              pend_q[s] = it_q;
-              pend_bh[s] = bh;
+              pend_q[ks] = it_q;
+              pend_bh[ks] = bh;
             }
           }
         }
-        if (ok) ok = flush(g % kStages);
-        if (ok) ok = flush((g + 1) % kStages);
+        // the outputs still staged, oldest first
+        for (int j = 0; ok && j < kKSlots; ++j) ok = flush((g + j) % kKSlots);
         bulk_wait_group0();
         if (*abort_flag) {
           if (res_issued) wait_bounded(BAR(B_RES_FULL), (res_issued - 1) & 1, wc, 2, true);
+          for (int s = 0; s < kKSlots; ++s) {
+            const int cnt = (k_issued - s + kKSlots - 1) / kKSlots;  // loads into K slot s
+            if (cnt > 0) wait_bounded(BAR(B_K_FULL + s), (cnt - 1) & 1, wc, 2, true);
+          }
           for (int s = 0; s < kStages; ++s) {
-            const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
-            if (cnt > 0) wait_bounded(BAR(B_ST_FULL + s), (cnt - 1) & 1, wc, 2, true);
+            const int cnt = (v_issued - s + kStages - 1) / kStages;  // loads into V slot s
+            if (cnt > 0) wait_bounded(BAR(B_DO_FULL + s), (cnt - 1) & 1, wc, 2, true);
           }
         }
       }
@@ -789,18 +812,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         int nround = 0, nit = 0, nbh = bh, nlvl = lvl, nn_blk = n_blk;
         auto issue_s = [&](int g, int r, int it_) -> bool {
           if (it_ == 0 && !wait_bounded(BAR(B_RES_FULL), r & 1, wc, 10)) return false;
-          if (!wait_bounded(BAR(B_ST_FULL + g % kStages), (g / kStages) & 1, wc, 11)) return false;
+          if (!wait_bounded(BAR(B_K_FULL + g % kKSlots), (g / kKSlots) & 1, wc, 11)) return false;
           tc_fence_after();
-          mma_rows_x_rows<D>(tmem + L::kColS, sQ, stage_addr(g));  // S = Q K^T
+          mma_rows_x_rows<D>(tmem + L::kColS, sQ, k_addr(g));  // S = Q K^T
           tc_commit(BAR(B_S_FULL));
           return true;
         };
-        auto issue_dp = [&](int g, int it_, int nb) {
-          mma_rows_x_rows<D>(tmem + L::kColDP, sDO, stage_addr(g) + L::kTileBytes);  // dP = dO V^T
+        auto issue_dp = [&](int g, int it_, int nb) -> bool {
+          if (!wait_bounded(BAR(B_DO_FULL + g % kStages), (g / kStages) & 1, wc, 16)) return false;
+          tc_fence_after();
+          mma_rows_x_rows<D>(tmem + L::kColDP, sDO, v_addr(g));  // dP = dO V^T
           tc_commit(BAR(B_DP_FULL));
+          tc_commit(BAR(B_DO_EMPTY + g % kStages));               // V read
           if (it_ == nb - 1) tc_commit(BAR(B_RES_EMPTY));  // the item's last reads of Q, dO
+          return true;
         };
-        if (ok && (ok = issue_s(0, 0, 0))) issue_dp(0, 0, n_blk);
+        if (ok && (ok = issue_s(0, 0, 0))) ok = issue_dp(0, 0, n_blk);
         for (int g = 0, it = 0; ok; ++g) {
           bool has_next = true;
           if (it + 1 < n_blk) {
@@ -820,8 +847,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && it == 0 && round > 0) ok = wait_bounded(BAR(B_ACC_EMPTY), (round - 1) & 1, wc, 17);
           if (!ok) break;
           tc_fence_after();
-          mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColDP, stage_addr(g), it > 0);  // dQ += dS K
-          tc_commit(BAR(B_ST_EMPTY + g % kStages));
+          mma_tmem_x_rows<D>(tmem + L::kColAcc0, tmem + L::kColDP, k_addr(g), it > 0);  // dQ += dS K
+          tc_commit(BAR(B_K_EMPTY + g % kKSlots));
           if (it == n_blk - 1) tc_commit(BAR(B_ACC_DONE));
           if (!has_next) break;
           if (!next_same_item) {
@@ -829,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) ok = issue_s(g + 1, nround, nit);
             if (!ok) break;
           }
-          issue_dp(g + 1, nit, nn_blk);
+          if (!(ok = issue_dp(g + 1, nit, nn_blk))) break;
           round = nround, it = nit, bh = nbh, lvl = nlvl, n_blk = nn_blk;
         }
         tc_commit(BAR(B_DRAIN));
@@ -910,14 +937,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int s = (g - 1) % kStages;
-      stage_acc_half<D>(tmem + lane_base + L::kColAcc0, smem + L::kOffStage + s * L::kStageBytes, r, half);
+      const int s = (g - 1) % kKSlots;
+      stage_acc_half<D>(tmem + lane_base + L::kColAcc0, smem + L::kOffKRing + s * L::kTileBytes, r, half);
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(BAR(B_ACC_EMPTY));
-        mbar_arrive(BAR(B_OUT_READY + s));
+        mbar_arrive(BAR(B_KOUT_READY + s));
       }
     }
   }

@@ -151,8 +151,10 @@ struct Plan {
   static constexpr int kOffBar = kStageEnd > kDqEnd ? kStageEnd : kDqEnd;
   static constexpr int kOffMisc = kOffBar + 8 * B_COUNT;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;
-  // TMEM columns
+  // TMEM columns; the dQ kernel keeps its resident Q and dO tiles (bf16, A
+  // operands) in the columns the second accumulator would use
   static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+  static constexpr uint32_t kColQT = 256 + D, kColDOT = 256 + D + D / 2;
 };
 
 // --------------------------------------------------------------------------
@@ -275,6 +277,31 @@ __device__ __forceinline__ void mma_rows_x_rows(uint32_t d_tmem, uint32_t r, uin
     const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
     mma_ss(d_tmem, sdesc_sw128(r + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), idesc,
            kk > 0 ? 1u : 0u);
+  }
+}
+
+// D[128 x 128] = A[128 x D] * B[128 x D]^T with A in TMEM (K-major: element
+// k of row m in lane m, column k/2) and B K-major in shared memory
+template <int D>
+__device__ __forceinline__ void mma_tmem_rows_x_rows(uint32_t d_tmem, uint32_t a_tmem, uint32_t b) {
+  using L = Plan<D>;
+  constexpr uint32_t idesc = idesc_bf16(kTile, kTile, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
+    mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// a resident 128 x D tile (K-major, 128-byte swizzle) into TMEM as an A
+// operand: D/16 copies of one K step each
+template <int D>
+__device__ __forceinline__ void copy_tile_to_tmem(uint32_t t_dst, uint32_t src) {
+  using L = Plan<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
+    tmem_cp_128x256b(t_dst + kk * 8, sdesc_sw128(src + off, 16, 1024));
   }
 }
 
@@ -802,29 +829,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       // per block g: S of the next block of the same item once S_g is in
       // registers; dQ_g after phase 2; then (for a new item, after dQ_g, since
       // it waits for the item's resident Q and dO) S of the next block, and
-      // dP of the next block. An item's resident Q, dO are released after its
-      // last S and dP; a new item's first dQ (which overwrites the
+      // dP of the next block. A new item's first dQ (which overwrites the
       // accumulator) waits until the compute warps have read the previous one.
       if (lane == 0) {
         int round = 0, bh, lvl;
         bool ok = bwd_item(p, 0, bh, lvl);
         int n_blk = ok ? blocks_of(tile_of(lvl)) : 0;
         int nround = 0, nit = 0, nbh = bh, nlvl = lvl, nn_blk = n_blk;
+        // an item's Q and dO go from shared memory into TMEM once (the A
+        // operands of its S and dP MMAs, which then read only K or V from
+        // shared memory); the shared copies are released right after, so the
+        // next item's Q and dO can load during this one
         auto issue_s = [&](int g, int r, int it_) -> bool {
-          if (it_ == 0 && !wait_bounded(BAR(B_RES_FULL), r & 1, wc, 10)) return false;
+          if (it_ == 0) {
+            if (!wait_bounded(BAR(B_RES_FULL), r & 1, wc, 10)) return false;
+            tc_fence_after();
+            copy_tile_to_tmem<D>(tmem + L::kColQT, sQ);
+            copy_tile_to_tmem<D>(tmem + L::kColDOT, sDO);
+            tc_commit(BAR(B_RES_EMPTY));
+          }
           if (!wait_bounded(BAR(B_K_FULL + g % kKSlots), (g / kKSlots) & 1, wc, 11)) return false;
           tc_fence_after();
-          mma_rows_x_rows<D>(tmem + L::kColS, sQ, k_addr(g));  // S = Q K^T
+          mma_tmem_rows_x_rows<D>(tmem + L::kColS, tmem + L::kColQT, k_addr(g));  // S = Q K^T
           tc_commit(BAR(B_S_FULL));
           return true;
         };
         auto issue_dp = [&](int g, int it_, int nb) -> bool {
+          (void)it_;
+          (void)nb;
           if (!wait_bounded(BAR(B_DO_FULL + g % kStages), (g / kStages) & 1, wc, 16)) return false;
           tc_fence_after();
-          mma_rows_x_rows<D>(tmem + L::kColDP, sDO, v_addr(g));  // dP = dO V^T
+          mma_tmem_rows_x_rows<D>(tmem + L::kColDP, tmem + L::kColDOT, v_addr(g));  // dP = dO V^T
           tc_commit(BAR(B_DP_FULL));
-          tc_commit(BAR(B_DO_EMPTY + g % kStages));               // V read
-          if (it_ == nb - 1) tc_commit(BAR(B_RES_EMPTY));  // the item's last reads of Q, dO
+          tc_commit(BAR(B_DO_EMPTY + g % kStages));  // V read
           return true;
         };
         if (ok && (ok = issue_s(0, 0, 0))) ok = issue_dp(0, 0, n_blk);

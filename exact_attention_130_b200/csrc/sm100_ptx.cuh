@@ -213,6 +213,14 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// shared memory -> tensor memory: 128 rows x 256 bits (16 bf16 per row, the
+// K slice of one MMA step of an operand described by s_desc) into TMEM lanes
+// 0-127, 8 columns from taddr. Runs in order with this thread's later
+// tcgen05.mma, so an MMA may read the copied columns as its A operand.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
+}
+
 // Instruction descriptor of tcgen05.mma .kind::f16 with bf16 A and B and an
 // fp32 accumulator. Bits: [4,6) D format (1 = f32), [7,10) A format
 // (1 = bf16), [10,13) B format (1 = bf16), 15 A major (1 = MN-major),

@@ -268,8 +268,20 @@ def fa_set_wait_limit(nanoseconds: int):
     load_library().fa_set_wait_limit(int(nanoseconds))
 
 
-def fa_debug_skip_load(enable: bool):
-    load_library().fa_debug_skip_load(int(bool(enable)))
+def fa_debug_skip_load(kernel=True):
+    """Test hook: the next call leaves one load out of the named kernel.
+
+    `kernel` is a kernel id or a name from KERNEL_NAMES ("fwd", "bwd_dkdv",
+    "bwd_dq", "decode_split"); True means the forward, False or 0 clears.
+    """
+    if isinstance(kernel, str):
+        ids = {name: kid for kid, name in KERNEL_NAMES.items()}
+        if kernel not in ids:
+            raise ValueError(f"unknown kernel name {kernel!r}")
+        kid = ids[kernel]
+    else:
+        kid = int(kernel)
+    load_library().fa_debug_skip_load(kid)
 
 
 def fa_profile_begin():

@@ -110,6 +110,7 @@ struct BwdParams {
   float scale, scale_log2;
   unsigned int* status;
   unsigned long long limit_ns;
+  int debug_skip;  // test hook: kernel id whose CTA 0 leaves out one load (0: none)
 };
 
 __device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
@@ -473,7 +474,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kLoadWarp) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
-        int q_issued = 0, do_issued = 0, res_issued = 0;
+        // loads started into each stage slot (the abort path waits for them)
+        int q_issued[kStages] = {0, 0}, do_issued[kStages] = {0, 0}, res_issued = 0;
+        bool skip_pending = p.debug_skip == KID_BWD && blockIdx.x == 0;
         // the item whose output is staged in slot s and not yet stored (-1:
         // none), with its coordinates, and how many stagings slot s has seen
         int pend_jt[kStages] = {-1, -1}, pend_bh[kStages] = {0, 0}, staged[kStages] = {0, 0};
@@ -514,13 +517,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < L::kGroups; ++c)
               tma_load_3d(sq + c * L::kSubBytes, &tmQ, BAR(B_ST_FULL + s), c * 64, q0, bh);
             tma_load_3d(qx_addr(g), &tmQX, BAR(B_ST_FULL + s), 0, q0, bh);
-            ++q_issued;
+            ++q_issued[s];
             if (!(ok = wait_bounded(BAR(B_DO_EMPTY + s), ph, wc, 3))) break;
-            mbar_arrive_expect_tx(BAR(B_DO_FULL + s), L::kTileBytes + L::kExtBytes);
-            for (int c = 0; c < L::kGroups; ++c)
-              tma_load_3d(do_addr(g) + c * L::kSubBytes, &tmDO, BAR(B_DO_FULL + s), c * 64, q0, bh);
-            tma_load_3d(dx_addr(g), &tmDX, BAR(B_DO_FULL + s), 0, q0, bh);
-            ++do_issued;
+            if (skip_pending) {
+              skip_pending = false;  // test hook: this dO block never arrives
+            } else {
+              mbar_arrive_expect_tx(BAR(B_DO_FULL + s), L::kTileBytes + L::kExtBytes);
+              for (int c = 0; c < L::kGroups; ++c)
+                tma_load_3d(do_addr(g) + c * L::kSubBytes, &tmDO, BAR(B_DO_FULL + s), c * 64, q0, bh);
+              tma_load_3d(dx_addr(g), &tmDX, BAR(B_DO_FULL + s), 0, q0, bh);
+              ++do_issued[s];
+            }
             if (it == n_blk - 1) {  // this slot will stage the item's output
               pend_jt[s] = jt;
               pend_bh[s] = bh;
@@ -533,11 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_wait_group0();
         if (*abort_flag) {
           if (res_issued) wait_bounded(BAR(B_RES_FULL), (res_issued - 1) & 1, wc, 2, true);
+          // the last load into a barrier completes its phase (loads - 1)
           for (int s = 0; s < kStages; ++s) {
-            const int cq = (q_issued - s + kStages - 1) / kStages;  // loads into slot s
-            if (cq > 0) wait_bounded(BAR(B_ST_FULL + s), (cq - 1) & 1, wc, 2, true);
-            const int cd = (do_issued - s + kStages - 1) / kStages;
-            if (cd > 0) wait_bounded(BAR(B_DO_FULL + s), (cd - 1) & 1, wc, 2, true);
+            if (q_issued[s]) wait_bounded(BAR(B_ST_FULL + s), (q_issued[s] - 1) & 1, wc, 2, true);
+            if (do_issued[s]) wait_bounded(BAR(B_DO_FULL + s), (do_issued[s] - 1) & 1, wc, 2, true);
           }
         }
       }
@@ -766,7 +772,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsControl>();
     if (warp == kLoadWarp) {
       if (lane == 0) {
-        int k_issued = 0, v_issued = 0, res_issued = 0;
+        // loads started into each ring slot (the abort path waits for them)
+        int k_issued[kKSlots] = {0, 0, 0}, v_issued[kStages] = {0, 0}, res_issued = 0;
+        bool skip_pending = p.debug_skip == KID_BWD_DQ && blockIdx.x == 0;
         int pend_q[kKSlots] = {-1, -1, -1}, pend_bh[kKSlots] = {0, 0, 0}, staged[kKSlots] = {0, 0, 0};
         auto flush = [&](int s) -> bool {
           if (pend_q[s] < 0) return true;
@@ -798,12 +806,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(BAR(B_K_FULL + ks), L::kTileBytes);
             for (int c = 0; c < L::kGroups; ++c)
               tma_load_3d(k_addr(g) + c * L::kSubBytes, &tmK, BAR(B_K_FULL + ks), c * 64, it * kTile, bh);
-            ++k_issued;
+            ++k_issued[ks];
             if (!(ok = wait_bounded(BAR(B_DO_EMPTY + vs), ((g / kStages) & 1) ^ 1, wc, 3))) break;
-            mbar_arrive_expect_tx(BAR(B_DO_FULL + vs), L::kTileBytes);
-            for (int c = 0; c < L::kGroups; ++c)
-              tma_load_3d(v_addr(g) + c * L::kSubBytes, &tmV, BAR(B_DO_FULL + vs), c * 64, it * kTile, bh);
-            ++v_issued;
+            if (skip_pending) {
+              skip_pending = false;  // test hook: this V block never arrives
+            } else {
+              mbar_arrive_expect_tx(BAR(B_DO_FULL + vs), L::kTileBytes);
+              for (int c = 0; c < L::kGroups; ++c)
+                tma_load_3d(v_addr(g) + c * L::kSubBytes, &tmV, BAR(B_DO_FULL + vs), c * 64, it * kTile, bh);
+              ++v_issued[vs];
+            }
             if (it == n_blk - 1) {
               pend_q[ks] = it_q;
               pend_bh[ks] = bh;
@@ -815,14 +827,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_wait_group0();
         if (*abort_flag) {
           if (res_issued) wait_bounded(BAR(B_RES_FULL), (res_issued - 1) & 1, wc, 2, true);
-          for (int s = 0; s < kKSlots; ++s) {
-            const int cnt = (k_issued - s + kKSlots - 1) / kKSlots;  // loads into K slot s
-            if (cnt > 0) wait_bounded(BAR(B_K_FULL + s), (cnt - 1) & 1, wc, 2, true);
-          }
-          for (int s = 0; s < kStages; ++s) {
-            const int cnt = (v_issued - s + kStages - 1) / kStages;  // loads into V slot s
-            if (cnt > 0) wait_bounded(BAR(B_DO_FULL + s), (cnt - 1) & 1, wc, 2, true);
-          }
+          // the last load into a barrier completes its phase (loads - 1)
+          for (int s = 0; s < kKSlots; ++s)
+            if (k_issued[s]) wait_bounded(BAR(B_K_FULL + s), (k_issued[s] - 1) & 1, wc, 2, true);
+          for (int s = 0; s < kStages; ++s)
+            if (v_issued[s]) wait_bounded(BAR(B_DO_FULL + s), (v_issued[s] - 1) & 1, wc, 2, true);
         }
       }
     } else if (warp == kMmaWarp) {
@@ -1086,6 +1095,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.scale_log2 = scale * kLog2e;
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
+  p.debug_skip = ctx.debug_skip_load;
 
   {
     const long long rows_per_warp = (32 / (d / 8)) * kPreSteps;

@@ -66,6 +66,7 @@ struct DecParams {
   float scale_log2;
   unsigned int* status;
   unsigned long long limit_ns;
+  int debug_skip;   // test hook: CTA (0,0,0) leaves out its first tile's loads
 };
 
 // kPer bf16 of one cached row (this lane's part) -> fp32
@@ -141,10 +142,16 @@ __global__ void __launch_bounds__(kThreads)
     if (lane == 0) {
       const uint16_t* kb = p.kc + (bh * p.Lmax + t0) * D;
       const uint16_t* vb = p.vc + (bh * p.Lmax + t0) * D;
-      int issued = 0;
+      int issued = 0, skip_stage = -1;
+      const bool skip = p.debug_skip && c == 0 && h == 0 && b == 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kStages;
         if (!wait_bounded(EMPTY(s), ((i / kStages) & 1) ^ 1, wc, 1)) break;
+        if (skip && i == 0) {  // test hook: this tile never arrives
+          skip_stage = s;
+          ++issued;
+          continue;
+        }
         const int rows = min(kStageTok, n_tok - i * kStageTok);
         const uint32_t bytes = uint32_t(rows) * D * 2;
         mbar_arrive_expect_tx(FULL(s), 2 * bytes);
@@ -154,8 +161,8 @@ __global__ void __launch_bounds__(kThreads)
       }
       if (*abort_flag)
         for (int s = 0; s < kStages; ++s) {
-          const int cnt = (issued - s + kStages - 1) / kStages;  // loads into stage s
-          if (cnt > 0) wait_bounded(FULL(s), (cnt - 1) & 1, wc, 2, true);
+          const int cnt = (issued - s + kStages - 1) / kStages - (s == skip_stage ? 1 : 0);
+          if (cnt > 0) wait_bounded(FULL(s), (cnt - 1) & 1, wc, 2, true);  // the last load into s
         }
     }
   } else {
@@ -370,6 +377,7 @@ fa_status launch_decode(const void* q, const void* kcache, const void* vcache, c
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
+  p.debug_skip = ctx.debug_skip_load == KID_DECODE;
   return d == 128 ? launch<128>(p, B, ctx) : launch<64>(p, B, ctx);
 }
 

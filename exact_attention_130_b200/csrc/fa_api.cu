@@ -260,7 +260,7 @@ void fa_set_wait_limit(unsigned long long ns) {
   g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs);
 }
 
-void fa_debug_skip_load(int enable) { g_debug_skip.store(enable ? 1 : 0); }
+void fa_debug_skip_load(int kernel_id) { g_debug_skip.store(kernel_id > 0 ? kernel_id : 0); }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int N, int d, float scale, int causal, cudaStream_t stream) {
@@ -310,6 +310,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!aligned16(workspace)) return invalid(FA_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
   LaunchCtx ctx;
   if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  ctx.debug_skip_load = g_debug_skip.exchange(0);
   return launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal != 0, workspace,
                     ctx);
 }
@@ -350,6 +351,7 @@ fa_status fa_decode_splitkv(const void* q, const void* kcache, const void* vcach
   if (!aligned16(workspace)) return invalid(FA_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
   LaunchCtx ctx;
   if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  ctx.debug_skip_load = g_debug_skip.exchange(0);
   return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Lmax, d, scale, chunks,
                        workspace, ctx);
 }

@@ -714,7 +714,7 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
-  p.debug_skip = ctx.debug_skip_load;
+  p.debug_skip = ctx.debug_skip_load == KID_FWD;
   if (causal) {
     if (d == 128)
       return snake ? launch<128, true, kModeSnake>(mq, mk, mv, mo, p, ctx) : launch<128, true>(mq, mk, mv, mo, p, ctx);

@@ -208,12 +208,17 @@ fa_status fa_device_status(cudaStream_t stream, unsigned int* detail);
 void fa_set_wait_limit(unsigned long long nanoseconds);
 
 /*
- * fa_debug_skip_load -- test hook: when nonzero, the next fa_fwd launch has
- * its first CTA skip one V-tile load, so that the consumer's wait runs out
- * and the kernel reports FA_ERR_TIMEOUT instead of producing output. Reset
- * to 0 by that launch.
+ * fa_debug_skip_load -- test hook for the bounded waits. kernel_id names the
+ * kernel (ids as in fa_profile_end) whose first CTA leaves out one load in
+ * the next call: 1 the forward (a V tile), 4 the backward dK/dV kernel (a dO
+ * block), 5 the backward dQ kernel (a V block), 6 the decode split kernel (its
+ * first tile). The wait for that load runs out, the kernel records
+ * FA_ERR_TIMEOUT in the device status word (fa_device_status) and returns
+ * without a fault; its outputs are then undefined. The next call of fa_fwd,
+ * fa_bwd or fa_decode_splitkv consumes the setting, whichever kernel it names;
+ * 0 or a negative value clears it.
  */
-void fa_debug_skip_load(int enable);
+void fa_debug_skip_load(int kernel_id);
 
 /*
  * Per-kernel timing, off by default. Between fa_profile_begin() and

@@ -76,10 +76,11 @@ enum : int {
   B_DRAIN = 6,
   B_K_FULL = 16,   // +stage
   B_V_FULL = 20,   // +stage
-  B_KV_EMPTY = 24, // +stage
+  B_V_EMPTY = 24,  // +stage: both tiles' P V of the stage's step are done
   B_STG_FREE = 28, // the O staging buffer may be rewritten (one arrival per epilogue)
   B_STG_READY = 29, // +t: the 4 warps of softmax group t have written the staging buffer
-  B_COUNT = 31
+  B_K_EMPTY = 31,  // +stage: the last Q K^T reading the stage's K tile is done
+  B_COUNT = 35
 };
 
 template <int D>
@@ -235,7 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(BAR(B_K_FULL + s), 1);
       mbar_init(BAR(B_V_FULL + s), 1);
-      mbar_init(BAR(B_KV_EMPTY + s), 1);
+      mbar_init(BAR(B_K_EMPTY + s), 1);
+      mbar_init(BAR(B_V_EMPTY + s), 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -260,9 +262,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kLoadWarp) {
       // ------------------------------------------------------------------ TMA producer
       if (lane == 0) {
+        // K and V tiles go through separate rings of kStages slots: a K slot
+        // is released by the last Q K^T that reads it, a step before the P V
+        // that releases the V slot of the same index, so K tiles load that
+        // much earlier. Loads started per slot, for the abort path:
+        int k_issued[L::kStages] = {}, v_issued[L::kStages] = {};
         int kv_issued = 0, unit_iter = 0;
         int q_issued0 = 0, q_issued1 = 0;
-        int v_skip_stage = -1;  // stage whose V load the test hook left out
         bool skip_pending = p.debug_skip && blockIdx.x == 0;
         bool ok = true;
         int item = MODE == kModeSnake ? 0 : int(blockIdx.x), half = 0, bh, pair, kv0, cnt, slot;
@@ -280,20 +286,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; ok && j < n1; ++j, ++kv_issued) {
             const int s = kv_issued % L::kStages;
             const uint32_t ph = (kv_issued / L::kStages) & 1;
-            ok = wait_bounded(BAR(B_KV_EMPTY + s), ph ^ 1, wc, 2);
+            ok = wait_bounded(BAR(B_K_EMPTY + s), ph ^ 1, wc, 2);
             if (!ok) break;
             mbar_arrive_expect_tx(BAR(B_K_FULL + s), L::kTileBytes);
             for (int c = 0; c < L::kSub; ++c)
               tma_load_3d(sbase + L::kOffK + s * L::kTileBytes + c * L::kSubBytes, &tmK,
                           BAR(B_K_FULL + s), c * 64, (kv0 + j) * kBN, bh);
+            ++k_issued[s];
+            ok = wait_bounded(BAR(B_V_EMPTY + s), ph ^ 1, wc, 4);
+            if (!ok) break;
             if (skip_pending) {
               skip_pending = false;  // test hook: this V tile never arrives
-              v_skip_stage = s;
             } else {
               mbar_arrive_expect_tx(BAR(B_V_FULL + s), L::kTileBytes);
               for (int c = 0; c < L::kSub; ++c)
                 tma_load_3d(sbase + L::kOffV + s * L::kTileBytes + c * L::kSubBytes, &tmV,
                             BAR(B_V_FULL + s), c * 64, (kv0 + j) * kBN, bh);
+              ++v_issued[s];
             }
           }
         }
@@ -303,10 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q_issued0) wait_bounded(BAR(B_Q_FULL + 0), (q_issued0 - 1) & 1, wc, 3, true);
           if (q_issued1) wait_bounded(BAR(B_Q_FULL + 1), (q_issued1 - 1) & 1, wc, 3, true);
           for (int s = 0; s < L::kStages; ++s) {
-            const int kc = (kv_issued - s + L::kStages - 1) / L::kStages;  // K loads into s
-            const int vc = kc - (s == v_skip_stage ? 1 : 0);
-            if (kc > 0) wait_bounded(BAR(B_K_FULL + s), (kc - 1) & 1, wc, 3, true);
-            if (vc > 0) wait_bounded(BAR(B_V_FULL + s), (vc - 1) & 1, wc, 3, true);
+            if (k_issued[s]) wait_bounded(BAR(B_K_FULL + s), (k_issued[s] - 1) & 1, wc, 3, true);
+            if (v_issued[s]) wait_bounded(BAR(B_V_FULL + s), (v_issued[s] - 1) & 1, wc, 3, true);
           }
         }
       }
@@ -358,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n0 == 1) tc_commit(BAR(B_Q_EMPTY + 0));
             issue_qk(1, s0);
             tc_commit(BAR(B_S_FULL + 1));
+            tc_commit(BAR(B_K_EMPTY + s0));  // tile 1 reads every K tile of the unit, last
             if (n1 == 1) tc_commit(BAR(B_Q_EMPTY + 1));
           }
           int k_ready = 0;
@@ -389,13 +397,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 issue_qk(t, s2);
                 tc_commit(BAR(B_S_FULL + t));
+                if (t == 1) tc_commit(BAR(B_K_EMPTY + s2));
                 if (j + 2 == nt) tc_commit(BAR(B_Q_EMPTY + t));
               } else {
                 tc_commit(BAR(B_O_FULL + t));
               }
             }
             if (!ok) break;
-            tc_commit(BAR(B_KV_EMPTY + s));
+            tc_commit(BAR(B_V_EMPTY + s));
           }
           kv_used += n1;
         }

@@ -72,7 +72,7 @@ _SIGNATURES = {
 }
 
 KERNEL_NAMES = {1: "fwd", 2: "fwd_f32", 3: "bwd_pre", 4: "bwd_dkdv", 5: "bwd_dq",
-                6: "decode_split", 7: "decode_merge", 8: "fwd_merge"}
+                6: "decode_split", 7: "decode_merge"}
 
 
 def load_library():

@@ -35,7 +35,6 @@ struct DeviceState {
   int num_sms = 0;
   int cc_major = 0, cc_minor = 0;
   unsigned int* status_word = nullptr;
-  cudaMemPool_t pool = nullptr;  // scratch of the forward's split work, created on first use
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -171,37 +170,6 @@ fa_status cuda_fail(cudaError_t e, const char* what) {
 
 fa_status current_launch_ctx(cudaStream_t stream, LaunchCtx* ctx) {
   return device_ctx(stream, ctx);
-}
-
-fa_status scratch_alloc(size_t bytes, const LaunchCtx& ctx, void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  DeviceState& ds = g_dev[dev];
-  {
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!ds.pool) {
-      cudaMemPoolProps props = {};
-      props.allocType = cudaMemAllocationTypePinned;
-      props.location.type = cudaMemLocationTypeDevice;
-      props.location.id = dev;
-      e = cudaMemPoolCreate(&ds.pool, &props);
-      if (e != cudaSuccess) {
-        ds.pool = nullptr;
-        return cuda_fail(e, "cudaMemPoolCreate(scratch)");
-      }
-      // keep freed blocks for the next call instead of returning them
-      unsigned long long keep = ~0ull;
-      cudaMemPoolSetAttribute(ds.pool, cudaMemPoolAttrReleaseThreshold, &keep);
-    }
-  }
-  e = cudaMallocFromPoolAsync(out, bytes, ds.pool, ctx.stream);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(scratch)");
-  return FA_OK;
-}
-
-void scratch_free(void* ptr, const LaunchCtx& ctx) {
-  if (ptr) cudaFreeAsync(ptr, ctx.stream);
 }
 
 fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t inner,

@@ -28,7 +28,6 @@ enum KernelId : unsigned int {
   KID_BWD_DQ = 5,   // dQ kernel
   KID_DECODE = 6,
   KID_DECODE_MERGE = 7,
-  KID_FWD_MERGE = 8,  // merge of the forward's split work units
 };
 
 // Brackets one kernel launch with CUDA events when profiling is on
@@ -53,13 +52,6 @@ fa_status current_launch_ctx(cudaStream_t stream, LaunchCtx* ctx);
 // Records a message for fa_last_error() on this thread.
 void set_last_error(const char* fmt, ...);
 fa_status cuda_fail(cudaError_t e, const char* what);
-
-// Stream-ordered device scratch from the library's own memory pool of the
-// current device (blocks are kept for reuse, never returned to the system):
-// allocation and release are ordered on ctx.stream, so concurrent calls on
-// different streams get different blocks, and both work under graph capture.
-fa_status scratch_alloc(size_t bytes, const LaunchCtx& ctx, void** out);
-void scratch_free(void* ptr, const LaunchCtx& ctx);
 
 // 3-D tiled tensor map over a [outer, rows, inner] bf16 or fp32 tensor
 // (inner contiguous), box = box_inner x box_rows x 1, zero fill out of bounds.

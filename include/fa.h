@@ -82,11 +82,8 @@ int fa_abi_version(void);
  * O~; O = diag(l)^-1 O~ at the end), "Online Softmax" (exp2 form with the
  * scores pre-scaled by log2 e), "Maskeleme ve Dropout" (tiles above the
  * diagonal skipped, the diagonal tile masked before the row maximum).
- * Without the mask, when the work units do not fill the last round of SMs,
- * the units of that round are split along the keys and their partial
- * results (O and LSE of each part) are merged by LSE, exactly as split-KV
- * decoding merges its chunks; the partials live in stream-ordered scratch
- * from the library's own memory pool (at most ~20 MB, reused across calls).
+ * Allocates nothing: O and LSE are written once each, straight from the
+ * kernel (one 128-row query tile per work unit).
  */
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o,
                  float* lse, int B, int H, int N, int d, float scale,
@@ -228,7 +225,7 @@ void fa_debug_skip_load(int kernel_id);
  * k in [0, capacity), the number of launches (launches[k]) and their summed
  * device time in milliseconds (total_ms[k]). Kernel ids: 1 forward (bf16),
  * 2 forward (fp32), 3 backward preprocess, 4 backward dK/dV, 5 backward
- * dQ, 6 decode split, 7 decode merge, 8 forward merge of split work units.
+ * dQ, 6 decode split, 7 decode merge (8 is not used).
  * Returns the number of ids (9), or -1 if a CUDA call failed. Not thread-safe against concurrent
  * begin/end pairs; launches from several threads are recorded.
  */

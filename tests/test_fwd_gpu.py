@@ -77,31 +77,29 @@ def test_fwd_long_causal_sampled_row_blocks():
     assert np.all(np.isfinite(o_np)) and np.all(np.isfinite(l_np))
 
 
-@pytest.mark.parametrize("shape", [(1, 25, 2048, 128), (1, 40, 2048, 64)],
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("shape", [(1, 25, 2048, 128), (1, 40, 2048, 64), (2, 3, 1500, 128)],
                          ids=lambda s: "x".join(map(str, s)))
-def test_fwd_split_last_round(shape):
-    """Without the mask, when the last round of work units (pairs of Q tiles)
-    fills at most half the SMs, those units are split along the keys and
-    merged by LSE. With H=25 (200 units on 148 SMs: one whole round, then 52
-    units in 2 parts) and H=40, d=64 (320 units: two whole rounds, then 24
-    units in 4 parts), every row of the heads whose units were split is
-    compared, plus the first row block of every head."""
+def test_fwd_partial_last_round(shape, causal):
+    """More work units (one per 128-row query tile and head) than SMs, with
+    the last round of the persistent CTAs partly filled: H=25 gives 400
+    units on 148 SMs, H=40 at d=64 gives 640, and B=2, H=3, N=1500 (a
+    ragged last tile) gives 72 units, fewer than the SMs. Every row of the
+    last heads (whose units fall in the last rounds) is compared, plus the
+    first and last row blocks of every other head."""
     B, H, N, d = shape
-    x = inputgen.make_small_inputs(77 + H, B, H, N, d)
-    o, lse = run_fwd(x, False)
+    x = inputgen.make_small_inputs(77 + H + (1000 if causal else 0), B, H, N, d)
+    o, lse = run_fwd(x, causal)
     o_np, l_np = o.float().cpu().numpy(), lse.cpu().numpy()
-    n_pairs = (N + 255) // 256
-    units = B * H * n_pairs
-    grid = min(units, torch.cuda.get_device_properties(0).multi_processor_count)
-    first_split_head = (units // grid) * grid // n_pairs
-    blocks = [(h, blk) for h in range(first_split_head, H) for blk in range(N // 128)]
-    blocks += [(h, 0) for h in range(first_split_head)]
-    for h, blk in blocks:
-        r0, r1 = blk * 128, (blk + 1) * 128
-        ro, rl = oracle.attention_fwd_rows(f64(x["q"][0, h]), f64(x["k"][0, h]), f64(x["v"][0, h]),
-                                           1 / math.sqrt(d), False, r0, r1)
-        assert np.max(np.abs(o_np[0, h, r0:r1] - ro)) <= TOL_O, (h, blk)
-        assert np.max(np.abs(l_np[0, h, r0:r1] - rl)) <= TOL_LSE, (h, blk)
+    nblk = (N + 127) // 128
+    blocks = [(b, h, blk) for b in range(B) for h in range(H)
+              for blk in (range(nblk) if (b == B - 1 and h >= H - 2) else (0, nblk - 1))]
+    for b, h, blk in blocks:
+        r0, r1 = blk * 128, min((blk + 1) * 128, N)
+        ro, rl = oracle.attention_fwd_rows(f64(x["q"][b, h]), f64(x["k"][b, h]), f64(x["v"][b, h]),
+                                           1 / math.sqrt(d), causal, r0, r1)
+        assert np.max(np.abs(o_np[b, h, r0:r1] - ro)) <= TOL_O, (b, h, blk)
+        assert np.max(np.abs(l_np[b, h, r0:r1] - rl)) <= TOL_LSE, (b, h, blk)
 
 
 @pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])

@@ -9,6 +9,7 @@ from .attention import (  # noqa: F401
     attention_fwd,
     attention_fwd_rows,
     decode,
+    decode_paged,
     decode_split,
     merge_partials,
     online_attention_fwd,

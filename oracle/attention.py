@@ -21,7 +21,9 @@ in float64 and follows the plain definition written out on the pages:
   "Geri Yayilim" (saved log-sum-exp L, P = exp(S - L), D = rowsum(dO*O),
   dS = P * (dP - D)),
   "Decode Asamasi: Flash-Decoding" (split the key/value axis into chunks,
-  each chunk gives (m, l, O~), merged by the rescale identity).
+  each chunk gives (m, l, O~), merged by the rescale identity),
+  "Duvarin Otesi" (the KV cache of decoding, and the inference-side methods
+  it names: paged KV caches and grouped / multi-query attention).
 
 Where those sections lost their display formulas in extraction, the reading
 taken is the standard identity the surrounding prose describes; the readings
@@ -48,6 +50,7 @@ __all__ = [
     "decode",
     "decode_split",
     "merge_partials",
+    "decode_paged",
 ]
 
 
@@ -281,4 +284,45 @@ def decode_split(q, kcache, vcache, seqlens, scale: float, num_chunks: int):
                 parts_l.append(l_row[0])
             o[b, h], lse[b, h] = merge_partials(np.array(parts_o),
                                                 np.array(parts_l))
+    return o, lse
+
+
+def decode_paged(q, kpages, vpages, block_table, seqlens, scale: float):
+    """Single-token attention over a paged KV cache with grouped query heads.
+
+    The KV cache of "Duvarin Otesi", stored in fixed-size pages and shared by
+    groups of query heads (the paged and grouped-query layouts that section
+    names), computed directly by gathering each sequence's keys and values.
+
+    q [B, Hq, d]. kpages, vpages [P, Hkv, page, d]: page p holds `page`
+    consecutive cache positions of every KV head. block_table [B, M] (ints):
+    cache position t of sequence b is row t % page of page
+    block_table[b, t // page]. Hq is a multiple of Hkv, and query head h
+    reads KV head h // (Hq // Hkv) (consecutive query heads share a KV head;
+    Hkv = 1 is multi-query attention). Keys 0 .. seqlens[b]-1 are visible. A
+    sequence with no visible key gets O = 0 and LSE = -inf (an empty sum).
+    Returns (O [B, Hq, dv], LSE [B, Hq]).
+    """
+    q = _as_f64(q)
+    bsz, hq, _ = q.shape
+    _, hkv, page, _ = kpages.shape
+    if hq % hkv:
+        raise ValueError("the number of query heads must be a multiple of the KV heads")
+    group = hq // hkv
+    table = np.asarray(block_table)
+    o = np.zeros((bsz, hq, vpages.shape[-1]))
+    lse = np.full((bsz, hq), -np.inf)
+    for b in range(bsz):
+        n = int(seqlens[b])
+        if n == 0:
+            continue
+        t = np.arange(n)
+        pg, row = table[b, t // page], t % page
+        for h in range(hq):
+            kv = h // group
+            kb = _as_f64(kpages[pg, kv, row])
+            vb = _as_f64(vpages[pg, kv, row])
+            p, l_row = softmax_rows(scores(q[b, h][None, :], kb, scale, False))
+            o[b, h] = (p @ vb)[0]
+            lse[b, h] = l_row[0]
     return o, lse

@@ -137,9 +137,44 @@ def _mut_decode_drop_last_key(q, kcache, vcache, seqlens, scale):
                            scale)
 
 
+def _mut_paged_head_modulo(q, kpages, vpages, block_table, seqlens, scale):
+    # planted: query head h reads KV head h % Hkv instead of h // (Hq / Hkv)
+    q = np.asarray(q, dtype=np.float64)
+    hkv = kpages.shape[1]
+    out_o = np.zeros((q.shape[0], q.shape[1], vpages.shape[-1]))
+    out_l = np.full(q.shape[:2], -np.inf)
+    for h in range(q.shape[1]):
+        kp = np.repeat(kpages[:, h % hkv:h % hkv + 1], 1, axis=1)
+        vp = np.repeat(vpages[:, h % hkv:h % hkv + 1], 1, axis=1)
+        o, l = _orig["decode_paged"](q[:, h:h + 1], kp, vp, block_table, seqlens, scale)
+        out_o[:, h], out_l[:, h] = o[:, 0], l[:, 0]
+    return out_o, out_l
+
+
+def _mut_paged_row_within_page(q, kpages, vpages, block_table, seqlens, scale):
+    # planted: the row inside a page taken as t // page instead of t % page
+    page = kpages.shape[2]
+    q = np.asarray(q, dtype=np.float64)
+    table = np.asarray(block_table)
+    o = np.zeros((q.shape[0], q.shape[1], vpages.shape[-1]))
+    lse = np.full(q.shape[:2], -np.inf)
+    g = q.shape[1] // kpages.shape[1]
+    for b in range(q.shape[0]):
+        n = int(seqlens[b])
+        if n == 0:
+            continue
+        t = np.arange(n)
+        pg, row = table[b, t // page], np.minimum(t // page, page - 1)
+        for h in range(q.shape[1]):
+            kb, vb = kpages[pg, h // g, row], vpages[pg, h // g, row]
+            p, l_row = A.softmax_rows(A.scores(q[b, h][None, :], kb, scale, False))
+            o[b, h], lse[b, h] = (p @ vb)[0], l_row[0]
+    return o, lse
+
+
 _orig = {name: getattr(A, name) for name in
          ("scores", "softmax_rows", "attention_fwd", "attention_bwd",
-          "online_attention_fwd", "merge_partials", "decode")}
+          "online_attention_fwd", "merge_partials", "decode", "decode_paged")}
 
 MUTANTS = {
     "scores_no_scale": {"scores": _mut_scores_no_scale},
@@ -155,6 +190,8 @@ MUTANTS = {
     "online_no_rescale": {"online_attention_fwd": _mut_online_no_rescale},
     "merge_unnormalised": {"merge_partials": _mut_merge_unnormalised},
     "decode_drops_last_key": {"decode": _mut_decode_drop_last_key},
+    "paged_head_modulo": {"decode_paged": _mut_paged_head_modulo},
+    "paged_row_within_page": {"decode_paged": _mut_paged_row_within_page},
 }
 
 

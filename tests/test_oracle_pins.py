@@ -16,6 +16,10 @@ Sources of the properties (page title, section):
   central finite differences; D = rowsum(dO * O) = rowsum(P * dP).
 * same page, "Decode Asamasi: Flash-Decoding": splitting the key/value axis
   into chunks and merging by log-sum-exp equals the unsplit result.
+* same page, "Duvarin Otesi": a paged, grouped-query KV cache is only a
+  different storage of the same keys and values: its decode equals the
+  decode of the contiguous cache with each KV head repeated for its query
+  heads, whatever the page size or page order.
 * "FlashAttention'i Anlamak Bolum 1", 0.2 Notasyon: the function itself,
   compared with an independent library implementation (PyTorch's
   scaled_dot_product_attention in float64, and its autograd).
@@ -260,6 +264,61 @@ def pin_against_library_sdpa():
         assert np.allclose(lse, torch.logsumexp(s, dim=-1).numpy(), atol=1e-12)
 
 
+def _paged_from_contiguous(rng, kc, vc, page, spare=3):
+    """Store contiguous caches [B, Hkv, L, d] in shuffled pages of `page`
+    rows (L a multiple of page), plus `spare` pages of noise that no block
+    table entry names. Returns kpages, vpages, block_table."""
+    B, hkv, L, d = kc.shape
+    per = L // page
+    total = B * per + spare
+    order = rng.permutation(total)
+    kp = rng.standard_normal((total, hkv, page, d)) * 100.0
+    vp = rng.standard_normal((total, hkv, page, d)) * 100.0
+    table = np.empty((B, per), dtype=np.int64)
+    for b in range(B):
+        for i in range(per):
+            pg = order[b * per + i]
+            table[b, i] = pg
+            kp[pg] = kc[b, :, i * page:(i + 1) * page]
+            vp[pg] = vc[b, :, i * page:(i + 1) * page]
+    return kp, vp, table
+
+
+def pin_paged_gqa_is_repeated_contiguous_decode():
+    rng = np.random.default_rng(RNG_SEED + 12)
+    B, hq, hkv, L, d = 3, 6, 2, 48, 8
+    q = _rand(rng, B, hq, d)
+    kc, vc = _rand(rng, B, hkv, L, d), _rand(rng, B, hkv, L, d)
+    lens = np.array([48, 1, 29])
+    # each KV head repeated for the hq / hkv consecutive query heads it serves
+    kr, vr = np.repeat(kc, hq // hkv, axis=1), np.repeat(vc, hq // hkv, axis=1)
+    o_ref, l_ref = oracle.decode(q, kr, vr, lens, 0.4)
+    for page in (1, 8, 16, 48):
+        kp, vp, table = _paged_from_contiguous(rng, kc, vc, page)
+        o, lse = oracle.decode_paged(q, kp, vp, table, lens, 0.4)
+        assert np.allclose(o, o_ref, atol=1e-13), page
+        assert np.allclose(lse, l_ref, atol=1e-13), page
+    # multi-query: one KV head for every query head
+    k1, v1 = kc[:, :1], vc[:, :1]
+    kp, vp, table = _paged_from_contiguous(rng, k1, v1, 16)
+    o, lse = oracle.decode_paged(q, kp, vp, table, lens, 0.4)
+    o1, l1 = oracle.decode(q, np.repeat(k1, hq, axis=1), np.repeat(v1, hq, axis=1), lens, 0.4)
+    assert np.allclose(o, o1, atol=1e-13) and np.allclose(lse, l1, atol=1e-13)
+
+
+def pin_paged_empty_and_one_key():
+    rng = np.random.default_rng(RNG_SEED + 13)
+    B, hq, hkv, L, d = 2, 2, 1, 16, 4
+    q = _rand(rng, B, hq, d)
+    kc, vc = _rand(rng, B, hkv, L, d), _rand(rng, B, hkv, L, d)
+    kp, vp, table = _paged_from_contiguous(rng, kc, vc, 8)
+    o, lse = oracle.decode_paged(q, kp, vp, table, np.array([0, 1]), 0.5)
+    assert np.all(o[0] == 0.0) and np.all(np.isneginf(lse[0]))
+    # one visible key: O is that key's value, LSE its score
+    assert np.allclose(o[1], vc[1, 0, 0][None, :], atol=1e-14)
+    assert np.allclose(lse[1], 0.5 * (q[1] @ kc[1, 0, 0]), atol=1e-14)
+
+
 PINS = [
     pin_rows_sum_to_one,
     pin_row_shift_invariance,
@@ -274,6 +333,8 @@ PINS = [
     pin_decode_is_last_causal_row,
     pin_rows_helper_matches_full,
     pin_against_library_sdpa,
+    pin_paged_gqa_is_repeated_contiguous_decode,
+    pin_paged_empty_and_one_key,
 ]
 
 

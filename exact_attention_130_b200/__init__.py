@@ -21,6 +21,7 @@ __all__ = [
     "FAError", "library_path", "load_library", "exported_symbols",
     "fa_fwd", "fa_fwd_f32", "fa_bwd", "fa_bwd_workspace_size",
     "fa_decode_splitkv", "fa_decode_workspace_size", "fa_decode_splitkv_static",
+    "fa_decode_paged",
     "fa_device_status",
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_abi_version",
     "fa_profile_begin", "fa_profile_end", "STATUS", "KERNEL_NAMES",
@@ -64,6 +65,8 @@ _SIGNATURES = {
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I,
                                _P, _S, _P]),
     "fa_decode_splitkv_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                             _P, _S, _P]),
     "fa_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "fa_set_wait_limit": (None, [ctypes.c_ulonglong]),
     "fa_debug_skip_load": (None, [_I]),
@@ -230,6 +233,36 @@ def fa_decode_splitkv(q, kcache, vcache, seqlens, scale: float | None = None,
                                  _ptr(o), _ptr(lse), B, H, Lmax, d, scale,
                                  num_splits, _ptr(workspace), workspace.numel(),
                                  _stream(stream)))
+    return o, lse
+
+
+def fa_decode_paged(q, kpages, vpages, block_table, seqlens, scale: float | None = None,
+                    num_splits: int = 0, o=None, lse=None, workspace=None, stream=None):
+    """Single-token attention over a paged KV cache with grouped query heads.
+
+    q [B, Hq, d]; kpages, vpages [num_pages, Hkv, page_size, d];
+    block_table int32 [B, max_pages]; seqlens int32 [B] (all on the device).
+    """
+    import torch
+    lib = load_library()
+    _need(q, torch.bfloat16, "q")
+    _need(kpages, torch.bfloat16, "kpages")
+    _need(vpages, torch.bfloat16, "vpages")
+    _need(block_table, torch.int32, "block_table")
+    _need(seqlens, torch.int32, "seqlens")
+    B, Hq, d = q.shape
+    num_pages, Hkv, page_size = kpages.shape[0], kpages.shape[1], kpages.shape[2]
+    max_pages = block_table.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = fa_decode_workspace_size(B, Hq, max_pages * page_size, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(lib.fa_decode_paged(_ptr(q), _ptr(kpages), _ptr(vpages), _ptr(block_table),
+                               _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, num_pages,
+                               page_size, max_pages, d, scale, num_splits, _ptr(workspace),
+                               workspace.numel(), _stream(stream)))
     return o, lse
 
 

@@ -25,6 +25,15 @@
 //    lanes together (5 shuffles for 4 rows instead of 4 per row), and the
 //    running maximum moves once per 4 rows;
 //  * positions at or past seqlens[b] are never read;
+//  * grouped query heads ("Duvarin Otesi": GQA / MQA): query head h reads
+//    KV head h / (Hq / Hkv); the CTAs of the query heads that share a KV
+//    head run side by side, so its chunk is read from HBM about once and
+//    from L2 by the others;
+//  * paged caches (the same section: PagedAttention): a separate
+//    instantiation whose producer finds each 64-row stage's page in the
+//    sequence's block table (chunks then start on 64-row boundaries); a
+//    page index outside the pool is never dereferenced but reported in the
+//    device status word;
 //  * all waits are bounded in time (see sm100_ptx.cuh).
 #include <mutex>
 
@@ -55,9 +64,13 @@ struct DecLayout {
 
 struct DecParams {
   const uint16_t* q;
-  const uint16_t* kc;
+  const uint16_t* kc;   // contiguous [B, Hkv, Lmax, D], or pages [num_pages, Hkv, page, D]
   const uint16_t* vc;
   const int* seqlens;
+  const int* table;     // paged: [B, max_pages] page of each page-sized run of positions
+  int group;            // query heads per KV head (Hq / Hkv)
+  int Hkv;
+  int page, max_pages, num_pages;  // paged layout
   float* part_o;    // [B, H, C, D]
   float* part_lse;  // [B, H, C], base 2
   uint16_t* o;
@@ -96,7 +109,7 @@ __device__ __forceinline__ void load_row_part(const uint8_t* row, int j, float (
 // owns 4 rows of every 64-row stage. A lane holds d/16 elements of q and of
 // its output accumulator, so one 16-byte shared load per lane reads a whole
 // row per half-warp.
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kThreads)
     decode_split_kernel(const DecParams p) {
   using L = DecLayout<D>;
@@ -112,10 +125,12 @@ __global__ void __launch_bounds__(kThreads)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t bh = size_t(b) * p.H + h;
   const size_t part = bh * p.C + c;
+  const int hkv = h / p.group;
 
   int Lb = p.seqlens[b];
   Lb = Lb < 0 ? 0 : (Lb > p.Lmax ? p.Lmax : Lb);
-  const int chunk = (Lb + p.C - 1) / p.C;
+  int chunk = (Lb + p.C - 1) / p.C;
+  if (PAGED) chunk = (chunk + kStageTok - 1) / kStageTok * kStageTok;  // stages start on 64-row boundaries
   const int t0 = c * chunk;
   const int t1 = min(t0 + chunk, Lb);
   if (t0 >= t1) {  // empty chunk: weight 0 in the merge
@@ -140,8 +155,9 @@ __global__ void __launch_bounds__(kThreads)
   if (warp == kConsumerWarps) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      const uint16_t* kb = p.kc + (bh * p.Lmax + t0) * D;
-      const uint16_t* vb = p.vc + (bh * p.Lmax + t0) * D;
+      const size_t bkv = size_t(b) * p.Hkv + hkv;
+      const uint16_t* kb = PAGED ? p.kc : p.kc + (bkv * p.Lmax + t0) * D;  // contiguous cache only
+      const uint16_t* vb = PAGED ? p.vc : p.vc + (bkv * p.Lmax + t0) * D;
       int issued = 0, skip_stage = -1;
       const bool skip = p.debug_skip && c == 0 && h == 0 && b == 0;
       for (int i = 0; i < n_tiles; ++i) {
@@ -153,10 +169,40 @@ __global__ void __launch_bounds__(kThreads)
           continue;
         }
         const int rows = min(kStageTok, n_tok - i * kStageTok);
-        const uint32_t bytes = uint32_t(rows) * D * 2;
-        mbar_arrive_expect_tx(FULL(s), 2 * bytes);
-        bulk_load(sbase + L::kOffK + s * L::kTileBytes, kb + size_t(i) * kStageTok * D, bytes, FULL(s));
-        bulk_load(sbase + L::kOffV + s * L::kTileBytes, vb + size_t(i) * kStageTok * D, bytes, FULL(s));
+        if (!PAGED) {
+          const uint32_t bytes = uint32_t(rows) * D * 2;
+          mbar_arrive_expect_tx(FULL(s), 2 * bytes);
+          bulk_load(sbase + L::kOffK + s * L::kTileBytes, kb + size_t(i) * kStageTok * D, bytes, FULL(s));
+          bulk_load(sbase + L::kOffV + s * L::kTileBytes, vb + size_t(i) * kStageTok * D, bytes, FULL(s));
+        } else {
+          // the stage's rows [t, t + rows) in runs that each lie in one page
+          // (one run when the page holds a multiple of 64 rows, 64 / page
+          // runs for pages of 16 or 32 rows); every page index is checked
+          // against the pool before its rows are read
+          const int t = t0 + i * kStageTok;
+          const int run = p.page < kStageTok ? p.page : kStageTok;
+          uint32_t total = 0;
+          for (int r0 = 0; r0 < rows; r0 += run) {
+            const int tp = t + r0;
+            const int pg = p.table[size_t(b) * p.max_pages + tp / p.page];
+            if (pg < 0 || pg >= p.num_pages) {
+              atomicCAS(p.status, 0u, (unsigned(KID_DECODE) << 16) | (9u << 8) | 2u);
+              continue;  // these rows stay unread (results undefined, error reported)
+            }
+            total += uint32_t(min(run, rows - r0)) * D * 2;
+          }
+          mbar_arrive_expect_tx(FULL(s), 2 * total);
+          for (int r0 = 0; r0 < rows; r0 += run) {
+            const int tp = t + r0;
+            const int pg = p.table[size_t(b) * p.max_pages + tp / p.page];
+            if (pg < 0 || pg >= p.num_pages) continue;
+            const uint32_t bytes = uint32_t(min(run, rows - r0)) * D * 2;
+            const size_t src = ((size_t(pg) * p.Hkv + hkv) * p.page + tp % p.page) * D;
+            const uint32_t dst = uint32_t(r0) * D * 2;
+            bulk_load(sbase + L::kOffK + s * L::kTileBytes + dst, p.kc + src, bytes, FULL(s));
+            bulk_load(sbase + L::kOffV + s * L::kTileBytes + dst, p.vc + src, bytes, FULL(s));
+          }
+        }
         ++issued;
       }
       if (*abort_flag)
@@ -307,16 +353,16 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecParams p) {
   if (i == 0) p.lse[bh] = (mx + lg2_approx(wsum)) * kLn2;
 }
 
-template <int D>
+template <int D, bool PAGED>
 fa_status launch(const DecParams& p, int B, const LaunchCtx& ctx) {
   const int smem = DecLayout<D>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, PAGED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   dim3 g1(p.C, p.H, B);
   {
     ProfileScope prof(KID_DECODE, ctx.stream);
-    decode_split_kernel<D><<<g1, kThreads, smem, ctx.stream>>>(p);
+    decode_split_kernel<D, PAGED><<<g1, kThreads, smem, ctx.stream>>>(p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode split kernel launch");
@@ -366,6 +412,10 @@ fa_status launch_decode(const void* q, const void* kcache, const void* vcache, c
   p.kc = static_cast<const uint16_t*>(kcache);
   p.vc = static_cast<const uint16_t*>(vcache);
   p.seqlens = seqlens;
+  p.table = nullptr;
+  p.group = 1;
+  p.Hkv = H;
+  p.page = p.max_pages = p.num_pages = 0;
   const size_t parts = size_t(B) * H * chunks;
   p.part_o = static_cast<float*>(workspace);
   p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(parts * d * 4));
@@ -378,7 +428,42 @@ fa_status launch_decode(const void* q, const void* kcache, const void* vcache, c
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load == KID_DECODE;
-  return d == 128 ? launch<128>(p, B, ctx) : launch<64>(p, B, ctx);
+  return d == 128 ? launch<128, false>(p, B, ctx) : launch<64, false>(p, B, ctx);
+}
+
+fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpages,
+                              const int* block_table, const int* seqlens, void* o, float* lse,
+                              int B, int Hq, int Hkv, int num_pages, int page_size, int max_pages,
+                              int d, float scale, int chunks, void* workspace,
+                              const LaunchCtx& ctx) {
+  if (Hq > 65535 || B > 65535) {
+    set_last_error("fa_decode_paged: B and Hq must each be <= 65535");
+    return FA_ERR_UNSUPPORTED;
+  }
+  DecParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.kc = static_cast<const uint16_t*>(kpages);
+  p.vc = static_cast<const uint16_t*>(vpages);
+  p.seqlens = seqlens;
+  p.table = block_table;
+  p.group = Hq / Hkv;
+  p.Hkv = Hkv;
+  p.page = page_size;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  const size_t parts = size_t(B) * Hq * chunks;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(parts * d * 4));
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.H = Hq;
+  p.Lmax = max_pages * page_size;
+  p.C = chunks;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = ctx.status_word;
+  p.limit_ns = ctx.wait_limit_ns;
+  p.debug_skip = ctx.debug_skip_load == KID_DECODE;
+  return d == 128 ? launch<128, true>(p, B, ctx) : launch<64, true>(p, B, ctx);
 }
 
 }  // namespace fa

@@ -222,7 +222,7 @@ const char* fa_status_string(fa_status s) {
 
 const char* fa_last_error(void) { return t_last_error; }
 
-int fa_abi_version(void) { return 100; }
+int fa_abi_version(void) { return 101; }
 
 void fa_set_wait_limit(unsigned long long ns) {
   g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs);
@@ -324,6 +324,47 @@ fa_status fa_decode_splitkv(const void* q, const void* kcache, const void* vcach
                        workspace, ctx);
 }
 
+fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
+                          const int* block_table, const int* seqlens, void* o, float* lse,
+                          int B, int Hq, int Hkv, int num_pages, int page_size, int max_pages,
+                          int d, float scale, int num_splits, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, kpages, vpages, o, lse}, "fa_decode_paged(q,kpages,vpages,o,lse)")) !=
+      FA_OK)
+    return st;
+  if (seqlens == nullptr || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return invalid(FA_ERR_INVALID_ARG, "seqlens must be a non-null, 4-byte aligned int32 array");
+  if (block_table == nullptr || (reinterpret_cast<uintptr_t>(block_table) & 3u))
+    return invalid(FA_ERR_INVALID_ARG, "block_table must be a non-null, 4-byte aligned int32 array");
+  if (B < 1 || Hq < 1 || Hkv < 1 || num_pages < 1 || max_pages < 1)
+    return invalid(FA_ERR_INVALID_ARG, "B, Hq, Hkv, num_pages, max_pages must be >= 1");
+  if (Hq % Hkv != 0)
+    return invalid(FA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (!(page_size == 16 || page_size == 32 || (page_size >= 64 && page_size % 64 == 0)))
+    return invalid(FA_ERR_UNSUPPORTED, "page_size %d (need 16, 32 or a multiple of 64)", page_size);
+  if ((long long)max_pages * page_size > 0x7fffffffLL ||
+      (long long)num_pages * Hkv * page_size > 0x7fffffffLL ||
+      (long long)B * max_pages > 0x7fffffffLL || (long long)B * Hq > 0x7fffffffLL)
+    return invalid(FA_ERR_INVALID_ARG, "sizes exceed 2^31-1");
+  if (d != 64 && d != 128) return invalid(FA_ERR_UNSUPPORTED, "head dim %d (need 64 or 128)", d);
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (num_splits < 0 || num_splits > 1024)
+    return invalid(FA_ERR_INVALID_ARG, "num_splits must be in [0, 1024] (got %d)", num_splits);
+  const int Lmax = max_pages * page_size;
+  const int chunks = decode_num_chunks(B, Hq, Lmax, num_splits, 0);
+  const size_t need = decode_workspace_bytes(B, Hq, d, chunks);
+  if (workspace == nullptr || workspace_bytes < need)
+    return invalid(FA_ERR_WORKSPACE, "fa_decode_paged needs %zu bytes of workspace (got %zu)",
+                   need, workspace ? workspace_bytes : size_t(0));
+  if (!aligned16(workspace)) return invalid(FA_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  ctx.debug_skip_load = g_debug_skip.exchange(0);
+  return launch_decode_paged(q, kpages, vpages, block_table, seqlens, o, lse, B, Hq, Hkv,
+                             num_pages, page_size, max_pages, d, scale, chunks, workspace, ctx);
+}
+
 void fa_profile_begin(void) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   for (auto& r : g_prof) {
@@ -373,6 +414,11 @@ fa_status fa_device_status(cudaStream_t stream, unsigned int* detail) {
     if (e != cudaSuccess) return cuda_fail(e, "clear status word");
   }
   if (detail) *detail = word;
+  if (word && (word & 0xffu) == 2u) {
+    set_last_error("a kernel found an invalid value in device memory: kernel %u, site %u",
+                   word >> 16, (word >> 8) & 0xff);
+    return FA_ERR_INVALID_ARG;
+  }
   if (word) {
     set_last_error("a device-side wait gave up: kernel %u, site %u", word >> 16, (word >> 8) & 0xff);
     return FA_ERR_TIMEOUT;

@@ -73,6 +73,11 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
 size_t bwd_workspace_bytes(int B, int H, int N, int d);
 int decode_num_chunks(int B, int H, int Lmax, int num_splits, int num_sms);
 size_t decode_workspace_bytes(int B, int H, int d, int chunks);
+fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpages,
+                              const int* block_table, const int* seqlens, void* o, float* lse,
+                              int B, int Hq, int Hkv, int num_pages, int page_size, int max_pages,
+                              int d, float scale, int chunks, void* workspace,
+                              const LaunchCtx& ctx);
 fa_status launch_decode(const void* q, const void* kcache, const void* vcache,
                         const int* seqlens, void* o, float* lse, int B, int H, int Lmax, int d,
                         float scale, int chunks, void* workspace, const LaunchCtx& ctx);

@@ -162,6 +162,44 @@ fa_status fa_decode_splitkv(const void* q, const void* kcache,
                             size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * fa_decode_paged -- the split-KV decode of fa_decode_splitkv over a paged
+ * KV cache, with grouped query heads ("Bellek Duvarinin Fizigi", section
+ * "Duvarin Otesi": the KV cache, and the paged / grouped-query layouts it
+ * names as the inference-side IO methods; "Decode Asamasi: Flash-Decoding"
+ * for the split and the log-sum-exp merge).
+ *   q              : bf16 [B, Hq, d]                       (input, device)
+ *   kpages, vpages : bf16 [num_pages, Hkv, page_size, d]   (input, device);
+ *                    page p holds page_size consecutive cache positions of
+ *                    every KV head
+ *   block_table    : int32 [B, max_pages] (device): cache position t of
+ *                    sequence b is row t % page_size of page
+ *                    block_table[b * max_pages + t / page_size]; entries past
+ *                    a sequence's last page are never read
+ *   seqlens        : int32 [B] (device); keys 0 .. seqlens[b]-1 are visible
+ *                    (clamped to [0, max_pages * page_size]; a sequence with
+ *                    no key gets O = 0, LSE = -inf)
+ *   o              : bf16 [B, Hq, d];  lse : fp32 [B, Hq]  (outputs, device)
+ *   Hq, Hkv        : Hq a multiple of Hkv; query head h reads KV head
+ *                    h / (Hq / Hkv) (Hkv = 1: multi-query; Hkv = Hq: one KV
+ *                    head per query head)
+ *   page_size      : 16, 32 or a multiple of 64
+ *   num_splits     : chunks per sequence, 0 = automatic, <= 1024
+ *   workspace      : >= fa_decode_workspace_size(B, Hq, max_pages *
+ *                    page_size, d, num_splits) bytes (caller-owned, device)
+ * Validation errors return before any launch. A block-table entry outside
+ * [0, num_pages) is never dereferenced: the kernel leaves those rows unread
+ * and records the fault in the device status word, and the next
+ * fa_device_status returns FA_ERR_INVALID_ARG (the outputs of that call are
+ * undefined). d : 128 or 64. Deterministic, like fa_decode_splitkv.
+ */
+fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
+                          const int* block_table, const int* seqlens, void* o,
+                          float* lse, int B, int Hq, int Hkv, int num_pages,
+                          int page_size, int max_pages, int d, float scale,
+                          int num_splits, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * fa_decode_splitkv_static -- fa_decode_splitkv for callers that cannot
  * allocate device memory when they decode (inside a stream capture, under an
  * allocator that forbids cudaMalloc on the hot path, or with no memory pool
@@ -191,9 +229,12 @@ fa_status fa_decode_splitkv_static(const void* q, const void* kcache,
 /*
  * fa_device_status -- synchronises `stream`, reads and clears the current
  * device's status word. Returns FA_ERR_TIMEOUT if any kernel of this
- * library gave up a wait since the last check, FA_ERR_CUDA if the
+ * library gave up a wait since the last check, FA_ERR_INVALID_ARG if a
+ * kernel found an invalid value in device memory (a block-table entry of
+ * fa_decode_paged outside the page pool), FA_ERR_CUDA if the
  * synchronisation itself failed, else FA_OK. *detail (may be NULL) gets the
- * raw word: kernel id << 16 | wait site << 8 | 1.
+ * raw word of the first such event: kernel id << 16 | site << 8 | kind,
+ * kind 1 = a wait gave up, 2 = an invalid value.
  */
 fa_status fa_device_status(cudaStream_t stream, unsigned int* detail);
 

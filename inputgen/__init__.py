@@ -20,6 +20,14 @@ Recipe
   head as [seqlen[b], d] blocks, so sequences can be drawn in parallel; cache
   positions at or past ``seqlen[b]`` are filled with NaN so that a kernel
   that reads past the logical end poisons its own result;
+* the paged, grouped-query decode inputs (``make_paged_decode_inputs``)
+  draw q from ``default_rng(seed)`` after the lengths (as above), the K (V)
+  rows of sequence b and KV head h from
+  ``default_rng(SeedSequence([seed, 1 (2 for V), b]))`` as [seqlen[b], d]
+  blocks head by head, and scatter them into pages whose order is a seeded
+  permutation (``default_rng(seed + 7)``); rows past a sequence's end, and
+  pages no sequence uses, hold NaN, and block-table entries past a
+  sequence's last page hold -1, so a kernel that reads any of them is caught;
 * bf16 rounding is round-to-nearest-even on the fp32 bit pattern.
 """
 from __future__ import annotations
@@ -38,6 +46,7 @@ __all__ = [
     "standard_normal_bf16",
     "make_attention_inputs",
     "make_decode_inputs",
+    "make_paged_decode_inputs",
     "make_small_inputs",
     "sample_row_blocks",
 ]
@@ -158,6 +167,41 @@ def make_decode_inputs(w: Workload, seqlens=None):
     with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
         list(ex.map(fill, jobs))
     return {"q": q, "kcache": kc, "vcache": vc, "seqlens": lens}
+
+
+def make_paged_decode_inputs(seed: int, B: int, Hq: int, Hkv: int, d: int, page: int,
+                             seqlen_range=None, seqlens=None, spare_pages: int = 3,
+                             max_pages: int | None = None):
+    """q [B,Hq,d]; K/V pages [num_pages, Hkv, page, d] (bf16 bits); block table
+    int32 [B, max_pages]; seqlens int32 [B]. See the recipe above."""
+    rng = np.random.default_rng(seed)
+    if seqlens is None:
+        lo, hi = seqlen_range
+        lens = rng.integers(lo, hi + 1, size=B).astype(np.int32)
+    else:
+        lens = np.asarray(seqlens, dtype=np.int32)
+    q = standard_normal_bf16(rng, (B, Hq, d))
+    used = [(int(n) + page - 1) // page for n in lens]
+    mp = max(max(used), 1) if max_pages is None else max_pages
+    num_pages = sum(used) + spare_pages
+    order = np.random.default_rng(seed + 7).permutation(num_pages)
+    table = np.full((B, mp), -1, dtype=np.int32)
+    kp = np.full((num_pages, Hkv, page, d), 0x7FC0, dtype=np.uint16)
+    vp = np.full((num_pages, Hkv, page, d), 0x7FC0, dtype=np.uint16)
+    nxt = 0
+    for b in range(B):
+        n = int(lens[b])
+        pages_b = order[nxt:nxt + used[b]]
+        nxt += used[b]
+        table[b, :used[b]] = pages_b
+        for which, dst in ((1, kp), (2, vp)):
+            g = np.random.default_rng(np.random.SeedSequence([seed, which, b]))
+            for h in range(Hkv):
+                rows = standard_normal_bf16(g, (n, d))
+                for i, pg in enumerate(pages_b):
+                    r0, r1 = i * page, min((i + 1) * page, n)
+                    dst[pg, h, :r1 - r0] = rows[r0:r1]
+    return {"q": q, "kpages": kp, "vpages": vp, "block_table": table, "seqlens": lens}
 
 
 def make_small_inputs(seed: int, B: int, H: int, N: int, d: int,

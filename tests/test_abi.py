@@ -12,7 +12,7 @@ EXPECTED = {
     "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd",
     "fa_decode_workspace_size", "fa_decode_splitkv", "fa_device_status",
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_profile_begin",
-    "fa_profile_end", "fa_decode_splitkv_static",
+    "fa_profile_end", "fa_decode_splitkv_static", "fa_decode_paged",
 }
 
 
@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     for code, name in fa.STATUS.items():
         assert lib.fa_status_string(code).decode() == name
-    assert lib.fa_abi_version() == 100
+    assert lib.fa_abi_version() == 101
 
 
 def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=8, d=64,
@@ -75,6 +75,26 @@ def test_bwd_and_decode_argument_errors(lib):
     st = lib.fa_decode_splitkv(P(16), P(16), P(16), P(16), P(16), P(16), 1, 1,
                                8, 64, 0.125, 2000, P(16), 1 << 20, None)
     assert st == 1
+
+
+def _paged(lib, table=16, B=1, Hq=4, Hkv=2, num_pages=4, page=64, max_pages=2, d=64,
+           scale=0.125, ws_bytes=1 << 20):
+    P = ctypes.c_void_p
+    return lib.fa_decode_paged(P(16), P(16), P(16), P(table), P(16), P(16), P(16), B, Hq, Hkv,
+                               num_pages, page, max_pages, d, scale, 0, P(16), ws_bytes, None)
+
+
+def test_paged_decode_argument_errors(lib):
+    assert _paged(lib, table=0) == 1              # no block table
+    assert _paged(lib, table=18) == 1             # block table not 4-byte aligned
+    assert _paged(lib, Hq=6, Hkv=4) == 1          # Hq not a multiple of Hkv
+    assert b"multiple" in lib.fa_last_error()
+    assert _paged(lib, page=48) == 2              # unsupported page size
+    assert _paged(lib, page=8) == 2
+    assert _paged(lib, num_pages=0) == 1
+    assert _paged(lib, d=96) == 2
+    assert _paged(lib, ws_bytes=8) == 4           # workspace too small
+    assert _paged(lib, max_pages=1 << 20, page=4096) == 1   # positions overflow
 
 
 def test_workspace_sizes(lib):

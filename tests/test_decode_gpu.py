@@ -104,3 +104,84 @@ def test_decode_matches_last_causal_row_of_forward():
     torch.cuda.synchronize()
     assert float((o_d.float() - o_f[:, :, -1].float()).abs().max()) <= 2e-2
     assert float((l_d - l_f[:, :, -1]).abs().max()) <= 2e-3
+
+
+# ---------------------------------------------------------------------------
+# paged KV cache with grouped query heads (fa_decode_paged)
+# ---------------------------------------------------------------------------
+
+def run_paged(x, num_splits=0, scale=None):
+    B, Hq, d = x["q"].shape
+    q = bf16_device(x["q"])
+    kp, vp = bf16_device(x["kpages"]), bf16_device(x["vpages"])
+    table = torch.from_numpy(x["block_table"]).cuda()
+    lens = torch.from_numpy(x["seqlens"].astype(np.int32)).cuda()
+    o = Guarded((B, Hq, d), torch.bfloat16)
+    lse = Guarded((B, Hq), torch.float32)
+    fa.fa_decode_paged(q, kp, vp, table, lens, scale=scale, num_splits=num_splits,
+                       o=o.t, lse=lse.t)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status()[0] == 0
+    assert o.guards_intact() and lse.guards_intact()
+    return o.t, lse.t
+
+
+def _check_paged(x, o, lse, scale):
+    ro, rl = oracle.decode_paged(f64(x["q"]), f64(x["kpages"]), f64(x["vpages"]),
+                                 x["block_table"], x["seqlens"], scale)
+    o_np, l_np = o.float().cpu().numpy(), lse.cpu().numpy()
+    empty = x["seqlens"] == 0
+    # a sequence with no key: O = 0 and LSE = -inf exactly
+    assert np.all(o_np[empty] == 0.0) and np.all(np.isneginf(l_np[empty]))
+    assert np.max(np.abs(o_np[~empty] - ro[~empty]), initial=0.0) <= TOL_O
+    assert np.max(np.abs(l_np[~empty] - rl[~empty]), initial=0.0) <= TOL_LSE
+
+
+@pytest.mark.parametrize("heads", [(4, 4), (8, 2), (6, 1)], ids=["mha", "gqa4", "mqa"])
+@pytest.mark.parametrize("page", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("d", [64, 128])
+def test_paged_decode_small(d, page, heads):
+    hq, hkv = heads
+    x = inputgen.make_paged_decode_inputs(500 + page + d + hq, 4, hq, hkv, d, page,
+                                          seqlens=[0, 1, 300, 517])
+    o, lse = run_paged(x)
+    _check_paged(x, o, lse, 1 / np.sqrt(d))
+
+
+@pytest.mark.parametrize("num_splits", [1, 2, 7, 64])
+def test_paged_decode_split_counts(num_splits):
+    x = inputgen.make_paged_decode_inputs(611, 3, 8, 2, 128, 64, seqlens=[2000, 63, 1025],
+                                          max_pages=40)
+    o, lse = run_paged(x, num_splits)
+    _check_paged(x, o, lse, 1 / np.sqrt(128))
+
+
+def test_paged_decode_workload():
+    """B=8, Hq=32, Hkv=8, d=128, pages of 64 rows, cache lengths drawn from
+    [16384, 32768] (the split-KV decode workload with grouped query heads and a
+    paged cache), every head compared."""
+    x = inputgen.make_paged_decode_inputs(20264, 8, 32, 8, 128, 64,
+                                          seqlen_range=(16384, 32768))
+    o, lse = run_paged(x)
+    _check_paged(x, o, lse, 1 / np.sqrt(128))
+
+
+def test_paged_decode_bad_page_is_reported_not_read():
+    """A block-table entry outside the page pool is never dereferenced: the
+    call reports FA_ERR_INVALID_ARG through fa_device_status, and the next
+    call with a correct table gives correct results."""
+    x = inputgen.make_paged_decode_inputs(612, 2, 4, 2, 128, 64, seqlens=[200, 130])
+    q = bf16_device(x["q"])
+    kp, vp = bf16_device(x["kpages"]), bf16_device(x["vpages"])
+    lens = torch.from_numpy(x["seqlens"]).cuda()
+    bad = x["block_table"].copy()
+    bad[1, 1] = kp.shape[0] + 5      # past the pool
+    bad[0, 2] = -3                   # negative
+    assert fa.fa_device_status()[0] == 0
+    fa.fa_decode_paged(q, kp, vp, torch.from_numpy(bad).cuda(), lens)
+    st, word = fa.fa_device_status()
+    assert st == 1, (st, word)                      # FA_ERR_INVALID_ARG
+    assert (word >> 16) == 6 and (word & 0xff) == 2, hex(word)
+    assert fa.fa_device_status()[0] == 0
+    o, lse = run_paged(x)
+    _check_paged(x, o, lse, 1 / np.sqrt(128))

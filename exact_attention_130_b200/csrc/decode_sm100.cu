@@ -26,9 +26,11 @@
 //    running maximum moves once per 4 rows;
 //  * positions at or past seqlens[b] are never read;
 //  * grouped query heads ("Duvarin Otesi": GQA / MQA): query head h reads
-//    KV head h / (Hq / Hkv); the CTAs of the query heads that share a KV
-//    head run side by side, so its chunk is read from HBM about once and
-//    from L2 by the others;
+//    KV head h / (Hq / Hkv); a CTA serves up to 4 query heads of one KV head
+//    from a single shared-memory copy of each K/V row (each lane keeps q, the
+//    running statistics and the output slice of every head), and the CTAs
+//    of the remaining heads of the group run side by side, so a chunk is
+//    read from HBM once and through L2 Hq / Hkv / 4 times at most;
 //  * paged caches (the same section: PagedAttention): a separate
 //    instantiation whose producer finds each 64-row stage's page in the
 //    sequence's block table (chunks then start on 64-row boundaries); a
@@ -58,8 +60,11 @@ struct DecLayout {
   static constexpr int kOffV = kStages * kTileBytes;
   static constexpr int kOffBar = 2 * kStages * kTileBytes;       // full[s], empty[s]
   static constexpr int kOffMisc = kOffBar + 8 * 2 * kStages;     // abort flag
-  static constexpr int kOffMerge = kOffMisc + 16;                // per half-warp m, l, acc[D]
-  static constexpr int kSmemBytes = kOffMerge + 2 * kConsumerWarps * (D + 2) * 4 + 128;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 128;
+  // after the stream: per half-warp and query head m, l, acc[D], over the
+  // stage buffers (no copy is in flight by then)
+  static constexpr int kOffMerge = 0;
+  static_assert(2 * kConsumerWarps * 4 * (D + 2) * 4 <= 2 * kStages * kTileBytes, "merge area");
 };
 
 struct DecParams {
@@ -109,8 +114,8 @@ __device__ __forceinline__ void load_row_part(const uint8_t* row, int j, float (
 // owns 4 rows of every 64-row stage. A lane holds d/16 elements of q and of
 // its output accumulator, so one 16-byte shared load per lane reads a whole
 // row per half-warp.
-template <int D, bool PAGED>
-__global__ void __launch_bounds__(kThreads)
+template <int D, bool PAGED, int GH>
+__global__ void __launch_bounds__(kThreads, 2)
     decode_split_kernel(const DecParams p) {
   using L = DecLayout<D>;
   constexpr int kPer = D / 16;  // elements per lane (16 lanes per row)
@@ -121,11 +126,11 @@ __global__ void __launch_bounds__(kThreads)
   auto FULL = [&](int s) -> uint32_t { return sbase + L::kOffBar + 8u * s; };
   auto EMPTY = [&](int s) -> uint32_t { return sbase + L::kOffBar + 8u * (kStages + s); };
 
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // GH query heads h0 .. h0+GH-1 that share KV head hkv (GH divides the group)
+  const int c = blockIdx.x, h0 = blockIdx.y * GH, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t bh = size_t(b) * p.H + h;
-  const size_t part = bh * p.C + c;
-  const int hkv = h / p.group;
+  const size_t bh0 = size_t(b) * p.H + h0;
+  const int hkv = h0 / p.group;
 
   int Lb = p.seqlens[b];
   Lb = Lb < 0 ? 0 : (Lb > p.Lmax ? p.Lmax : Lb);
@@ -134,8 +139,11 @@ __global__ void __launch_bounds__(kThreads)
   const int t0 = c * chunk;
   const int t1 = min(t0 + chunk, Lb);
   if (t0 >= t1) {  // empty chunk: weight 0 in the merge
-    for (int i = threadIdx.x; i < D; i += blockDim.x) p.part_o[part * D + i] = 0.f;
-    if (threadIdx.x == 0) p.part_lse[part] = -INFINITY;
+    for (int g = 0; g < GH; ++g) {
+      const size_t part = (bh0 + g) * p.C + c;
+      for (int i = threadIdx.x; i < D; i += blockDim.x) p.part_o[part * D + i] = 0.f;
+      if (threadIdx.x == 0) p.part_lse[part] = -INFINITY;
+    }
     return;
   }
   const int n_tok = t1 - t0;
@@ -159,7 +167,7 @@ __global__ void __launch_bounds__(kThreads)
       const uint16_t* kb = PAGED ? p.kc : p.kc + (bkv * p.Lmax + t0) * D;  // contiguous cache only
       const uint16_t* vb = PAGED ? p.vc : p.vc + (bkv * p.Lmax + t0) * D;
       int issued = 0, skip_stage = -1;
-      const bool skip = p.debug_skip && c == 0 && h == 0 && b == 0;
+      const bool skip = p.debug_skip && c == 0 && h0 == 0 && b == 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kStages;
         if (!wait_bounded(EMPTY(s), ((i / kStages) & 1) ^ 1, wc, 1)) break;
@@ -217,15 +225,21 @@ __global__ void __launch_bounds__(kThreads)
     const int j = lane & 15;      // this lane's slice of a row
     // the row whose full score this lane holds after the reduction below
     const int u_own = 2 * ((j >> 3) & 1) + ((j >> 2) & 1);
-    float qv[kPer];
-    {
-      const uint16_t* qp = p.q + bh * D + j * kPer;
+    float qv[GH][kPer];
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) qv[i] = __uint_as_float(uint32_t(qp[i]) << 16) * p.scale_log2;
+    for (int g = 0; g < GH; ++g) {
+      const uint16_t* qp = p.q + (bh0 + g) * D + j * kPer;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) qv[g][i] = __uint_as_float(uint32_t(qp[i]) << 16) * p.scale_log2;
     }
-    float m = -INFINITY, l = 0.f, acc[kPer];
+    float m[GH], l[GH], acc[GH][kPer];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+    for (int g = 0; g < GH; ++g) {
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) acc[g][i] = 0.f;
+    }
 
     for (int it = 0; it < n_tiles; ++it) {
       const int s = it % kStages;
@@ -235,88 +249,122 @@ __global__ void __launch_bounds__(kThreads)
       const int rows = min(kStageTok, n_tok - it * kStageTok);
       const uint8_t* ktile = smem + L::kOffK + s * L::kTileBytes;
       const uint8_t* vtile = smem + L::kOffV + s * L::kTileBytes;
-      // partial q.k of this lane's slice for the half-warp's 4 rows
-      float sc[kRowsPerHalf];
+      // partial q.k of this lane's slice for the half-warp's 4 rows, every
+      // query head from the one shared-memory read of the row
+      float sc[GH][kRowsPerHalf];
 #pragma unroll
       for (int u = 0; u < kRowsPerHalf; ++u) {
         const int r = warp * 2 * kRowsPerHalf + 2 * u + half;
-        float dot = 0.f;
+        float kx[kPer];
         if (r < rows) {
-          float kx[kPer];
           load_row_part<kPer>(ktile + r * D * 2, j, kx);
+        } else {
 #pragma unroll
-          for (int i = 0; i < kPer; ++i) dot = fmaf(qv[i], kx[i], dot);
+          for (int i = 0; i < kPer; ++i) kx[i] = 0.f;
         }
-        sc[u] = dot;
+#pragma unroll
+        for (int g = 0; g < GH; ++g) {
+          float dot = 0.f;
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) dot = fmaf(qv[g][i], kx[i], dot);
+          sc[g][u] = dot;
+        }
       }
       // sum over the 16 lanes of the half for all 4 rows at once: each
       // exchange halves the number of rows a lane carries
       const bool b3 = (j >> 3) & 1, b2 = (j >> 2) & 1;
-      float t0v = b3 ? sc[2] : sc[0], t1v = b3 ? sc[3] : sc[1];
-      t0v += __shfl_xor_sync(0xffffffffu, b3 ? sc[0] : sc[2], 8);
-      t1v += __shfl_xor_sync(0xffffffffu, b3 ? sc[1] : sc[3], 8);
-      float sv = b2 ? t1v : t0v;
-      sv += __shfl_xor_sync(0xffffffffu, b2 ? t0v : t1v, 4);
-      sv += __shfl_xor_sync(0xffffffffu, sv, 2);
-      sv += __shfl_xor_sync(0xffffffffu, sv, 1);
       const int r_own = warp * 2 * kRowsPerHalf + 2 * u_own + half;
       const bool valid = r_own < rows;
-      sv = valid ? sv : -INFINITY;
-      float mt = fmaxf(sv, __shfl_xor_sync(0xffffffffu, sv, 4));
-      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+      float sv[GH], mt[GH];
+#pragma unroll
+      for (int g = 0; g < GH; ++g) {
+        float t0v = b3 ? sc[g][2] : sc[g][0], t1v = b3 ? sc[g][3] : sc[g][1];
+        t0v += __shfl_xor_sync(0xffffffffu, b3 ? sc[g][0] : sc[g][2], 8);
+        t1v += __shfl_xor_sync(0xffffffffu, b3 ? sc[g][1] : sc[g][3], 8);
+        float v = b2 ? t1v : t0v;
+        v += __shfl_xor_sync(0xffffffffu, b2 ? t0v : t1v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        sv[g] = valid ? v : -INFINITY;
+        float x = fmaxf(sv[g], __shfl_xor_sync(0xffffffffu, sv[g], 4));
+        mt[g] = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+      }
       // warp-uniform (the shuffles below span both halves); a half with no
       // valid row in this stage keeps its state: alpha = 1 (or 0 before its
       // first row), p = 0
-      if (__any_sync(0xffffffffu, mt != -INFINITY)) {
-        const float m_new = fmaxf(m, mt);
-        const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-        m = m_new;
-        const float pr = valid ? ex2_approx(sv - m) : 0.f;
-        float ps = pr + __shfl_xor_sync(0xffffffffu, pr, 4);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-        l = l * alpha + ps;
+      if (__any_sync(0xffffffffu, valid)) {
+        float pr[GH];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) acc[i] *= alpha;
+        for (int g = 0; g < GH; ++g) {
+          const float m_new = fmaxf(m[g], mt[g]);
+          const float alpha = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - m_new);
+          m[g] = m_new;
+          pr[g] = valid ? ex2_approx(sv[g] - m[g]) : 0.f;
+          float ps = pr[g] + __shfl_xor_sync(0xffffffffu, pr[g], 4);
+          ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+          l[g] = l[g] * alpha + ps;
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) acc[g][i] *= alpha;
+        }
 #pragma unroll
         for (int u = 0; u < kRowsPerHalf; ++u) {
           // row u's probability sits in lanes with (j>>3, j>>2) = (u>>1, u&1)
-          const float pu = __shfl_sync(0xffffffffu, pr, half * 16 + 8 * (u >> 1) + 4 * (u & 1));
+          const int src = half * 16 + 8 * (u >> 1) + 4 * (u & 1);
+          float pu[GH];
+#pragma unroll
+          for (int g = 0; g < GH; ++g) pu[g] = __shfl_sync(0xffffffffu, pr[g], src);
           const int r = warp * 2 * kRowsPerHalf + 2 * u + half;
           if (r < rows) {
             float vx[kPer];
             load_row_part<kPer>(vtile + r * D * 2, j, vx);
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) acc[i] = fmaf(pu, vx[i], acc[i]);
+            for (int g = 0; g < GH; ++g)
+#pragma unroll
+              for (int i = 0; i < kPer; ++i) acc[g][i] = fmaf(pu[g], vx[i], acc[g][i]);
           }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(EMPTY(s));
     }
-    // per half-warp state to shared memory for the merge
-    float* mw = merge + (warp * 2 + half) * (D + 2);
-    if (j == 0) {
-      mw[0] = m;
-      mw[1] = l;
-    }
+    // every copy has landed and been read (or the CTA is aborting, and the
+    // producer lets its copies land before the barrier below)
+    __syncthreads();
+    if (*abort_flag) return;
+    // per half-warp and head state to shared memory (over the stage buffers)
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) mw[2 + j * kPer + i] = acc[i];
+    for (int g = 0; g < GH; ++g) {
+      float* mw = merge + ((warp * 2 + half) * GH + g) * (D + 2);
+      if (j == 0) {
+        mw[0] = m[g];
+        mw[1] = l[g];
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) mw[2 + j * kPer + i] = acc[g][i];
+    }
+  }
+  // the producer warp joins the consumers' first barrier here
+  if (warp == kConsumerWarps) {
+    __syncthreads();
+    if (*abort_flag) return;
   }
   __syncthreads();
-  if (*abort_flag) return;
-  // merge the 16 half-warp states (base-2 statistics) into this chunk's partial
+  // merge the 16 half-warp states (base-2 statistics) of each head into this
+  // chunk's partial
   constexpr int kStates = 2 * kConsumerWarps;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+  for (int e = threadIdx.x; e < GH * D; e += blockDim.x) {
+    const int g = e / D, i = e % D;
     float mm = -INFINITY;
-    for (int w = 0; w < kStates; ++w) mm = fmaxf(mm, merge[w * (D + 2)]);
+    for (int w = 0; w < kStates; ++w) mm = fmaxf(mm, merge[(w * GH + g) * (D + 2)]);
     float ll = 0.f, oo = 0.f;
     for (int w = 0; w < kStates; ++w) {
-      const float mw = merge[w * (D + 2)];
-      if (mw == -INFINITY) continue;
-      const float f = ex2_approx(mw - mm);
-      ll = fmaf(merge[w * (D + 2) + 1], f, ll);
-      oo = fmaf(merge[w * (D + 2) + 2 + i], f, oo);
+      const float* st = merge + (w * GH + g) * (D + 2);
+      if (st[0] == -INFINITY) continue;
+      const float f = ex2_approx(st[0] - mm);
+      ll = fmaf(st[1], f, ll);
+      oo = fmaf(st[2 + i], f, oo);
     }
+    const size_t part = (bh0 + g) * p.C + c;
     p.part_o[part * D + i] = oo / ll;
     if (i == 0) p.part_lse[part] = mm + lg2_approx(ll);
   }
@@ -353,16 +401,16 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecParams p) {
   if (i == 0) p.lse[bh] = (mx + lg2_approx(wsum)) * kLn2;
 }
 
-template <int D, bool PAGED>
+template <int D, bool PAGED, int GH>
 fa_status launch(const DecParams& p, int B, const LaunchCtx& ctx) {
   const int smem = DecLayout<D>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, PAGED>,
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, PAGED, GH>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
-  dim3 g1(p.C, p.H, B);
+  dim3 g1(p.C, p.H / GH, B);
   {
     ProfileScope prof(KID_DECODE, ctx.stream);
-    decode_split_kernel<D, PAGED><<<g1, kThreads, smem, ctx.stream>>>(p);
+    decode_split_kernel<D, PAGED, GH><<<g1, kThreads, smem, ctx.stream>>>(p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode split kernel launch");
@@ -428,7 +476,7 @@ fa_status launch_decode(const void* q, const void* kcache, const void* vcache, c
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load == KID_DECODE;
-  return d == 128 ? launch<128, false>(p, B, ctx) : launch<64, false>(p, B, ctx);
+  return d == 128 ? launch<128, false, 1>(p, B, ctx) : launch<64, false, 1>(p, B, ctx);
 }
 
 fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpages,
@@ -463,7 +511,13 @@ fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpa
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load == KID_DECODE;
-  return d == 128 ? launch<128, true>(p, B, ctx) : launch<64, true>(p, B, ctx);
+  // query heads per CTA: up to 4 of the heads that share a KV head
+  const int gh = (p.group % 4 == 0) ? 4 : (p.group % 2 == 0) ? 2 : 1;
+  if (d == 128)
+    return gh == 4 ? launch<128, true, 4>(p, B, ctx)
+                   : gh == 2 ? launch<128, true, 2>(p, B, ctx) : launch<128, true, 1>(p, B, ctx);
+  return gh == 4 ? launch<64, true, 4>(p, B, ctx)
+                 : gh == 2 ? launch<64, true, 2>(p, B, ctx) : launch<64, true, 1>(p, B, ctx);
 }
 
 }  // namespace fa

@@ -61,7 +61,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     # single-kernel mode, for profiler captures (prints timings, no bench line)
-    ap.add_argument("--kernel", choices=["fwd", "bwd", "decode"], default=None)
+    ap.add_argument("--kernel", choices=["fwd", "bwd", "decode", "decode_paged"], default=None)
+    ap.add_argument("--hkv", type=int, default=8, help="KV heads of --kernel decode_paged")
+    ap.add_argument("--page", type=int, default=64, help="page rows of --kernel decode_paged")
     ap.add_argument("--causal", type=int, default=0)
     ap.add_argument("--B", type=int, default=16)
     ap.add_argument("--H", type=int, default=16)
@@ -560,7 +562,22 @@ def run_single_kernel(args):
     def rnd(*shape):
         return torch.randn(shape, device="cuda", dtype=torch.bfloat16, generator=g)
 
-    if args.kernel == "decode":
+    if args.kernel == "decode_paged":
+        # pages [P, Hkv, page, d] in a shuffled order; N is the cache capacity
+        # per sequence, lengths drawn in [N/2, N]; H query heads share Hkv KV heads
+        page, hkv = args.page, args.hkv
+        lens = torch.randint(N // 2, N + 1, (B,), device="cuda", dtype=torch.int32, generator=g)
+        max_pages = (N + page - 1) // page
+        num_pages = B * max_pages
+        kp, vp = rnd(num_pages, hkv, page, d), rnd(num_pages, hkv, page, d)
+        perm = torch.randperm(num_pages, device="cuda", generator=g).to(torch.int32)
+        table = perm.view(B, max_pages).contiguous()
+        q = rnd(B, H, d)
+        ws = torch.empty(fa.fa_decode_workspace_size(B, H, max_pages * page, d, 0),
+                         dtype=torch.uint8, device="cuda")
+        kv_bytes = int(lens.sum().item()) * hkv * d * 2 * 2
+        fn = lambda: fa.fa_decode_paged(q, kp, vp, table, lens, workspace=ws)  # noqa: E731
+    elif args.kernel == "decode":
         q, kc, vc = rnd(B, H, d), rnd(B, H, N, d), rnd(B, H, N, d)
         lens = torch.randint(N // 2, N + 1, (B,), device="cuda", dtype=torch.int32, generator=g)
         ws = torch.empty(fa.fa_decode_workspace_size(B, H, N, d, 0), dtype=torch.uint8, device="cuda")
@@ -582,8 +599,12 @@ def run_single_kernel(args):
         fn()
         b.record()
         torch.cuda.synchronize()
+        extra = ""
+        if args.kernel == "decode_paged":
+            extra = (f" Hkv={args.hkv} page={args.page}: "
+                     f"{kv_bytes / (a.elapsed_time(b) * 1e-3) / 1e9:.1f} GB/s of KV pages")
         print(f"{args.kernel} B={B} H={H} N={N} d={d} causal={args.causal} "
-              f"iter {i}: {a.elapsed_time(b):.4f} ms", flush=True)
+              f"iter {i}: {a.elapsed_time(b):.4f} ms{extra}", flush=True)
     st, word = fa.fa_device_status()
     if st != 0:
         raise SystemExit(f"device status {st} ({word:#x})")

@@ -52,6 +52,7 @@ constexpr int kThreads = 32 * (kConsumerWarps + 1);
 constexpr int kRowsPerHalf = kStageTok / (2 * kConsumerWarps);  // 4
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSmHint = 148;      // B200 SM count, for the automatic split
+constexpr int kTcMinGroup = 4;    // query heads per KV head from which the tensor-core path runs
 
 template <int D>
 struct DecLayout {
@@ -401,6 +402,18 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecParams p) {
   if (i == 0) p.lse[bh] = (mx + lg2_approx(wsum)) * kLn2;
 }
 
+template <int D>
+fa_status launch_merge(const DecParams& p, int B, const LaunchCtx& ctx) {
+  dim3 g2(p.H, B);
+  {
+    ProfileScope prof(KID_DECODE_MERGE, ctx.stream);
+    decode_merge_kernel<D><<<g2, D, 0, ctx.stream>>>(p);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode merge kernel launch");
+  return FA_OK;
+}
+
 template <int D, bool PAGED, int GH>
 fa_status launch(const DecParams& p, int B, const LaunchCtx& ctx) {
   const int smem = DecLayout<D>::kSmemBytes;
@@ -511,6 +524,15 @@ fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpa
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load == KID_DECODE;
+  if (p.group >= kTcMinGroup) {
+    // large groups: the query heads of a KV head as the M rows of the tensor
+    // cores (decode_tc_sm100.cu), then the same merge
+    fa_status st = launch_decode_paged_tc(q, kpages, vpages, block_table, seqlens, B, Hq, Hkv,
+                                          num_pages, page_size, max_pages, d, scale, chunks,
+                                          p.part_o, p.part_lse, ctx);
+    if (st != FA_OK) return st;
+    return d == 128 ? launch_merge<128>(p, B, ctx) : launch_merge<64>(p, B, ctx);
+  }
   // query heads per CTA: up to 4 of the heads that share a KV head
   const int gh = (p.group % 4 == 0) ? 4 : (p.group % 2 == 0) ? 2 : 1;
   if (d == 128)

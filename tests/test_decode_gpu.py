@@ -185,3 +185,31 @@ def test_paged_decode_bad_page_is_reported_not_read():
     assert fa.fa_device_status()[0] == 0
     o, lse = run_paged(x)
     _check_paged(x, o, lse, 1 / np.sqrt(128))
+
+
+@pytest.mark.parametrize("heads", [(16, 1), (64, 1), (128, 2)], ids=["g16", "g64", "g128-2kv"])
+def test_paged_decode_large_groups(heads):
+    """Groups of 16, 64 and 128 query heads per KV head: the tensor-core path
+    with one, two and four softmax warps; lengths leave partial last tiles
+    over NaN-filled page rows."""
+    hq, hkv = heads
+    x = inputgen.make_paged_decode_inputs(620 + hq, 3, hq, hkv, 128, 64, seqlens=[1, 700, 4097])
+    o, lse = run_paged(x)
+    _check_paged(x, o, lse, 1 / np.sqrt(128))
+
+
+def test_paged_decode_tensor_core_bad_page_is_reported_not_read():
+    """As the bad-page test above, on the tensor-core path (4 query heads per
+    KV head): no page outside the pool is read, the status says so."""
+    x = inputgen.make_paged_decode_inputs(613, 2, 8, 2, 128, 32, seqlens=[200, 130])
+    q = bf16_device(x["q"])
+    kp, vp = bf16_device(x["kpages"]), bf16_device(x["vpages"])
+    lens = torch.from_numpy(x["seqlens"]).cuda()
+    bad = x["block_table"].copy()
+    bad[1, 2] = kp.shape[0]          # one past the pool
+    assert fa.fa_device_status()[0] == 0
+    fa.fa_decode_paged(q, kp, vp, torch.from_numpy(bad).cuda(), lens)
+    st, word = fa.fa_device_status()
+    assert st == 1 and (word >> 16) == 6 and (word & 0xff) == 2, (st, hex(word))
+    o, lse = run_paged(x)
+    _check_paged(x, o, lse, 1 / np.sqrt(128))

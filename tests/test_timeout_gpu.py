@@ -107,3 +107,20 @@ def test_hook_is_consumed_by_the_next_call():
     finally:
         fa.fa_debug_skip_load(0)
         fa.fa_set_wait_limit(0)
+
+
+def test_paged_tensor_core_decode_missing_load_times_out():
+    """The tensor-core paged decode (8 query heads per KV head): its first
+    CTA leaves out a V tile, the wait runs out and reports the decode kernel."""
+    x = inputgen.make_paged_decode_inputs(614, 2, 16, 2, 128, 64, seqlens=[500, 300])
+    q = bf16_device(x["q"])
+    kp, vp = bf16_device(x["kpages"]), bf16_device(x["vpages"])
+    table = torch.from_numpy(x["block_table"]).cuda()
+    lens = torch.from_numpy(x["seqlens"]).cuda()
+    _expect_timeout(6, lambda: fa.fa_decode_paged(q, kp, vp, table, lens))
+    o, lse = fa.fa_decode_paged(q, kp, vp, table, lens)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status()[0] == 0
+    ro, rl = oracle.decode_paged(f64(x["q"]), f64(x["kpages"]), f64(x["vpages"]),
+                                 x["block_table"], x["seqlens"], 1 / math.sqrt(128))
+    assert max_abs(o, ro) <= TOL_O and max_abs(lse, rl) <= TOL_LSE

@@ -28,6 +28,13 @@ Recipe
   permutation (``default_rng(seed + 7)``); rows past a sequence's end, and
   pages no sequence uses, hold NaN, and block-table entries past a
   sequence's last page hold -1, so a kernel that reads any of them is caught;
+* the FP8 inputs (``make_fp8_inputs``) draw, from ``default_rng(seed)`` in
+  this order, the d random signs of the rotation (``rng.choice([-1, 1])``
+  as float32), then for each of Q, K, V in turn a float32 N(0,1) array, a
+  uniform array that marks a fraction ``outlier_frac`` of the entries, and
+  a float32 N(0,1) array whose marked entries, times ``outlier_std``, are
+  added (outliers; 0.1% with std 10 in the tests); the sum is rounded to
+  bf16;
 * bf16 rounding is round-to-nearest-even on the fp32 bit pattern.
 """
 from __future__ import annotations
@@ -48,6 +55,7 @@ __all__ = [
     "make_decode_inputs",
     "make_paged_decode_inputs",
     "make_small_inputs",
+    "make_fp8_inputs",
     "sample_row_blocks",
 ]
 
@@ -216,6 +224,22 @@ def make_small_inputs(seed: int, B: int, H: int, N: int, d: int,
             out[n] = rng.standard_normal(shape, dtype=np.float32)
         else:
             out[n] = standard_normal_bf16(rng, shape)
+    return out
+
+
+def make_fp8_inputs(seed: int, B: int, H: int, N: int, d: int,
+                    outlier_frac: float = 0.0, outlier_std: float = 10.0):
+    """Q, K, V (bf16 bit patterns, [B, H, N, d]) with optional outliers, and
+    the d random signs of the rotation (float32 +-1)."""
+    rng = np.random.default_rng(seed)
+    signs = rng.choice(np.array([-1.0, 1.0], dtype=np.float32), size=d)
+    shape = (B, H, N, d)
+    out = {"signs": signs.astype(np.float32)}
+    for n in ("q", "k", "v"):
+        x = rng.standard_normal(shape, dtype=np.float32)
+        mark = rng.random(shape) < outlier_frac
+        extra = rng.standard_normal(shape, dtype=np.float32) * np.float32(outlier_std)
+        out[n] = bf16_round_bits(np.where(mark, x + extra, x).astype(np.float32))
     return out
 
 

@@ -16,3 +16,13 @@ from .attention import (  # noqa: F401
     scores,
     softmax_rows,
 )
+from .fp8 import (  # noqa: F401
+    attention_fp8,
+    attention_fp8_rounded_p,
+    e4m3_decode,
+    e4m3_encode,
+    fp8_dequantize,
+    fp8_prepare,
+    hadamard_rotate_f32,
+    quantize_blocks,
+)

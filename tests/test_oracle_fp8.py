@@ -1,0 +1,312 @@
+"""Pins of the FP8 oracle (CPU only), and planted mistakes they must catch.
+
+What pins it, besides itself: torch's float8_e4m3fn conversion (a library
+routine) and codes decoded by hand from the e4m3 format; scipy's Sylvester
+Hadamard matrix; the identities H H = d I and (x R)(y R)^T = d x y^T;
+inputs that lie exactly on the e4m3 grid, which must come back exactly; and
+the page's claim that the rotation lowers the FP8 attention error on inputs
+with outliers ("FlashAttention-3 (TR)", section "FlashAttention-3'un
+Teknik Yenilikleri", item 3).
+"""
+import contextlib
+import math
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import inputgen
+import oracle
+from oracle import fp8 as F
+
+
+def _torch_e4m3(x):
+    t = torch.from_numpy(np.asarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def _bf16(bits):
+    return inputgen.bf16_bits_to_f32(bits)
+
+
+# ---------------------------------------------------------------------------
+# pins
+# ---------------------------------------------------------------------------
+
+def pin_decode_table():
+    c = np.array([0x00, 0x01, 0x07, 0x08, 0x38, 0x3F, 0x40, 0x7E, 0x80, 0xB8, 0xFE], dtype=np.uint8)
+    want = [0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, 1.875, 2.0, 448.0, -0.0, -1.0, -448.0]
+    got = F.e4m3_decode(c)
+    assert np.array_equal(got, np.array(want))
+    assert np.signbit(got[8])
+    assert np.isnan(F.e4m3_decode(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+    pos = F.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0)  # codes 0..126 increase strictly
+
+
+def pin_encode_matches_library():
+    rng = np.random.default_rng(5)
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * 40,
+        rng.standard_normal(20000).astype(np.float32) * 0.01,  # subnormal range
+        np.float32([0.0, -0.0, 448.0, -448.0, 2 ** -10, 3 * 2 ** -10, 2 ** -7 * 1.5]),
+    ])
+    # exact midpoints between neighbouring codes: ties go to the even code
+    vals = F.e4m3_decode(np.arange(0x7E, dtype=np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids])
+    x = np.clip(x, -448, 448)
+    assert np.array_equal(F.e4m3_encode(x), _torch_e4m3(x))
+    even = F.e4m3_encode(mids) & 1
+    assert not even.any()
+
+
+def pin_encode_saturates_and_round_trips():
+    big = np.float32([449.0, 463.9, 464.0, 1000.0, 3e38, -500.0])
+    assert list(F.e4m3_encode(big)) == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    assert np.array_equal(F.e4m3_encode(F.e4m3_decode(codes).astype(np.float32)), codes)
+
+
+def pin_rotation_is_sylvester_hadamard():
+    rng = np.random.default_rng(6)
+    for d in (64, 128):
+        H = scipy.linalg.hadamard(d).astype(np.float64)
+        signs = rng.choice([-1.0, 1.0], size=d).astype(np.float32)
+        xi = rng.integers(-8, 9, size=(5, d)).astype(np.float32)  # sums stay exact
+        assert np.array_equal(F.hadamard_rotate_f32(xi, signs).astype(np.float64),
+                              (xi * signs) @ H)
+        x = rng.standard_normal((7, d)).astype(np.float32)
+        np.testing.assert_allclose(F.hadamard_rotate_f32(x, signs), (x.astype(np.float64) * signs) @ H,
+                                   rtol=0, atol=1e-4)
+
+
+def pin_rotation_identities():
+    rng = np.random.default_rng(7)
+    d = 128
+    xi = rng.integers(-4, 5, size=(3, d)).astype(np.float32)
+    ones = np.ones(d, dtype=np.float32)
+    twice = F.hadamard_rotate_f32(F.hadamard_rotate_f32(xi, ones), ones)
+    assert np.array_equal(twice, d * xi)  # H H = d I
+    signs = rng.choice([-1.0, 1.0], size=d).astype(np.float32)
+    x, y = rng.standard_normal((4, d)), rng.standard_normal((6, d))
+    xr = F.hadamard_rotate_f32(x, signs).astype(np.float64)
+    yr = F.hadamard_rotate_f32(y, signs).astype(np.float64)
+    np.testing.assert_allclose(xr @ yr.T, d * (x.astype(np.float32).astype(np.float64)
+                                               @ y.astype(np.float32).astype(np.float64).T),
+                               rtol=1e-5, atol=1e-3)
+
+
+def _grid_values(rng, shape, scale_exp):
+    """Values on the e4m3 grid times 2^scale_exp, each 128-row block holding
+    a +-448 entry so that its scale is exactly 2^scale_exp."""
+    codes = rng.integers(0, 0x7F, size=shape).astype(np.uint8) | (
+        rng.integers(0, 2, size=shape).astype(np.uint8) << 7)
+    x = F.e4m3_decode(codes) * 2.0 ** scale_exp
+    x[..., ::128, 0] = 448.0 * 2.0 ** scale_exp
+    return x.astype(np.float32)
+
+
+def pin_quantize_exact_on_grid():
+    rng = np.random.default_rng(8)
+    x = _grid_values(rng, (2, 200, 64), -3)
+    codes, scales = F.quantize_blocks(x)
+    assert scales.shape == (2, 2) and np.all(scales == np.float32(2.0 ** -3))
+    rows = np.arange(200) // 128
+    back = F.e4m3_decode(codes) * scales[:, rows][..., None]
+    assert np.array_equal(back, x.astype(np.float64))
+    z_codes, z_scales = F.quantize_blocks(np.zeros((1, 130, 64), dtype=np.float32))
+    assert np.all(z_scales == 1) and not z_codes.any()
+
+
+def pin_quantize_error_bound():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((1, 300, 128)).astype(np.float32) * 3
+    codes, scales = F.quantize_blocks(x)
+    back = F.e4m3_decode(codes) * scales[:, np.arange(300) // 128][..., None]
+    s = scales[:, np.arange(300) // 128][..., None].astype(np.float64)
+    # normal codes: relative error <= 2^-4; subnormal codes: absolute 2^-10 * scale
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * s)
+    assert np.all(np.abs(back - x) <= bound * (1 + 1e-12))
+    for b in range(3):
+        blk = np.abs(F.e4m3_decode(codes[0, b * 128:(b + 1) * 128]))
+        assert blk.max() == 448.0  # every block's largest entry maps to 448
+
+
+def pin_attention_exact_on_grid():
+    """No rotation and operands on the grid: the FP8 attention is the exact
+    attention of the inputs themselves."""
+    rng = np.random.default_rng(10)
+    q, k = _grid_values(rng, (1, 2, 256, 128), -7), _grid_values(rng, (1, 2, 256, 128), -7)
+    v = _grid_values(rng, (1, 2, 256, 128), -6)
+    for h in range(2):
+        v[0, h].flat[0] = 448.0 * 2.0 ** -6  # per-head amax -> scale 2^-6
+    prep = F.fp8_prepare(q, k, v, None)
+    for causal in (False, True):
+        o, lse = F.attention_fp8(prep, 1 / math.sqrt(128), causal)
+        ro, rl = oracle.attention_fwd(q, k, v, 1 / math.sqrt(128), causal)
+        np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-12)
+
+
+def _rms(a, b):
+    return float(np.sqrt(np.mean((np.asarray(a) - np.asarray(b)) ** 2)))
+
+
+def pin_rotation_keeps_attention():
+    """With the rotation, the dequantised Q^ K^T is Q K^T up to FP8 rounding:
+    the FP8 attention is within the FP8 error of the exact one, and dropping
+    the rotation's 1/d (or the signs on one side) would not be."""
+    x = inputgen.make_fp8_inputs(11, 1, 2, 256, 128)
+    q, k, v = (_bf16(x[n]) for n in ("q", "k", "v"))
+    prep = F.fp8_prepare(q, k, v, x["signs"])
+    o, lse = F.attention_fp8(prep, 1 / math.sqrt(128), True)
+    ro, rl = oracle.attention_fwd(q, k, v, 1 / math.sqrt(128), True)
+    assert _rms(o, ro) < 1e-2 and np.max(np.abs(lse - rl)) < 0.1
+    assert _rms(o, ro) > 1e-5  # FP8 is not exact
+
+
+def pin_rotation_lowers_error_with_outliers():
+    """The page's claim, at a smaller size: 0.1% outliers of std 10 in Q, K
+    and V; the rotation lowers the RMS error of the FP8 attention against
+    the exact attention of the bf16 inputs (1.33-1.40x for seeds 12-14 at
+    this size, block scales on both sides)."""
+    x = inputgen.make_fp8_inputs(12, 1, 2, 512, 128, outlier_frac=0.001, outlier_std=10.0)
+    q, k, v = (_bf16(x[n]) for n in ("q", "k", "v"))
+    ro, _ = oracle.attention_fwd(q, k, v, 1 / math.sqrt(128), False)
+    plain, _ = F.attention_fp8(F.fp8_prepare(q, k, v, None), 1 / math.sqrt(128), False)
+    rot, _ = F.attention_fp8(F.fp8_prepare(q, k, v, x["signs"]), 1 / math.sqrt(128), False)
+    ratio = _rms(plain, ro) / _rms(rot, ro)
+    assert ratio > 1.2, ratio
+
+
+def pin_rounded_p_is_small_and_nonzero():
+    x = inputgen.make_fp8_inputs(13, 1, 1, 384, 128)
+    q, k, v = (_bf16(x[n]) for n in ("q", "k", "v"))
+    prep = F.fp8_prepare(q, k, v, x["signs"])
+    exact, _ = F.attention_fp8(prep, 1 / math.sqrt(128), False)
+    rp = F.attention_fp8_rounded_p(prep, 1 / math.sqrt(128), False)
+    assert 1e-5 < _rms(rp, exact) < 5e-3
+
+
+PINS = [
+    pin_decode_table,
+    pin_encode_matches_library,
+    pin_encode_saturates_and_round_trips,
+    pin_rotation_is_sylvester_hadamard,
+    pin_rotation_identities,
+    pin_quantize_exact_on_grid,
+    pin_quantize_error_bound,
+    pin_attention_exact_on_grid,
+    pin_rotation_keeps_attention,
+    pin_rotation_lowers_error_with_outliers,
+    pin_rounded_p_is_small_and_nonzero,
+]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin(pin):
+    pin()
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes
+# ---------------------------------------------------------------------------
+
+_orig = {n: getattr(F, n) for n in ("e4m3_encode", "e4m3_decode", "hadamard_rotate_f32",
+                                     "quantize_blocks", "fp8_prepare", "fp8_dequantize")}
+
+
+def _mut_encode_half_up(x):
+    x = np.asarray(x, dtype=np.float32)
+    a = np.abs(x.astype(np.float64))
+    with np.errstate(divide="ignore"):
+        e = np.clip(np.floor(np.log2(np.where(a > 0, a, 1.0))), -6, 8)
+    step = np.exp2(e - 3)
+    q = np.minimum(np.floor(a / step + 0.5) * step, 448.0)
+    return _orig["e4m3_encode"](np.where(np.signbit(x), -q, q).astype(np.float32))
+
+
+def _mut_encode_no_subnormals(x):
+    x = np.asarray(x, dtype=np.float32)
+    return np.where(np.abs(x) < 2.0 ** -6, np.where(np.signbit(x), 0x80, 0),
+                    _orig["e4m3_encode"](x)).astype(np.uint8)
+
+
+def _mut_decode_bias_8(codes):
+    return _orig["e4m3_decode"](codes) / 2.0
+
+
+def _mut_rotate_no_signs(x, signs):
+    return _orig["hadamard_rotate_f32"](x, np.ones_like(np.asarray(signs)))
+
+
+def _mut_rotate_wrong_butterfly(x, signs):
+    y = np.asarray(x, dtype=np.float32).copy()
+    y = np.where(np.signbit(np.asarray(signs, dtype=np.float32)), -y, y).astype(np.float32)
+    d, h = y.shape[-1], 1
+    while h < d:
+        idx = np.arange(d)
+        lo = idx[(idx & h) == 0]
+        a, b = y[..., lo].copy(), y[..., lo + h].copy()
+        y[..., lo], y[..., lo + h] = a + b, b - a  # sign of the difference flipped
+        h *= 2
+    return y
+
+
+def _mut_quantize_scale_per_tensor(x, block=128):
+    n = np.asarray(x).shape[1]
+    codes, scales = _orig["quantize_blocks"](x, block=n)  # one scale per head
+    return codes, np.repeat(scales, -(-n // block), axis=1)
+
+
+def _mut_prepare_no_inverse_d(q, k, v, signs=None):
+    prep = _orig["fp8_prepare"](q, k, v, signs)
+    if signs is not None:
+        prep["q_scale"] = prep["q_scale"] * np.float32(len(signs))
+    return prep
+
+
+def _mut_dequantize_v_unscaled(prep):
+    qd, kd, vd = _orig["fp8_dequantize"](prep)
+    return qd, kd, F.e4m3_decode(prep["v8"])
+
+
+FP8_MUTANTS = {
+    "encode_round_half_up": {"e4m3_encode": _mut_encode_half_up},
+    "encode_flushes_subnormals": {"e4m3_encode": _mut_encode_no_subnormals},
+    "decode_wrong_bias": {"e4m3_decode": _mut_decode_bias_8},
+    "rotate_without_signs": {"hadamard_rotate_f32": _mut_rotate_no_signs},
+    "rotate_difference_flipped": {"hadamard_rotate_f32": _mut_rotate_wrong_butterfly},
+    "quantize_per_tensor": {"quantize_blocks": _mut_quantize_scale_per_tensor},
+    "prepare_drops_inverse_d": {"fp8_prepare": _mut_prepare_no_inverse_d},
+    "dequantize_v_unscaled": {"fp8_dequantize": _mut_dequantize_v_unscaled},
+}
+
+
+@contextlib.contextmanager
+def planted(patches):
+    saved = []
+    for name, fn in patches.items():
+        for mod in (F, oracle):
+            if hasattr(mod, name):
+                saved.append((mod, name, getattr(mod, name)))
+                setattr(mod, name, fn)
+    try:
+        yield
+    finally:
+        for mod, name, fn in reversed(saved):
+            setattr(mod, name, fn)
+
+
+@pytest.mark.parametrize("mutant", sorted(FP8_MUTANTS))
+def test_fp8_mutant_is_caught(mutant):
+    caught = []
+    with planted(FP8_MUTANTS[mutant]):
+        for pin in PINS:
+            try:
+                pin()
+            except Exception:
+                caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {mutant}"

@@ -61,7 +61,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     # single-kernel mode, for profiler captures (prints timings, no bench line)
-    ap.add_argument("--kernel", choices=["fwd", "bwd", "decode", "decode_paged"], default=None)
+    ap.add_argument("--kernel", choices=["fwd", "fwd_fp8", "fp8_prep", "bwd", "decode", "decode_paged"],
+                    default=None)
     ap.add_argument("--hkv", type=int, default=8, help="KV heads of --kernel decode_paged")
     ap.add_argument("--page", type=int, default=64, help="page rows of --kernel decode_paged")
     ap.add_argument("--causal", type=int, default=0)
@@ -577,6 +578,18 @@ def run_single_kernel(args):
                          dtype=torch.uint8, device="cuda")
         kv_bytes = int(lens.sum().item()) * hkv * d * 2 * 2
         fn = lambda: fa.fa_decode_paged(q, kp, vp, table, lens, workspace=ws)  # noqa: E731
+    elif args.kernel in ("fwd_fp8", "fp8_prep"):
+        # FP8 forward with incoherent processing: random signs, rotated and
+        # block-quantised Q, K; the timed call is the forward on the codes
+        # (fwd_fp8) or the preparation itself (fp8_prep)
+        q, k, v = rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d)
+        signs = torch.where(torch.rand(d, device="cuda", generator=g) < 0.5, -1.0, 1.0)
+        prep = fa.fa_fp8_prepare(q, k, v, signs)
+        if args.kernel == "fp8_prep":
+            fn = lambda: fa.fa_fp8_prepare(q, k, v, signs, out=prep)  # noqa: E731
+        else:
+            o, lse = fa.fa_fwd_fp8(prep, causal=bool(args.causal))
+            fn = lambda: fa.fa_fwd_fp8(prep, causal=bool(args.causal), o=o, lse=lse)  # noqa: E731
     elif args.kernel == "decode":
         q, kc, vc = rnd(B, H, d), rnd(B, H, N, d), rnd(B, H, N, d)
         lens = torch.randint(N // 2, N + 1, (B,), device="cuda", dtype=torch.int32, generator=g)
@@ -603,6 +616,9 @@ def run_single_kernel(args):
         if args.kernel == "decode_paged":
             extra = (f" Hkv={args.hkv} page={args.page}: "
                      f"{kv_bytes / (a.elapsed_time(b) * 1e-3) / 1e9:.1f} GB/s of KV pages")
+        elif args.kernel in ("fwd", "fwd_fp8"):
+            fl = 4.0 * B * H * N * N * d / (2 if args.causal else 1)
+            extra = f": {fl / (a.elapsed_time(b) * 1e-3) / 1e12:.1f} TFLOP/s"
         print(f"{args.kernel} B={B} H={H} N={N} d={d} causal={args.causal} "
               f"iter {i}: {a.elapsed_time(b):.4f} ms{extra}", flush=True)
     st, word = fa.fa_device_status()

@@ -6,7 +6,8 @@ memory and the current stream. There is no CPU fallback: if the library is
 missing, every call raises.
 
 Functions carry the C names:
-    fa_fwd, fa_fwd_f32, fa_bwd, fa_bwd_workspace_size,
+    fa_fwd, fa_fwd_f32, fa_fp8_prepare, fa_fwd_fp8, fa_fp8_vt_keys,
+    fa_bwd, fa_bwd_workspace_size,
     fa_decode_splitkv, fa_decode_workspace_size,
     fa_device_status, fa_set_wait_limit, fa_debug_skip_load
 """
@@ -19,7 +20,8 @@ import re
 
 __all__ = [
     "FAError", "library_path", "load_library", "exported_symbols",
-    "fa_fwd", "fa_fwd_f32", "fa_bwd", "fa_bwd_workspace_size",
+    "fa_fwd", "fa_fwd_f32", "fa_fp8_prepare", "fa_fwd_fp8", "fa_fp8_vt_keys",
+    "fa_bwd", "fa_bwd_workspace_size",
     "fa_decode_splitkv", "fa_decode_workspace_size", "fa_decode_splitkv_static",
     "fa_decode_paged",
     "fa_device_status",
@@ -58,6 +60,9 @@ _SIGNATURES = {
     "fa_abi_version": (_I, []),
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fp8_vt_keys": (_I, [_I]),
+    "fa_fp8_prepare": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I,
                     _P, _S, _P]),
@@ -75,7 +80,7 @@ _SIGNATURES = {
 }
 
 KERNEL_NAMES = {1: "fwd", 2: "fwd_f32", 3: "bwd_pre", 4: "bwd_dkdv", 5: "bwd_dq",
-                6: "decode_split", 7: "decode_merge"}
+                6: "decode_split", 7: "decode_merge", 9: "fp8_prep"}
 
 
 def load_library():
@@ -176,6 +181,72 @@ def fa_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None,
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     _check(lib.fa_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N,
                           d, scale, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_fp8_vt_keys(N: int) -> int:
+    """Keys per row of the transposed V codes (N rounded up to 16)."""
+    return int(load_library().fa_fp8_vt_keys(N))
+
+
+def fa_fp8_prepare(q, k, v, signs=None, out=None, stream=None):
+    """Rotate (when ``signs`` is given) and quantise bf16 q, k, v
+    [B, H, N, 128] to e4m3 codes for ``fa_fwd_fp8``. Returns a dict with
+    q8, k8 (uint8 [B, H, N, 128]), vt8 (uint8 [B, H, 128, fa_fp8_vt_keys(N)]),
+    q_scale, k_scale (fp32 [B, H, ceil(N / 128)]) and v_amax (fp32 [B, H]);
+    ``out`` may supply those tensors."""
+    import torch
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    if signs is not None:
+        _need(signs, torch.float32, "signs")
+        if signs.numel() != d:
+            raise ValueError("signs must hold d entries")
+    nb = (N + 127) // 128
+    dev = q.device
+    if out is None:
+        u8 = torch.uint8
+        out = {
+            "q8": torch.empty((B, H, N, d), dtype=u8, device=dev),
+            "k8": torch.empty((B, H, N, d), dtype=u8, device=dev),
+            "vt8": torch.empty((B, H, d, max(fa_fp8_vt_keys(N), 1)), dtype=u8, device=dev),
+            "q_scale": torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+            "k_scale": torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+            "v_amax": torch.empty((B, H), dtype=torch.float32, device=dev),
+        }
+    for n in ("q8", "k8", "vt8"):
+        _need(out[n], torch.uint8, n)
+    for n in ("q_scale", "k_scale", "v_amax"):
+        _need(out[n], torch.float32, n)
+    _check(lib.fa_fp8_prepare(_ptr(q), _ptr(k), _ptr(v), _ptr(signs) if signs is not None else None,
+                              B, H, N, d, _ptr(out["q8"]), _ptr(out["k8"]), _ptr(out["vt8"]),
+                              _ptr(out["q_scale"]), _ptr(out["k_scale"]), _ptr(out["v_amax"]),
+                              _stream(stream)))
+    return out
+
+
+def fa_fwd_fp8(prep, causal: bool = False, scale: float | None = None, o=None, lse=None,
+               stream=None):
+    """O (bf16), LSE = attention of the FP8 operands that ``fa_fp8_prepare``
+    made (``scale`` applies to the original Q K^T, default 1/sqrt(d))."""
+    import torch
+    lib = load_library()
+    q8 = prep["q8"]
+    B, H, N, d = q8.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if o is None:
+        o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    _check(lib.fa_fwd_fp8(_ptr(q8), _ptr(prep["k8"]), _ptr(prep["vt8"]), _ptr(prep["q_scale"]),
+                          _ptr(prep["k_scale"]), _ptr(prep["v_amax"]), _ptr(o), _ptr(lse),
+                          B, H, N, d, scale, int(bool(causal)), _stream(stream)))
     return o, lse
 
 

@@ -1038,16 +1038,16 @@ fa_status launch_all(const void* q, const void* k, const void* v, const void* dO
   CUtensorMap m[8], mq[8];
   const void* src[4] = {q, dO, k, v};
   for (int i = 0; i < 4; ++i) {
-    fa_status st = make_tmap_3d(&m[i], src[i], true, D, p.N, p.BH, 64, kTile, 128);
+    fa_status st = make_tmap_3d(&m[i], src[i], 2, D, p.N, p.BH, 64, kTile, 128);
     if (st != FA_OK) return st;
   }
-  fa_status st = make_tmap_3d(&m[4], p.qext, true, 16, p.Np, p.BH, 16, kTile, 32);
-  if (st == FA_OK) st = make_tmap_3d(&m[5], p.dext, true, 16, p.Np, p.BH, 16, kTile, 32);
-  if (st == FA_OK) st = make_tmap_3d(&m[6], p.dk, true, D, p.N, p.BH, 64, kTile, 128);
-  if (st == FA_OK) st = make_tmap_3d(&m[7], p.dv, true, D, p.N, p.BH, 64, kTile, 128);
+  fa_status st = make_tmap_3d(&m[4], p.qext, 2, 16, p.Np, p.BH, 16, kTile, 32);
+  if (st == FA_OK) st = make_tmap_3d(&m[5], p.dext, 2, 16, p.Np, p.BH, 16, kTile, 32);
+  if (st == FA_OK) st = make_tmap_3d(&m[6], p.dk, 2, D, p.N, p.BH, 64, kTile, 128);
+  if (st == FA_OK) st = make_tmap_3d(&m[7], p.dv, 2, D, p.N, p.BH, 64, kTile, 128);
   if (st != FA_OK) return st;
   for (int i = 0; i < 6; ++i) mq[i] = m[i];
-  st = make_tmap_3d(&mq[6], p.dq, true, D, p.N, p.BH, 64, kTile, 128);
+  st = make_tmap_3d(&mq[6], p.dq, 2, D, p.N, p.BH, 64, kTile, 128);
   if (st != FA_OK) return st;
   mq[7] = mq[6];
   // both kernels are persistent: one CTA per SM walks its items

@@ -426,9 +426,9 @@ fa_status launch_decode_paged_tc(const void* q, const void* kpages, const void* 
   const uint32_t box_rows = page_size < kTileKeys ? uint32_t(page_size) : uint32_t(kTileKeys);
   CUtensorMap mk, mv;
   fa_status st;
-  if ((st = make_tmap_3d(&mk, kpages, true, d, page_size, outer, 64, box_rows, 128)) != FA_OK)
+  if ((st = make_tmap_3d(&mk, kpages, 2, d, page_size, outer, 64, box_rows, 128)) != FA_OK)
     return st;
-  if ((st = make_tmap_3d(&mv, vpages, true, d, page_size, outer, 64, box_rows, 128)) != FA_OK)
+  if ((st = make_tmap_3d(&mv, vpages, 2, d, page_size, outer, 64, box_rows, 128)) != FA_OK)
     return st;
   TcParams p;
   p.q = static_cast<const uint16_t*>(q);

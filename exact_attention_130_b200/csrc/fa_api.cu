@@ -172,7 +172,7 @@ fa_status current_launch_ctx(cudaStream_t stream, LaunchCtx* ctx) {
   return device_ctx(stream, ctx);
 }
 
-fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t inner,
+fa_status make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner,
                        uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows,
                        int swizzle_bytes) {
   std::call_once(g_encode_once, [] {
@@ -184,13 +184,17 @@ fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
   });
   if (!g_encode) return invalid(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  const uint64_t elem = is_bf16 ? 2 : 4;
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4)
+    return invalid(FA_ERR_UNSUPPORTED, "tensor map element size %d", elem_bytes);
+  const uint64_t elem = uint64_t(elem_bytes);
+  const CUtensorMapDataType dtype = elem_bytes == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                    : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   cuuint64_t dims[3] = {inner, rows, outer};
   cuuint64_t strides[2] = {inner * elem, inner * rows * elem};
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                        3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = g_encode(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                         : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
@@ -222,7 +226,7 @@ const char* fa_status_string(fa_status s) {
 
 const char* fa_last_error(void) { return t_last_error; }
 
-int fa_abi_version(void) { return 101; }
+int fa_abi_version(void) { return 102; }
 
 void fa_set_wait_limit(unsigned long long ns) {
   g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs);
@@ -253,6 +257,47 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, f
   LaunchCtx ctx;
   if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
   return launch_fwd_f32(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx);
+}
+
+int fa_fp8_vt_keys(int N) { return N >= 1 && N <= 0x7ffffff0 ? fp8_vt_keys(N) : 0; }
+
+fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const float* signs, int B,
+                         int H, int N, int d, void* q8, void* k8, void* vt8, float* q_scale,
+                         float* k_scale, float* v_amax, cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, k, v, q8, k8, vt8, q_scale, k_scale, v_amax},
+                       "fa_fp8_prepare(q,k,v,q8,k8,vt8,q_scale,k_scale,v_amax)")) != FA_OK)
+    return st;
+  if (signs != nullptr && (reinterpret_cast<uintptr_t>(signs) & 3u) != 0)
+    return invalid(FA_ERR_ALIGNMENT, "signs is not 4-byte aligned");
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if (d != 128) return invalid(FA_ERR_UNSUPPORTED, "the FP8 path needs d = 128 (got %d)", d);
+  if ((long long)B * H > 65535)
+    return invalid(FA_ERR_INVALID_ARG, "B*H = %lld exceeds 65535", (long long)B * H);
+  if ((long long)B * H * d * fp8_vt_keys(N) > 0x7fffffffffffLL)
+    return invalid(FA_ERR_INVALID_ARG, "the transposed V is too large");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  return launch_fp8_prepare(q, k, v, signs, B, H, N, d, q8, k8, vt8, q_scale, k_scale, v_amax,
+                            ctx);
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* q_scale,
+                     const float* k_scale, const float* v_amax, void* o, float* lse, int B, int H,
+                     int N, int d, float scale, int causal, cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q8, k8, vt8, q_scale, k_scale, v_amax, o, lse},
+                       "fa_fwd_fp8(q8,k8,vt8,q_scale,k_scale,v_amax,o,lse)")) != FA_OK)
+    return st;
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if (d != 128) return invalid(FA_ERR_UNSUPPORTED, "the FP8 path needs d = 128 (got %d)", d);
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (causal != 0 && causal != 1) return invalid(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  ctx.debug_skip_load = g_debug_skip.exchange(0);
+  return launch_fwd_fp8(q8, k8, vt8, q_scale, k_scale, v_amax, o, lse, B, H, N, d, scale,
+                        causal != 0, ctx);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -382,7 +427,7 @@ int fa_profile_end(int* launches, double* total_ms, int capacity) {
     if (launches) launches[k] = 0;
     if (total_ms) total_ms[k] = 0.0;
   }
-  int rc = 9;
+  int rc = 10;
   for (auto& r : g_prof) {
     float ms = 0.f;
     if (cudaEventSynchronize(r.stop) != cudaSuccess ||

@@ -28,6 +28,7 @@ enum KernelId : unsigned int {
   KID_BWD_DQ = 5,   // dQ kernel
   KID_DECODE = 6,
   KID_DECODE_MERGE = 7,
+  KID_FP8_PREP = 9,  // FP8 rotation and quantisation (no waits)
 };
 
 // Brackets one kernel launch with CUDA events when profiling is on
@@ -53,16 +54,26 @@ fa_status current_launch_ctx(cudaStream_t stream, LaunchCtx* ctx);
 void set_last_error(const char* fmt, ...);
 fa_status cuda_fail(cudaError_t e, const char* what);
 
-// 3-D tiled tensor map over a [outer, rows, inner] bf16 or fp32 tensor
-// (inner contiguous), box = box_inner x box_rows x 1, zero fill out of bounds.
-// swizzle_bytes: 128 or 32 (box_inner * elem must then equal it) or 0.
-fa_status make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t inner,
+// 3-D tiled tensor map over a [outer, rows, inner] tensor of 1-byte (uint8
+// codes), 2-byte (bf16) or 4-byte (fp32) elements (inner contiguous), box =
+// box_inner x box_rows x 1, zero fill out of bounds. swizzle_bytes: 128 or
+// 32 (box_inner * elem_bytes must then equal it) or 0.
+fa_status make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner,
                        uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows,
                        int swizzle_bytes);
 
 fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int N, int d, float scale, bool causal,
                           const LaunchCtx& ctx);
+// Keys per row of the transposed FP8 V ([B, H, d, fp8_vt_keys(N)] codes):
+// N rounded up to 16, so that every row starts 16-byte aligned.
+inline int fp8_vt_keys(int N) { return (N + 15) & ~15; }
+fa_status launch_fp8_prepare(const void* q, const void* k, const void* v, const float* signs,
+                             int B, int H, int N, int d, void* q8, void* k8, void* vt8,
+                             float* q_scale, float* k_scale, float* v_amax, const LaunchCtx& ctx);
+fa_status launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* q_scale,
+                         const float* k_scale, const float* v_amax, void* o, float* lse, int B,
+                         int H, int N, int d, float scale, bool causal, const LaunchCtx& ctx);
 fa_status launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                          int B, int H, int N, int d, float scale, bool causal,
                          const LaunchCtx& ctx);

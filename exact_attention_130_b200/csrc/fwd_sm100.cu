@@ -47,6 +47,17 @@
 //    waited for each of its phases in turn by its one waiter, or indexed so
 //    that a waiter is never more than one phase away from the phase it
 //    waits for (the arguments are given at each barrier).
+//
+// The FP8 instantiation (F8, d = 128; "FlashAttention-3 (TR)", section
+// "FlashAttention-3'un Teknik Yenilikleri", item 3) runs the same pipeline
+// on e4m3 codes prepared by fp8_prep.cu: Q and K codes with one scale per
+// 128-row block, V transposed ([d, keys] per head, so it is the K-major B
+// operand of P V) with one scale per head. Both products are
+// tcgen05.mma .kind::f8f6f4 (K = 32 per instruction); the scores of step j
+// are scaled by scale * log2(e) * q_scale(Q tile) * k_scale(K tile); P~ is
+// rounded to e4m3 (it is at most 2^8, the lazy-rescale bound, inside
+// e4m3's 448) while the row sum keeps the fp32 values; the epilogue
+// multiplies O~ by v_scale / l.
 #include <cfloat>
 
 #include "fa_internal.h"
@@ -103,17 +114,22 @@ enum : int {
   B_COUNT = B_V_EMPTY + kMaxStages
 };
 
-template <int D>
+template <int D, bool F8>
 struct Layout {
-  static constexpr int kSub = D / 64;          // 128-byte column groups per row
-  static constexpr int kSubBytes = 128 * 128;  // 128 rows x 128 bytes
-  static constexpr int kTileBytes = kSub * kSubBytes;
-  static constexpr int kKStages = (D == 128) ? 2 : 4;
-  static constexpr int kVStages = (D == 128) ? 2 : 4;
+  static constexpr int kElem = F8 ? 1 : 2;             // bytes per Q/K/V element
+  static constexpr int kSub = D * kElem / 128;         // 128-byte column groups per row
+  static constexpr int kSubBytes = 128 * 128;          // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kSub * kSubBytes;  // a Q, K or V (V^T for F8) tile
+  static constexpr int kStgBytes = (D * 2 / 128) * kSubBytes;  // bf16 O staging tile
+  static constexpr int kKSteps = D * kElem / 32;       // 32-byte K steps of Q K^T
+  static constexpr int kPvSteps = kBN * kElem / 32;    // 32-byte K steps of P V
+  static constexpr int kSubElems = 128 / kElem;        // elements per 128-byte group
+  static constexpr int kKStages = (F8 || D == 64) ? 4 : 2;
+  static constexpr int kVStages = kKStages;
   static_assert(kKStages <= kMaxStages && kVStages <= kMaxStages, "barrier slots");
   static constexpr int kOffQ = 0;
   static constexpr int kOffStg = kTileBytes;  // O staging tile
-  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffK = kOffStg + kStgBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
   static constexpr int kOffMref = kOffBar + 8 * B_COUNT;  // [128] reference maxima
@@ -121,9 +137,10 @@ struct Layout {
   static constexpr int kOffMisc = kOffLsum + 4 * kBM * 4;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory");
-  // TMEM columns
-  static constexpr uint32_t kColS1 = 128, kColO = 256, kColQ = 256 + D, kColP = kColQ + D / 2;
-  static_assert(kColP + 64 <= 512, "TMEM columns");
+  // TMEM columns: S_0 | S_1 | O | Q | P (Q and P packed, 4 bytes per column)
+  static constexpr uint32_t kColS1 = 128, kColO = 256, kColQ = 256 + D;
+  static constexpr uint32_t kColP = kColQ + kKSteps * 8;
+  static_assert(kColP + kPvSteps * 8 <= 512, "TMEM columns");
 };
 struct FwdParams {
   float* lse;
@@ -135,6 +152,10 @@ struct FwdParams {
   unsigned int* status;
   unsigned long long limit_ns;
   int debug_skip;
+  // F8 only: block scales of the Q and K codes [BH, n_q], V amax [BH]
+  const float* q_scale;
+  const float* k_scale;
+  const float* v_amax;
 };
 
 // The work list every role of a CTA walks (G = grid size). No mask: item i
@@ -172,12 +193,13 @@ __device__ __forceinline__ int steps_of(int qt, int n_q) {
   return CAUSAL ? qt + 1 : n_q;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                 const FwdParams p) {
-  using L = Layout<D>;
+  static_assert(!F8 || D == 128, "the FP8 forward is built for d = 128");
+  using L = Layout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -253,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(BAR(B_Q_FULL), L::kTileBytes);
         for (int c = 0; c < L::kSub; ++c)
-          tma_load_3d(sbase + L::kOffQ + c * L::kSubBytes, &tmQ, BAR(B_Q_FULL), c * 64, qt * kBM,
-                      bh);
+          tma_load_3d(sbase + L::kOffQ + c * L::kSubBytes, &tmQ, BAR(B_Q_FULL), c * L::kSubElems,
+                      qt * kBM, bh);
         ++q_issued;
         for (int j = 0; ok && j < n; ++j, ++kv) {
           const int s = kv % L::kKStages;
@@ -263,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(BAR(B_K_FULL + s), L::kTileBytes);
           for (int c = 0; c < L::kSub; ++c)
             tma_load_3d(sbase + L::kOffK + s * L::kTileBytes + c * L::kSubBytes, &tmK,
-                        BAR(B_K_FULL + s), c * 64, j * kBN, bh);
+                        BAR(B_K_FULL + s), c * L::kSubElems, j * kBN, bh);
           ++k_issued[s];
         }
       }
@@ -292,9 +314,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           mbar_arrive_expect_tx(BAR(B_V_FULL + s), L::kTileBytes);
-          for (int c = 0; c < L::kSub; ++c)
-            tma_load_3d(sbase + L::kOffV + s * L::kTileBytes + c * L::kSubBytes, &tmV,
-                        BAR(B_V_FULL + s), c * 64, j * kBN, bh);
+          if constexpr (F8) {
+            // V^T tile: d rows x 128 keys
+            tma_load_3d(sbase + L::kOffV + s * L::kTileBytes, &tmV, BAR(B_V_FULL + s), j * kBN, 0,
+                        bh);
+          } else {
+            for (int c = 0; c < L::kSub; ++c)
+              tma_load_3d(sbase + L::kOffV + s * L::kTileBytes + c * L::kSubBytes, &tmV,
+                          BAR(B_V_FULL + s), c * 64, j * kBN, bh);
+          }
           ++v_issued[s];
         }
       }
@@ -304,7 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == kQkMmaWarp && lane == 0) {
       // ------------------------------------------------------------------ Q K^T issuer
-      constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t idesc_qk =
+          F8 ? idesc_e4m3(kBM, kBN, false, false) : idesc_bf16(kBM, kBN, false, false);
       const uint32_t tQ = tmem + L::kColQ;
       bool ok = true;
       Walk<CAUSAL> w = walk_start<CAUSAL>();
@@ -317,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < L::kKSteps; ++kk) {
           const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
           tmem_cp_128x256b(tQ + kk * 8, sdesc_sw128(sbase + L::kOffQ + off, 16, 1024));
         }
@@ -336,10 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t kb = sbase + L::kOffK + s * L::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < L::kKSteps; ++kk) {
             const uint32_t off = (kk >> 2) * L::kSubBytes + (kk & 3) * 32;
-            mma_ts(tmem + (b ? L::kColS1 : 0u), tQ + kk * 8, sdesc_sw128(kb + off, 16, 1024),
-                   idesc_qk, kk > 0 ? 1u : 0u);
+            if constexpr (F8)
+              mma_ts_f8(tmem + (b ? L::kColS1 : 0u), tQ + kk * 8, sdesc_sw128(kb + off, 16, 1024),
+                        idesc_qk, kk > 0 ? 1u : 0u);
+            else
+              mma_ts(tmem + (b ? L::kColS1 : 0u), tQ + kk * 8, sdesc_sw128(kb + off, 16, 1024),
+                     idesc_qk, kk > 0 ? 1u : 0u);
           }
           tc_commit(BAR(B_S_FULL + b));
           tc_commit(BAR(B_K_EMPTY + s));
@@ -350,7 +383,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_bounded(BAR(B_DRAIN + 0), 0, wc, 16, true);
     } else if (warp == kPvMmaWarp && lane == 0) {
       // ------------------------------------------------------------------ P V issuer
-      constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, false, true);
+      // bf16: V [keys, d] tile, MN-major B; F8: V^T [d, keys] tile, K-major B
+      constexpr uint32_t idesc_pv =
+          F8 ? idesc_e4m3(kBM, D, false, false) : idesc_bf16(kBM, D, false, true);
       const uint32_t tO = tmem + L::kColO, tP = tmem + L::kColP;
       bool ok = true;
       Walk<CAUSAL> w = walk_start<CAUSAL>();
@@ -371,9 +406,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t vb = sbase + L::kOffV + s * L::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tO, tP + kk * 8, sdesc_sw128(vb + kk * 16 * 128, L::kSubBytes, 1024), idesc_pv,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < L::kPvSteps; ++kk) {
+            if constexpr (F8)
+              mma_ts_f8(tO, tP + kk * 8, sdesc_sw128(vb + kk * 32, 16, 1024), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+            else
+              mma_ts(tO, tP + kk * 8, sdesc_sw128(vb + kk * 16 * 128, L::kSubBytes, 1024), idesc_pv,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+          }
           tc_commit(BAR(B_P_EMPTY + (g & 1)));
           tc_commit(BAR(B_V_EMPTY + s));
           if (j + 1 == n) tc_commit(BAR(B_O_FULL + (g & 1)));  // group g % 2 finishes the unit
@@ -397,8 +437,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + L::kColO;
     const uint32_t tP = tmem + lane_base + L::kColP;
     const bool store_thread = (warp & 3) == 0 && lane == 0;
-    const float c = p.scale_log2;
-    const uint64_t c2 = f2_pack(c, c);
     bool ok = true;
     bool store_pending = false;  // this group's last O store is not yet confirmed read
     Walk<CAUSAL> w = walk_start<CAUSAL>();
@@ -407,6 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = steps_of<CAUSAL>(qt, p.n_q);
       const int row = qt * kBM + r;
       const bool final_group = ((g + n - 1) & 1) == grp;
+      // scores -> log2 units: scale * log2(e), times the Q and K block scales for F8
+      const float cq = F8 ? p.scale_log2 * p.q_scale[size_t(bh) * p.n_q + qt] : p.scale_log2;
       float m_ref = -INFINITY, l_part = 0.f;
       for (int j = 0; j < n; ++j, ++g) {
         if ((g & 1) != grp) continue;
@@ -421,6 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // S(g): this group loaded S(g-2) itself, and Q K^T(g+2) needs this
         // step's S_FREE, so the wait is exact
+        const float c = F8 ? cq * p.k_scale[size_t(bh) * p.n_q + j] : cq;
+        const uint64_t c2 = f2_pack(c, c);
         ok = wait_bounded(BAR(B_S_FULL + (g & 1)), (g >> 1) & 1, wc, 20);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -500,10 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(B_DEC + (g & 1)));
         // P = 2^(s c - m_ref) by one paired FMA per two columns and MUFU ex2,
-        // row sum by paired adds, packed to bf16 in registers
+        // row sum by paired adds, packed to bf16 (e4m3 for F8) in registers
         const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
         uint64_t sum_a = f2_pack(0.f, 0.f), sum_b = sum_a;
-        uint32_t pk[64];
+        uint32_t pk[L::kPvSteps * 8];
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           float x0, x1;
@@ -513,13 +555,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             sum_b = f2_add(sum_b, f2_pack(p0, p1));
           else
             sum_a = f2_add(sum_a, f2_pack(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
+          if constexpr (F8) {
+            const uint32_t h = pack_e4m3x2(p0, p1);
+            pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
+          } else {
+            pk[i] = pack_bf16x2(p0, p1);
+          }
         }
         // P(g) over P(g-1) once P V(g-1) has read it
         ok = wait_pv_prev();
         if (!ok) break;
         tc_fence_after();
-        tmem_st64(tP, pk);
+        if constexpr (F8) {
+          tmem_st32(tP, pk);
+        } else {
+          tmem_st64(tP, pk);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -574,7 +625,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row < p.N) p.lse[size_t(bh) * p.N + row] = (m_ref + lg2_approx(l)) * kLn2;
       // O = O~ / l as bf16 into the staging tile (128-byte swizzle, the layout
       // of the tensor map), then TMA stores; rows past N fall outside the tensor
-      const float inv_l = 1.0f / l;
+      float inv_l = 1.0f / l;
+      if constexpr (F8) {
+        const float va = p.v_amax[bh];
+        inv_l *= va > 0.f ? __fdiv_rn(va, 448.0f) : 1.0f;  // the V codes' scale
+      }
       uint8_t* stg = smem + L::kOffStg + r * 128;
 #pragma unroll
       for (int k16 = 0; k16 < D / 8; ++k16) {
@@ -597,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // STG_READY: the previous unit's phase completed before its store,
         // which we waited for above; the next needs our store
         if (wait_bounded(BAR(B_STG_READY), u & 1, wc, 26)) {
-          for (int gs = 0; gs < L::kSub; ++gs)
+          for (int gs = 0; gs < L::kStgBytes / L::kSubBytes; ++gs)
             tma_store_3d(&tmO, sbase + L::kOffStg + gs * L::kSubBytes, gs * 64, qt * kBM, bh);
           bulk_commit_group();
         }
@@ -614,11 +669,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F8 = false>
 fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                   const CUtensorMap& mo, const FwdParams& p, const LaunchCtx& ctx) {
-  auto kern = fwd_kernel<D, CAUSAL>;
-  const int smem = Layout<D>::kSmemBytes;
+  auto kern = fwd_kernel<D, CAUSAL, F8>;
+  const int smem = Layout<D, F8>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fwd)");
   // the setmaxnreg split is sized for exactly kRegsAtLaunch registers per
@@ -649,10 +704,10 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   const uint64_t BH = uint64_t(B) * uint64_t(H);
   CUtensorMap mq, mk, mv, mo;
   fa_status st;
-  if ((st = make_tmap_3d(&mq, q, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&mk, k, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&mv, v, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
-  if ((st = make_tmap_3d(&mo, o, true, d, N, BH, 64, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mq, q, 2, d, N, BH, 64, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mk, k, 2, d, N, BH, 64, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mv, v, 2, d, N, BH, 64, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mo, o, 2, d, N, BH, 64, 128, 128)) != FA_OK) return st;
   FwdParams p;
   p.lse = lse;
   p.N = N;
@@ -663,11 +718,44 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load == KID_FWD;
+  p.q_scale = p.k_scale = p.v_amax = nullptr;
   if (causal)
     return d == 128 ? launch<128, true>(mq, mk, mv, mo, p, ctx)
                     : launch<64, true>(mq, mk, mv, mo, p, ctx);
   return d == 128 ? launch<128, false>(mq, mk, mv, mo, p, ctx)
                   : launch<64, false>(mq, mk, mv, mo, p, ctx);
+}
+
+fa_status launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* q_scale,
+                         const float* k_scale, const float* v_amax, void* o, float* lse, int B,
+                         int H, int N, int d, float scale, bool causal, const LaunchCtx& ctx) {
+  const uint64_t BH = uint64_t(B) * uint64_t(H);
+  const uint64_t n_vt = uint64_t(fp8_vt_keys(N));
+  CUtensorMap mq, mk, mv, mo;
+  fa_status st;
+  if ((st = make_tmap_3d(&mq, q8, 1, d, N, BH, 128, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mk, k8, 1, d, N, BH, 128, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mv, vt8, 1, n_vt, d, BH, 128, 128, 128)) != FA_OK) return st;
+  if ((st = make_tmap_3d(&mo, o, 2, d, N, BH, 64, 128, 128)) != FA_OK) return st;
+  FwdParams p;
+  p.lse = lse;
+  p.N = N;
+  p.BH = int(BH);
+  p.n_q = (N + kBM - 1) / kBM;
+  p.num_items = p.BH * p.n_q;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = ctx.status_word;
+  p.limit_ns = ctx.wait_limit_ns;
+  p.debug_skip = ctx.debug_skip_load == KID_FWD;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_amax = v_amax;
+  if (d != 128) {
+    set_last_error("the FP8 forward needs d = 128 (got %d)", d);
+    return FA_ERR_UNSUPPORTED;
+  }
+  return causal ? launch<128, true, true>(mq, mk, mv, mo, p, ctx)
+                : launch<128, false, true>(mq, mk, mv, mo, p, ctx);
 }
 
 }  // namespace fa

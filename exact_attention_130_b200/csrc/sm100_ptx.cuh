@@ -228,6 +228,20 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem], 8-bit floating-point operands (.kind::f8f6f4;
+// the formats are in the instruction descriptor, K = 32 per instruction)
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // shared memory -> tensor memory: 128 rows x 256 bits (16 bf16 per row, the
 // K slice of one MMA step of an operand described by s_desc) into TMEM lanes
 // 0-127, 8 columns from taddr. Runs in order with this thread's later
@@ -243,6 +257,14 @@ __device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t s_desc
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t(N) >> 3) << 17) | ((uint32_t(M) >> 4) << 24);
+}
+
+// Instruction descriptor of tcgen05.mma .kind::f8f6f4 with e4m3 A and B
+// (format code 0 in [7,10) and [10,13)) and an fp32 accumulator; the other
+// fields as in idesc_bf16.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t(N) >> 3) << 17) | ((uint32_t(M) >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle. Bits: [0,14) start
@@ -347,6 +369,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// two fp32 -> two e4m3 codes (round to nearest even, saturating to +-448);
+// `lo` in the low byte
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return uint32_t(r);
 }
 // two fp32 of a packed pair -> bf16x2 (round to nearest even), .x in the low half
 __device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) {

@@ -101,6 +101,59 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o,
                      int causal, cudaStream_t stream);
 
 /*
+ * FP8 forward with incoherent processing ("FlashAttention-3 (TR)", section
+ * "FlashAttention-3'un Teknik Yenilikleri", item 3: Q and K multiplied by a
+ * random orthogonal matrix before FP8 quantisation, which spreads outliers
+ * and cancels in Q K^T; "Bellek Duvarinin Fizigi", section
+ * "FlashAttention-2, -3 ve -4: Utilizasyon Savasi": block-wise scaling and
+ * random signs). Two calls: fa_fp8_prepare makes the e4m3 operands once,
+ * fa_fwd_fp8 runs attention on them. d = 128 only (else FA_ERR_UNSUPPORTED).
+ *
+ * fa_fp8_vt_keys -- keys per row of the transposed V codes: N rounded up
+ * to a multiple of 16 (0 for N < 1).
+ */
+int fa_fp8_vt_keys(int N);
+
+/*
+ * fa_fp8_prepare -- rotation and e4m3 quantisation.
+ *   q, k, v  : bf16 [B, H, N, 128]          (input, device)
+ *   signs    : fp32 [128] or NULL            (input, device; only the sign
+ *              of each entry is used; NULL = no rotation)
+ *   q8, k8   : e4m3 codes [B, H, N, 128]     (output, device, uint8)
+ *   vt8      : e4m3 codes [B, H, 128, fa_fp8_vt_keys(N)] (output; V
+ *              transposed, zero codes past N)
+ *   q_scale, k_scale : fp32 [B, H, ceil(N/128)] (output) one scale per
+ *              128-row block; q_scale includes the rotation's 1/128
+ *   v_amax   : fp32 [B, H] (output) max |v| of each head; V's scale is
+ *              v_amax / 448 (1 when v_amax is 0)
+ *   B*H <= 65535. Rotation: x * sign(signs) times the unnormalised
+ *   Sylvester Hadamard matrix, as fp32 butterflies of stride 1, 2, ..., 64
+ *   (pair (i, i+h) -> (x_i + x_{i+h}, x_i - x_{i+h})). Block scale
+ *   s = max|x| / 448 (fp32 division; 1 for a zero block); code =
+ *   e4m3(x / s), nearest even, saturating. The codes are reproducible bit
+ *   for bit. Pointers 16-byte aligned except signs (4). Allocates nothing.
+ */
+fa_status fa_fp8_prepare(const void* q, const void* k, const void* v,
+                         const float* signs, int B, int H, int N, int d,
+                         void* q8, void* k8, void* vt8, float* q_scale,
+                         float* k_scale, float* v_amax, cudaStream_t stream);
+
+/*
+ * fa_fwd_fp8 -- attention forward on fa_fp8_prepare's operands.
+ *   q8, k8, vt8, q_scale, k_scale, v_amax : as written by fa_fp8_prepare
+ *   o   : bf16 [B, H, N, 128] (output)   lse : fp32 [B, H, N] (output)
+ *   scale, causal : as for fa_fwd (scale applies to the original Q K^T)
+ * Both products run on the tensor cores in e4m3 with fp32 accumulation;
+ * P~ is rounded to e4m3 before P V, the row sums stay fp32. Result: the
+ * attention of the dequantised operands, up to that rounding of P~.
+ */
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* vt8,
+                     const float* q_scale, const float* k_scale,
+                     const float* v_amax, void* o, float* lse, int B, int H,
+                     int N, int d, float scale, int causal,
+                     cudaStream_t stream);
+
+/*
  * fa_bwd_workspace_size -- bytes of scratch fa_bwd needs: two fp32 vectors
  * [B, H, Np] (the saved LSE in base 2, and D = rowsum(dO * O), in the forms
  * the kernels add) and two bf16 arrays [B, H, Np, 16] (-L/scale and -D, each
@@ -266,8 +319,9 @@ void fa_debug_skip_load(int kernel_id);
  * k in [0, capacity), the number of launches (launches[k]) and their summed
  * device time in milliseconds (total_ms[k]). Kernel ids: 1 forward (bf16),
  * 2 forward (fp32), 3 backward preprocess, 4 backward dK/dV, 5 backward
- * dQ, 6 decode split, 7 decode merge (8 is not used).
- * Returns the number of ids (9), or -1 if a CUDA call failed. Not thread-safe against concurrent
+ * dQ, 6 decode split, 7 decode merge, 9 FP8 preparation (8 is not used;
+ * the FP8 forward reports as 1).
+ * Returns the number of ids (10), or -1 if a CUDA call failed. Not thread-safe against concurrent
  * begin/end pairs; launches from several threads are recorded.
  */
 void fa_profile_begin(void);

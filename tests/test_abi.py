@@ -13,6 +13,7 @@ EXPECTED = {
     "fa_decode_workspace_size", "fa_decode_splitkv", "fa_device_status",
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_profile_begin",
     "fa_profile_end", "fa_decode_splitkv_static", "fa_decode_paged",
+    "fa_fp8_vt_keys", "fa_fp8_prepare", "fa_fwd_fp8",
 }
 
 
@@ -37,7 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     for code, name in fa.STATUS.items():
         assert lib.fa_status_string(code).decode() == name
-    assert lib.fa_abi_version() == 101
+    assert lib.fa_abi_version() == 102
 
 
 def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=8, d=64,
@@ -95,6 +96,31 @@ def test_paged_decode_argument_errors(lib):
     assert _paged(lib, d=96) == 2
     assert _paged(lib, ws_bytes=8) == 4           # workspace too small
     assert _paged(lib, max_pages=1 << 20, page=4096) == 1   # positions overflow
+
+
+def test_fp8_argument_errors(lib):
+    P = ctypes.c_void_p
+
+    def prep(signs=None, B=1, H=1, N=8, d=128, q8=16):
+        return lib.fa_fp8_prepare(P(16), P(16), P(16), P(signs) if signs else None, B, H, N, d,
+                                  P(q8), P(16), P(16), P(16), P(16), P(16), None)
+
+    def fwd(d=128, N=8, causal=0, scale=0.125, vt8=16):
+        return lib.fa_fwd_fp8(P(16), P(16), P(vt8), P(16), P(16), P(16), P(16), P(16), 1, 1, N, d,
+                              scale, causal, None)
+
+    assert prep(d=64) == 2                         # FP8 path: d = 128 only
+    assert prep(q8=0) == 1
+    assert prep(q8=24) == 3
+    assert prep(signs=18) == 3                     # signs not 4-byte aligned
+    assert prep(B=300, H=300) == 1                 # B*H > 65535
+    assert prep(N=0) == 1
+    assert fwd(d=64) == 2
+    assert fwd(vt8=0) == 1
+    assert fwd(causal=3) == 1
+    assert fwd(scale=0.0) == 1
+    assert lib.fa_fp8_vt_keys(1) == 16 and lib.fa_fp8_vt_keys(32) == 32
+    assert lib.fa_fp8_vt_keys(1000) == 1008 and lib.fa_fp8_vt_keys(0) == 0
 
 
 def test_workspace_sizes(lib):

@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     # single-kernel mode, for profiler captures (prints timings, no bench line)
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the FP8 forward and paged decode measured after the step")
     ap.add_argument("--kernel", choices=["fwd", "fwd_fp8", "fp8_prep", "bwd", "decode", "decode_paged"],
                     default=None)
     ap.add_argument("--hkv", type=int, default=8, help="KV heads of --kernel decode_paged")
@@ -420,6 +422,8 @@ def run_ours(args, world, rank, local):
                "pipelining": "host-to-device copies of step i+1, kernels of step i and device-to-host "
                              "copies of step i-1 on three streams, double-buffered"}
 
+    next_rows = None if args.no_next_rows else measure_next_rows(fa, torch, dev, flush, peaks)
+
     st, word = fa.fa_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} ({word:#x}) after timing")
@@ -455,6 +459,7 @@ def run_ours(args, world, rank, local):
         "clocks": sampler.summary(),
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "next_rows": next_rows,
         "impl": "ours",
     }
     if rank == 0:
@@ -462,6 +467,72 @@ def run_ours(args, world, rank, local):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def measure_next_rows(fa, torch, dev, flush, peaks, iters=8):
+    """Rows beyond the headline step, timed on their own after it (not part
+    of `value`): the FP8 forward on the prefill inputs (rotated, e4m3), and
+    the paged grouped-query decode. Median of `iters` launches, L2 flushed
+    before each."""
+    import statistics
+
+    def med_ms(fn):
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    B, H, N, d = dev["q"].shape
+    g = torch.Generator(device="cuda").manual_seed(20264)
+    signs = torch.where(torch.rand(d, device="cuda", generator=g) < 0.5, -1.0, 1.0)
+    prep = fa.fa_fp8_prepare(dev["q"], dev["k"], dev["v"], signs)
+    o = torch.empty_like(dev["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    rows = {"fwd_fp8": {
+        "workload": f"prefill B={B} H={H} N={N} d={d}, Q and K rotated (random signs x Hadamard), "
+                    "e4m3 with 128-row block scales, V e4m3 per head",
+        "prep_ms": round(med_ms(lambda: fa.fa_fp8_prepare(dev["q"], dev["k"], dev["v"], signs,
+                                                          out=prep)), 4),
+        "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+        "peak_source": "2 x " + peaks["source"] + " (nominal fp8 / bf16 dense ratio)"}}
+    for causal in (False, True):
+        ms = med_ms(lambda: fa.fa_fwd_fp8(prep, causal=causal, o=o, lse=lse))
+        tf = 4.0 * B * H * N * N * d / (2 if causal else 1) / (ms * 1e-3) / 1e12
+        key = "causal" if causal else "full"
+        rows["fwd_fp8"][f"ms_{key}"] = round(ms, 4)
+        rows["fwd_fp8"][f"tflops_{key}"] = round(tf, 1)
+        rows["fwd_fp8"][f"frac_{key}"] = round(tf / fp8_peak, 4)
+    del prep, o, lse
+
+    # paged decode: B=8, Hq=32, Hkv=8, d=128, 64-row pages in a shuffled
+    # order, lengths uniform in [16384, 32768]
+    Bq, Hq, Hkv, page, cap = 8, 32, 8, 64, 32768
+    lens = torch.randint(cap // 2, cap + 1, (Bq,), device="cuda", dtype=torch.int32, generator=g)
+    max_pages = cap // page
+    kp = torch.randn((Bq * max_pages, Hkv, page, d), device="cuda", dtype=torch.bfloat16, generator=g)
+    vp = torch.randn((Bq * max_pages, Hkv, page, d), device="cuda", dtype=torch.bfloat16, generator=g)
+    table = torch.randperm(Bq * max_pages, device="cuda", generator=g).to(torch.int32).view(Bq, max_pages)
+    qd = torch.randn((Bq, Hq, d), device="cuda", dtype=torch.bfloat16, generator=g)
+    ws = torch.empty(fa.fa_decode_workspace_size(Bq, Hq, cap, d, 0), dtype=torch.uint8, device="cuda")
+    od = torch.empty_like(qd)
+    lsed = torch.empty((Bq, Hq), dtype=torch.float32, device="cuda")
+    ms = med_ms(lambda: fa.fa_decode_paged(qd, kp, vp, table, lens, o=od, lse=lsed, workspace=ws))
+    kv_bytes = int(lens.sum().item()) * Hkv * d * 2 * 2
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    rows["decode_paged"] = {
+        "workload": f"B={Bq} Hq={Hq} Hkv={Hkv} d={d}, {page}-row pages shuffled, lengths uniform "
+                    f"[{cap // 2}, {cap}] (tensor-core kernel: 4 query heads per KV head)",
+        "us": round(ms * 1e3, 1), "gbs_unique_kv": round(gbs, 1), "peak": peaks["hbm_gbs"],
+        "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    del kp, vp
+    return rows
 
 
 def cpu_baseline(x, w, heads=16):

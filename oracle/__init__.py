@@ -26,3 +26,10 @@ from .fp8 import (  # noqa: F401
     hadamard_rotate_f32,
     quantize_blocks,
 )
+from .dropout_bias import (  # noqa: F401
+    attention_bwd_ex,
+    attention_fwd_ex,
+    dropout_keep,
+    keep_threshold,
+    philox4x32_10,
+)

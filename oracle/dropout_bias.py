@@ -26,10 +26,10 @@ Readings taken where the pages stop (listed with the design notes):
   (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)) with
   M0 = 0xD2511F53, M1 = 0xCD9E8D57, and the key bumped by the Weyl
   constants W0 = 0x9E3779B9, W1 = 0xBB67AE85 between rounds;
-* one call covers a 4 x 4 block of (query, key) pairs: counter =
-  (j // 4, i // 4, b * H + h, offset), key = (seed mod 2^32, seed >> 32);
-  the byte of pair (i, j) is byte j % 4 (least significant first) of output
-  word i % 4;
+* one call covers 16 consecutive keys of one query row: counter =
+  (j // 16, i, b * H + h, offset), key = (seed mod 2^32, seed >> 32); the
+  byte of pair (i, j) is byte (j % 16) % 4 (least significant first) of
+  output word (j % 16) // 4;
 * keep iff that byte < t with t = round(256 (1 - p)) (1 <= t <= 256), and
   a kept P is scaled by 256 / t, so the expected P is unchanged;
 * the bias is read as bias[b, h, i, j] with broadcasting over b and h
@@ -106,18 +106,18 @@ def keep_threshold(p_drop: float) -> int:
 def dropout_keep(B: int, H: int, N: int, seed: int, offset: int, p_drop: float):
     """Boolean keep mask [B, H, N (query), N (key)] and the scale 256 / t."""
     t = keep_threshold(p_drop)
-    nb = -(-N // 4)
+    nb = -(-N // 16)
     jb = np.arange(nb)[None, :]
-    ib = np.arange(nb)[:, None]
-    keep = np.empty((B, H, nb * 4, nb * 4), dtype=bool)
+    rows = np.arange(N)[:, None]
+    keep = np.empty((B, H, N, nb * 16), dtype=bool)
     for b in range(B):
         for h in range(H):
-            w = philox4x32_10(jb, ib, b * H + h, offset, seed & 0xFFFFFFFF, seed >> 32)
-            # bytes[ib, jb, word, byte] -> pair (4 ib + word, 4 jb + byte)
-            words = np.stack(w, axis=-1)                       # [nb, nb, 4]
+            w = philox4x32_10(jb, rows, b * H + h, offset, seed & 0xFFFFFFFF, seed >> 32)
+            # bytes[i, jb, word, byte] -> pair (i, 16 jb + 4 word + byte)
+            words = np.stack(w, axis=-1)                       # [N, nb, 4]
             by = (words[..., None] >> (8 * np.arange(4, dtype=np.uint32))) & 0xFF
-            keep[b, h] = (by < t).transpose(0, 2, 1, 3).reshape(nb * 4, nb * 4)
-    return keep[:, :, :N, :N], 256.0 / t
+            keep[b, h] = (by < t).reshape(N, nb * 16)
+    return keep[:, :, :, :N], 256.0 / t
 
 
 def _scores_ex(q, k, scale, causal, bias):

@@ -63,7 +63,8 @@ def parse_args():
     # single-kernel mode, for profiler captures (prints timings, no bench line)
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the FP8 forward and paged decode measured after the step")
-    ap.add_argument("--kernel", choices=["fwd", "fwd_fp8", "fp8_prep", "bwd", "decode", "decode_paged"],
+    ap.add_argument("--kernel", choices=["fwd", "fwd_ex", "fwd_fp8", "fp8_prep", "bwd", "bwd_ex",
+                                         "decode", "decode_paged"],
                     default=None)
     ap.add_argument("--hkv", type=int, default=8, help="KV heads of --kernel decode_paged")
     ap.add_argument("--page", type=int, default=64, help="page rows of --kernel decode_paged")
@@ -73,6 +74,9 @@ def parse_args():
     ap.add_argument("--N", type=int, default=2048)
     ap.add_argument("--d", type=int, default=128)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--p-drop", type=float, default=0.1, help="dropout of --kernel fwd_ex/bwd_ex")
+    ap.add_argument("--bias", type=int, default=1, help="--kernel fwd_ex/bwd_ex: 1 = a bf16 bias "
+                    "[1, H, N, N] (broadcast over the batch), 0 = none")
     return ap.parse_args()
 
 
@@ -666,6 +670,18 @@ def run_single_kernel(args):
         lens = torch.randint(N // 2, N + 1, (B,), device="cuda", dtype=torch.int32, generator=g)
         ws = torch.empty(fa.fa_decode_workspace_size(B, H, N, d, 0), dtype=torch.uint8, device="cuda")
         fn = lambda: fa.fa_decode_splitkv(q, kc, vc, lens, workspace=ws)  # noqa: E731
+    elif args.kernel in ("fwd_ex", "bwd_ex"):
+        q, k, v, do = rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d)
+        bias = rnd(1, H, N, N) if args.bias else None
+        ex = dict(causal=bool(args.causal), bias=bias, p_drop=args.p_drop, seed=1234, offset=0)
+        o, lse = fa.fa_fwd_ex(q, k, v, **ex)
+        if args.kernel == "fwd_ex":
+            fn = lambda: fa.fa_fwd_ex(q, k, v, o=o, lse=lse, **ex)  # noqa: E731
+        else:
+            ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+            fn = lambda: fa.fa_bwd_ex(q, k, v, o, lse, do, dq=dq, dk=dk, dv=dv,  # noqa: E731
+                                      workspace=ws, **ex)
     else:
         q, k, v, do = rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d)
         o, lse = fa.fa_fwd(q, k, v, causal=bool(args.causal))
@@ -687,7 +703,7 @@ def run_single_kernel(args):
         if args.kernel == "decode_paged":
             extra = (f" Hkv={args.hkv} page={args.page}: "
                      f"{kv_bytes / (a.elapsed_time(b) * 1e-3) / 1e9:.1f} GB/s of KV pages")
-        elif args.kernel in ("fwd", "fwd_fp8"):
+        elif args.kernel in ("fwd", "fwd_fp8", "fwd_ex"):
             fl = 4.0 * B * H * N * N * d / (2 if args.causal else 1)
             extra = f": {fl / (a.elapsed_time(b) * 1e-3) / 1e12:.1f} TFLOP/s"
         print(f"{args.kernel} B={B} H={H} N={N} d={d} causal={args.causal} "

@@ -6,7 +6,8 @@ memory and the current stream. There is no CPU fallback: if the library is
 missing, every call raises.
 
 Functions carry the C names:
-    fa_fwd, fa_fwd_f32, fa_fp8_prepare, fa_fwd_fp8, fa_fp8_vt_keys,
+    fa_fwd, fa_fwd_ex, fa_fwd_f32, fa_fp8_prepare, fa_fwd_fp8, fa_fp8_vt_keys,
+    fa_bwd_ex,
     fa_bwd, fa_bwd_workspace_size,
     fa_decode_splitkv, fa_decode_workspace_size,
     fa_device_status, fa_set_wait_limit, fa_debug_skip_load
@@ -20,7 +21,8 @@ import re
 
 __all__ = [
     "FAError", "library_path", "load_library", "exported_symbols",
-    "fa_fwd", "fa_fwd_f32", "fa_fp8_prepare", "fa_fwd_fp8", "fa_fp8_vt_keys",
+    "fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_f32", "fa_fp8_prepare", "fa_fwd_fp8",
+    "fa_fp8_vt_keys",
     "fa_bwd", "fa_bwd_workspace_size",
     "fa_decode_splitkv", "fa_decode_workspace_size", "fa_decode_splitkv_static",
     "fa_decode_paged",
@@ -60,6 +62,11 @@ _SIGNATURES = {
     "fa_abi_version": (_I, []),
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, ctypes.c_longlong,
+                       ctypes.c_longlong, _F, ctypes.c_ulonglong, ctypes.c_uint, _P]),
+    "fa_bwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P,
+                       ctypes.c_longlong, ctypes.c_longlong, _F, ctypes.c_ulonglong, ctypes.c_uint,
+                       _P, _S, _P]),
     "fa_fp8_vt_keys": (_I, [_I]),
     "fa_fp8_prepare": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
@@ -162,6 +169,68 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None,
     _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                       scale, int(bool(causal)), _stream(stream)))
     return o, lse
+
+
+def _bias_args(bias, B, H, N):
+    """(pointer, stride_b, stride_h) of a bf16 bias broadcastable to [B, H, N, N]."""
+    import torch
+    if bias is None:
+        return None, 0, 0
+    if bias.dtype != torch.bfloat16 or not bias.is_cuda:
+        raise TypeError("bias must be a bf16 CUDA tensor")
+    if bias.dim() != 4 or bias.shape[-2:] != (N, N) or bias.shape[0] not in (1, B) \
+            or bias.shape[1] not in (1, H):
+        raise ValueError("bias must have shape [B or 1, H or 1, N, N]")
+    if bias.stride(3) != 1 or bias.stride(2) != N:
+        raise ValueError("bias rows must be contiguous")
+    sb = bias.stride(0) if bias.shape[0] > 1 else 0
+    sh = bias.stride(1) if bias.shape[1] > 1 else 0
+    return _ptr(bias), sb, sh
+
+
+def fa_fwd_ex(q, k, v, causal: bool = False, scale: float | None = None, bias=None,
+              p_drop: float = 0.0, seed: int = 0, offset: int = 0, o=None, lse=None,
+              stream=None):
+    """fa_fwd with an additive bf16 bias [B|1, H|1, N, N] and dropout on P
+    (Philox4x32-10 keyed by ``seed``, sequence ``offset``)."""
+    import torch
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    bp, sb, sh = _bias_args(bias, B, H, N)
+    _check(lib.fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                         int(bool(causal)), bp, sb, sh, float(p_drop), int(seed), int(offset),
+                         _stream(stream)))
+    return o, lse
+
+
+def fa_bwd_ex(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, bias=None,
+              p_drop: float = 0.0, seed: int = 0, offset: int = 0, dq=None, dk=None, dv=None,
+              workspace=None, stream=None):
+    """fa_bwd for fa_fwd_ex (same bias, p_drop, seed and offset)."""
+    import torch
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    bp, sb, sh = _bias_args(bias, B, H, N)
+    _check(lib.fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                         _ptr(dk), _ptr(dv), B, H, N, d, scale, int(bool(causal)), bp, sb, sh,
+                         float(p_drop), int(seed), int(offset), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dq, dk, dv
 
 
 def fa_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None,

@@ -27,6 +27,25 @@
 //                 S = Q K^T, dP = dO V^T; dS = scale P (dP - D); dQ += dS K.
 // The scale is folded into dS before it is rounded to bf16.
 //
+// The EX instantiations add the bias and dropout options of the forward
+// ("FlashAttention'i Anlamak Bolum 1", 0.2; "Bellek Duvarinin Fizigi",
+// "Maskeleme ve Dropout": the backward regenerates the forward's dropout
+// mask from the same seed and offset instead of storing it). With the keep
+// factor z = keep * 256/t (0 for a dropped pair):
+//     P = exp(S + bias - L), dV = (P z)^T dO, dS = P (z dP - D),
+// and dQ, dK as before. The bias (an input, no gradient) is added to the raw
+// scores before the exponential: in the dQ kernel a thread reads its query
+// row (16-byte loads when possible), in the dK/dV kernel a warp reads 32
+// consecutive keys of one query row per load. The keep bits come from the
+// same Philox4x32-10 calls as the forward (counter (key / 16, query, b H + h,
+// offset)): a dQ thread makes four calls for its 64 keys; in the dK/dV
+// kernel, whose threads own keys, each lane makes four calls for
+// (query, 16 keys) pairs of its warp, reduces them to 16 keep bits, and a
+// warp shuffle per query hands every lane its bit. The dK/dV kernel's TMEM
+// holds dP^T - D (D enters through the extension step), so there
+// scale (z dP - D) = z u + (1 - z)(-scale D) with u = scale (dP - D), and
+// -scale D is read per query column.
+//
 // Splitting dQ from dK/dV recomputes S and dP once more (7 tensor-core GEMMs
 // instead of 5) but needs no atomics and gives deterministic results. Both
 // kernels use 128-wide blocks, so every MMA is M = 128, N = 128 (the full-rate
@@ -111,7 +130,27 @@ struct BwdParams {
   unsigned int* status;
   unsigned long long limit_ns;
   int debug_skip;  // test hook: kernel id whose CTA 0 leaves out one load (0: none)
+  // EX only: bias (bf16, element strides over b and h, rows of N) and dropout
+  const uint16_t* bias;
+  long long bias_sb, bias_sh;
+  int H;
+  int bias_vec;  // rows and strides are multiples of 8 elements: 16-byte loads
+  float inv_scale;
+  uint32_t seed_lo, seed_hi, rng_offset;
+  int keep_t;    // keep iff byte < keep_t; 256 = no dropout
+  float keep_scale;
 };
+
+__device__ __forceinline__ const uint16_t* bias_head(const BwdParams& p, int bh) {
+  const int b = bh / p.H, h = bh - b * p.H;
+  return p.bias + b * p.bias_sb + h * p.bias_sh;
+}
+
+// keep bits of query q for keys 16 kb .. 16 kb + 15 (bit e: key 16 kb + e)
+__device__ __forceinline__ uint32_t keep16(const BwdParams& p, int bh, int q, int kb) {
+  return keep_bits16(make_uint4(uint32_t(kb), uint32_t(q), uint32_t(bh), p.rng_offset), p.seed_lo,
+                     p.seed_hi, uint32_t(p.keep_t));
+}
 
 __device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
@@ -380,6 +419,33 @@ __device__ __forceinline__ void write_ds_half(uint32_t t_dp, const uint64_t (&pr
   }
 }
 
+// write_ds_half with the dropout factor: column i of dP is scaled by szk
+// when bit i of keep64 is set, else by 0
+template <typename NsdFn>
+__device__ __forceinline__ void write_ds_half_z(uint32_t t_dp, const uint64_t (&pr2)[kHalfCols / 2],
+                                                uint64_t keep64, float szk, NsdFn nsd4) {
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    uint32_t dr[32];
+    tmem_ld32_wait(t_dp + ch * 32, dr);
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = ch * 32 + 4 * j;
+      const float4 n = nsd4(ch * 8 + j);
+      const float z0 = (keep64 >> c) & 1 ? szk : 0.f, z1 = (keep64 >> (c + 1)) & 1 ? szk : 0.f;
+      const float z2 = (keep64 >> (c + 2)) & 1 ? szk : 0.f, z3 = (keep64 >> (c + 3)) & 1 ? szk : 0.f;
+      const uint64_t t0 = f2_fma(f2_pack(__uint_as_float(dr[4 * j]), __uint_as_float(dr[4 * j + 1])),
+                                 f2_pack(z0, z1), f2_pack(n.x, n.y));
+      const uint64_t t1 = f2_fma(f2_pack(__uint_as_float(dr[4 * j + 2]), __uint_as_float(dr[4 * j + 3])),
+                                 f2_pack(z2, z3), f2_pack(n.z, n.w));
+      pk[2 * j] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j], t0));
+      pk[2 * j + 1] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j + 1], t1));
+    }
+    tmem_st16(t_dp + ch * 16, pk);
+  }
+}
+
 // P for this warp's 64 columns of a row: 2^(s c + nl2) in pairs, where nl2 is
 // minus the base-2 LSE of the query (the row's one value, or a per-column
 // vector); nl4(j) gives it for local columns 4j..4j+3. Columns with
@@ -429,7 +495,7 @@ __device__ __forceinline__ bool bwd_item(const BwdParams& p, int round, int& bh,
   return true;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool EX>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -648,11 +714,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = CAUSAL ? jt : 0, n_blk = blocks_of(jt);
       const int key = jt * kTile + r;
       for (int it = 0; it < n_blk; ++it, ++g) {
+        const int q0 = (i0 + it) * kTile;
+        // EX dropout: keep bit c of this key for query q0 + 64 half + c. Lane L
+        // computes the calls for queries qb + 16 rnd + L/2, key block of
+        // keys key - lane + 16 (L % 2); lane src = 2 qq + lane/16 holds the bits
+        // of query qq of the round for this lane's 16-key block.
+        uint64_t keep64 = ~0ull;
+        if constexpr (EX) {
+          if (p.keep_t < 256) {
+            keep64 = 0;
+            const int qb = q0 + half * kHalfCols;
+            const int kb0 = (key - lane) / 16;
+#pragma unroll
+            for (int rnd = 0; rnd < 4; ++rnd) {
+              const uint32_t m16 = keep16(p, bh, qb + 16 * rnd + (lane >> 1), kb0 + (lane & 1));
+#pragma unroll
+              for (int qq = 0; qq < 16; ++qq) {
+                const uint32_t bits = __shfl_sync(0xffffffffu, m16, 2 * qq + (lane >> 4));
+                keep64 |= uint64_t((bits >> (lane & 15)) & 1u) << (16 * rnd + qq);
+              }
+            }
+          }
+        }
+        // EX bias: bias[q][key] of the 64 query columns, loaded before the
+        // wait for S^T so that the loads overlap it (lanes read 32
+        // consecutive keys of one row per load)
+        uint32_t bpre[kHalfCols];
+        const bool bias_on = EX && p.bias != nullptr && key < p.N;
+        if constexpr (EX) {
+          if (bias_on) {
+            const uint16_t* bcol = bias_head(p, bh) + key;
+            const int qb = q0 + half * kHalfCols;
+#pragma unroll
+            for (int c = 0; c < kHalfCols; ++c)
+              bpre[c] = qb + c < p.N ? uint32_t(bcol[size_t(qb + c) * p.N]) : 0u;
+          }
+        }
         ok = wait_bounded(BAR(B_S_FULL), g & 1, wc, 20);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const int q0 = (i0 + it) * kTile;
         // phase 1: read S^T - L/scale (after which the next S^T may overwrite
         // it) and form P^T = 2^(scale log2e (s - L_q/scale)) in registers. Only
         // the first block under the causal mask hides queries (q < key). Rows
@@ -665,6 +766,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(BAR(B_PHASE1));
+          if constexpr (EX) {
+            if (bias_on) {
+#pragma unroll
+              for (int c = 0; c < kHalfCols; ++c)
+                sr[c] = __float_as_uint(fmaf(bf16f(bpre[c]), p.inv_scale, __uint_as_float(sr[c])));
+            }
+          }
           auto nl4 = [&](int) { return zero4; };
           if (CAUSAL && it == 0) {
             const int qlim = key - q0 - half * kHalfCols;  // local columns below qlim are hidden
@@ -682,21 +790,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         {
           uint32_t pk_ds[kHalfCols / 2];
+          const bool drop = EX && p.keep_t < 256;
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
             uint32_t dr[32];
             tmem_ld32_wait(tDP + ch * 32, dr);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const uint64_t t0 = f2_mul(f2_pack(__uint_as_float(dr[4 * j]), __uint_as_float(dr[4 * j + 1])), scale2);
-              const uint64_t t1 = f2_mul(f2_pack(__uint_as_float(dr[4 * j + 2]), __uint_as_float(dr[4 * j + 3])), scale2);
+              uint64_t t0 = f2_mul(f2_pack(__uint_as_float(dr[4 * j]), __uint_as_float(dr[4 * j + 1])), scale2);
+              uint64_t t1 = f2_mul(f2_pack(__uint_as_float(dr[4 * j + 2]), __uint_as_float(dr[4 * j + 3])), scale2);
+              if constexpr (EX) {
+                if (drop) {
+                  // z u + (1 - z)(-scale D_q), u = scale (dP - D)
+                  const int c0 = ch * 32 + 4 * j;
+                  const float* nsd = p.dvec + size_t(bh) * p.Np + q0 + half * kHalfCols + c0;
+                  float u[4];
+                  f2_unpack(t0, u[0], u[1]);
+                  f2_unpack(t1, u[2], u[3]);
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const float z = (keep64 >> (c0 + e)) & 1 ? p.keep_scale : 0.f;
+                    u[e] = fmaf(z, u[e], (1.f - z) * nsd[e]);
+                  }
+                  t0 = f2_pack(u[0], u[1]);
+                  t1 = f2_pack(u[2], u[3]);
+                }
+              }
               pk_ds[ch * 16 + 2 * j] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j], t0));
               pk_ds[ch * 16 + 2 * j + 1] = f2_to_bf16x2(f2_mul(pr2[ch * 16 + 2 * j + 1], t1));
             }
           }
           uint32_t pk_p[kHalfCols / 2];
 #pragma unroll
-          for (int i = 0; i < kHalfCols / 2; ++i) pk_p[i] = f2_to_bf16x2(pr2[i]);
+          for (int i = 0; i < kHalfCols / 2; ++i) {
+            if constexpr (EX) {
+              if (drop) {
+                float a, b;
+                f2_unpack(pr2[i], a, b);
+                a = (keep64 >> (2 * i)) & 1 ? a * p.keep_scale : 0.f;
+                b = (keep64 >> (2 * i + 1)) & 1 ? b * p.keep_scale : 0.f;
+                pk_p[i] = pack_bf16x2(a, b);
+                continue;
+              }
+            }
+            pk_p[i] = f2_to_bf16x2(pr2[i]);
+          }
           tmem_st32(tDP, pk_p);
           tmem_st32(tDP + 32, pk_ds);
         }
@@ -739,7 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // --------------------------------------------------------------------------
 // 3. dQ: query-tile-outer
 // --------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool EX>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -936,17 +1074,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4 nl2q4 = make_float4(nl2q, nl2q, nl2q, nl2q);
       const float4 nsdq4 = make_float4(nsdq, nsdq, nsdq, nsdq);
       for (int it = 0; it < n_blk; ++it, ++g) {
+        const int k0 = it * kTile;
+        // EX dropout: keep bit c of this query for key k0 + 64 half + c
+        uint64_t keep64 = ~0ull;
+        if constexpr (EX) {
+          if (p.keep_t < 256) {
+            const int kb = (k0 + half * kHalfCols) / 16;
+            keep64 = uint64_t(keep16(p, bh, q, kb)) | (uint64_t(keep16(p, bh, q, kb + 1)) << 16) |
+                     (uint64_t(keep16(p, bh, q, kb + 2)) << 32) |
+                     (uint64_t(keep16(p, bh, q, kb + 3)) << 48);
+          }
+        }
+        // EX bias (16-byte rows): this half's 64 keys of row q, loaded before
+        // the wait for S so that the loads overlap it
+        uint4 bq[kHalfCols / 8];
+        const bool bias_pf = EX && p.bias != nullptr && p.bias_vec && q < p.N;
+        if constexpr (EX) {
+          if (bias_pf) {
+            const int kb0 = k0 + half * kHalfCols;
+            const uint16_t* brow = bias_head(p, bh) + size_t(q) * p.N + kb0;
+            const int n = min(kHalfCols, p.N - kb0);
+#pragma unroll
+            for (int c8 = 0; c8 < kHalfCols / 8; ++c8)
+              bq[c8] = 8 * c8 < n ? *reinterpret_cast<const uint4*>(brow + 8 * c8) : make_uint4(0, 0, 0, 0);
+          }
+        }
         ok = wait_bounded(BAR(B_S_FULL), g & 1, wc, 20);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const int k0 = it * kTile;
         // phase 1: read S (then the MMA may overwrite it) and form P
         uint32_t sr[kHalfCols];
         tmem_ld64_wait(tS, sr);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(B_PHASE1));
+        if constexpr (EX) {
+          // bias[q][keys] / scale for this half's 64 keys
+          if (p.bias != nullptr && q < p.N) {
+            const int kb0 = k0 + half * kHalfCols;
+            const uint16_t* brow = bias_head(p, bh) + size_t(q) * p.N + kb0;
+            const int n = min(kHalfCols, p.N - kb0);
+            if (bias_pf) {
+#pragma unroll
+              for (int c8 = 0; c8 < kHalfCols / 8; ++c8) {
+                if (8 * c8 < n) {
+                  const uint4 u = bq[c8];
+                  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    sr[8 * c8 + 2 * e] = __float_as_uint(
+                        fmaf(bf16f(w[e] & 0xffffu), p.inv_scale, __uint_as_float(sr[8 * c8 + 2 * e])));
+                    sr[8 * c8 + 2 * e + 1] = __float_as_uint(
+                        fmaf(bf16f(w[e] >> 16), p.inv_scale, __uint_as_float(sr[8 * c8 + 2 * e + 1])));
+                  }
+                }
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < kHalfCols; ++c)
+                if (c < n)
+                  sr[c] = __float_as_uint(fmaf(bf16f(brow[c]), p.inv_scale, __uint_as_float(sr[c])));
+            }
+          }
+        }
         uint64_t pr2[kHalfCols / 2];
         auto nl4 = [&](int) { return nl2q4; };
         // keys past N, or (causal) past q, are hidden: only the last block has any
@@ -963,7 +1154,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        write_ds_half(tDP, pr2, scale2, [&](int) { return nsdq4; });
+        if constexpr (EX) {
+          if (p.keep_t < 256) {
+            // dS = P (scale z dP - scale D): the scale of each dP entry is scale z
+            const float szk = p.scale * p.keep_scale;
+            write_ds_half_z(tDP, pr2, keep64, szk, [&](int) { return nsdq4; });
+          } else {
+            write_ds_half(tDP, pr2, scale2, [&](int) { return nsdq4; });
+          }
+        } else {
+          write_ds_half(tDP, pr2, scale2, [&](int) { return nsdq4; });
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -1028,7 +1229,7 @@ fa_status launch_main(Kern kern, unsigned kid, int smem, unsigned grid, const CU
   return FA_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool EX>
 fa_status launch_all(const void* q, const void* k, const void* v, const void* dO, const BwdParams& p,
                      const LaunchCtx& ctx) {
   // maps 0-3: Q, dO, K, V; 4-5: extension rows; 6-7: outputs (dK, dV for the
@@ -1052,9 +1253,9 @@ fa_status launch_all(const void* q, const void* k, const void* v, const void* dO
   mq[7] = mq[6];
   // both kernels are persistent: one CTA per SM walks its items
   const unsigned grid_kv = grid < unsigned(ctx.num_sms) ? grid : unsigned(ctx.num_sms);
-  st = launch_main(bwd_dkdv_kernel<D, CAUSAL>, KID_BWD, smem, grid_kv, m, p, ctx, "bwd dK/dV kernel");
+  st = launch_main(bwd_dkdv_kernel<D, CAUSAL, EX>, KID_BWD, smem, grid_kv, m, p, ctx, "bwd dK/dV kernel");
   if (st != FA_OK) return st;
-  return launch_main(bwd_dq_kernel<D, CAUSAL>, KID_BWD_DQ, smem, grid_kv, mq, p, ctx, "bwd dQ kernel");
+  return launch_main(bwd_dq_kernel<D, CAUSAL, EX>, KID_BWD_DQ, smem, grid_kv, mq, p, ctx, "bwd dQ kernel");
 }
 
 }  // namespace
@@ -1068,7 +1269,8 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d) {
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                     float scale, bool causal, void* workspace, const LaunchCtx& ctx) {
+                     float scale, bool causal, void* workspace, const LaunchCtx& ctx,
+                     const FwdExtras* ex) {
   const int BH = B * H;
   BwdParams p;
   p.o = static_cast<const uint16_t*>(o);
@@ -1096,6 +1298,18 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load;
+  const bool use_ex = ex != nullptr && (ex->bias != nullptr || ex->keep_t < 256);
+  p.bias = use_ex ? static_cast<const uint16_t*>(ex->bias) : nullptr;
+  p.bias_sb = use_ex ? ex->bias_stride_b : 0;
+  p.bias_sh = use_ex ? ex->bias_stride_h : 0;
+  p.H = H;
+  p.bias_vec = (use_ex && N % 8 == 0 && p.bias_sb % 8 == 0 && p.bias_sh % 8 == 0) ? 1 : 0;
+  p.inv_scale = 1.0f / scale;
+  p.seed_lo = use_ex ? uint32_t(ex->seed) : 0u;
+  p.seed_hi = use_ex ? uint32_t(ex->seed >> 32) : 0u;
+  p.rng_offset = use_ex ? ex->offset : 0u;
+  p.keep_t = use_ex ? ex->keep_t : 256;
+  p.keep_scale = 256.0f / float(p.keep_t);
 
   {
     const long long rows_per_warp = (32 / (d / 8)) * kPreSteps;
@@ -1109,9 +1323,18 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "bwd preprocess launch");
   }
+  if (use_ex) {
+    if (d == 128)
+      return causal ? launch_all<128, true, true>(q, k, v, dO, p, ctx)
+                    : launch_all<128, false, true>(q, k, v, dO, p, ctx);
+    return causal ? launch_all<64, true, true>(q, k, v, dO, p, ctx)
+                  : launch_all<64, false, true>(q, k, v, dO, p, ctx);
+  }
   if (d == 128)
-    return causal ? launch_all<128, true>(q, k, v, dO, p, ctx) : launch_all<128, false>(q, k, v, dO, p, ctx);
-  return causal ? launch_all<64, true>(q, k, v, dO, p, ctx) : launch_all<64, false>(q, k, v, dO, p, ctx);
+    return causal ? launch_all<128, true, false>(q, k, v, dO, p, ctx)
+                  : launch_all<128, false, false>(q, k, v, dO, p, ctx);
+  return causal ? launch_all<64, true, false>(q, k, v, dO, p, ctx)
+                : launch_all<64, false, false>(q, k, v, dO, p, ctx);
 }
 
 }  // namespace fa

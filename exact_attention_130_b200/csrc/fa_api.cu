@@ -226,7 +226,7 @@ const char* fa_status_string(fa_status s) {
 
 const char* fa_last_error(void) { return t_last_error; }
 
-int fa_abi_version(void) { return 102; }
+int fa_abi_version(void) { return 103; }
 
 void fa_set_wait_limit(unsigned long long ns) {
   g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs);
@@ -245,6 +245,54 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
   ctx.debug_skip_load = g_debug_skip.exchange(0);
   return launch_fwd_bf16(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx);
+}
+
+// Validates the bias / dropout options shared by fa_fwd_ex and fa_bwd_ex.
+static fa_status make_extras(const void* bias, long long bias_stride_b, long long bias_stride_h,
+                             int B, int H, int N, float p_drop, unsigned long long seed,
+                             unsigned int offset, FwdExtras* ex) {
+  if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 15u) != 0)
+    return invalid(FA_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  if (bias_stride_b < 0 || bias_stride_h < 0)
+    return invalid(FA_ERR_INVALID_ARG, "bias strides must be >= 0");
+  if (bias != nullptr) {
+    // the last element read: (B-1) sb + (H-1) sh + N*N - 1 must not overflow
+    const long double last = (long double)(B - 1) * bias_stride_b +
+                             (long double)(H - 1) * bias_stride_h + (long double)N * N;
+    if (last > 9.0e18L) return invalid(FA_ERR_INVALID_ARG, "bias extent overflows");
+  }
+  if (!(p_drop >= 0.f && p_drop < 1.f))
+    return invalid(FA_ERR_INVALID_ARG, "dropout probability must be in [0, 1) (got %g)",
+                   (double)p_drop);
+  double t = std::nearbyint(256.0 * (1.0 - (double)p_drop));
+  if (t < 1.0) t = 1.0;
+  if (t > 256.0) t = 256.0;
+  ex->bias = bias;
+  ex->bias_stride_b = bias_stride_b;
+  ex->bias_stride_h = bias_stride_h;
+  ex->seed = seed;
+  ex->offset = offset;
+  ex->keep_t = int(t);
+  return FA_OK;
+}
+
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int N, int d, float scale, int causal, const void* bias,
+                    long long bias_stride_b, long long bias_stride_h, float p_drop,
+                    unsigned long long seed, unsigned int offset, cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, k, v, o, lse}, "fa_fwd_ex(q,k,v,o,lse)")) != FA_OK) return st;
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (causal != 0 && causal != 1) return invalid(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  FwdExtras ex;
+  if ((st = make_extras(bias, bias_stride_b, bias_stride_h, B, H, N, p_drop, seed, offset,
+                        &ex)) != FA_OK)
+    return st;
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  ctx.debug_skip_load = g_debug_skip.exchange(0);
+  return launch_fwd_bf16(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx, &ex);
 }
 
 fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B,
@@ -326,6 +374,35 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   ctx.debug_skip_load = g_debug_skip.exchange(0);
   return launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal != 0, workspace,
                     ctx);
+}
+
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                    float scale, int causal, const void* bias, long long bias_stride_b,
+                    long long bias_stride_h, float p_drop, unsigned long long seed,
+                    unsigned int offset, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv},
+                       "fa_bwd_ex(q,k,v,o,lse,dO,dq,dk,dv)")) != FA_OK)
+    return st;
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (causal != 0 && causal != 1) return invalid(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  FwdExtras ex;
+  if ((st = make_extras(bias, bias_stride_b, bias_stride_h, B, H, N, p_drop, seed, offset,
+                        &ex)) != FA_OK)
+    return st;
+  const size_t need = bwd_workspace_bytes(B, H, N, d);
+  if (workspace == nullptr || workspace_bytes < need)
+    return invalid(FA_ERR_WORKSPACE, "fa_bwd_ex needs %zu bytes of workspace (got %zu)", need,
+                   workspace ? workspace_bytes : size_t(0));
+  if (!aligned16(workspace)) return invalid(FA_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  ctx.debug_skip_load = g_debug_skip.exchange(0);
+  return launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal != 0, workspace,
+                    ctx, &ex);
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Lmax, int d, int num_splits) {

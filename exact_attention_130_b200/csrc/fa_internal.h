@@ -62,9 +62,19 @@ fa_status make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint6
                        uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows,
                        int swizzle_bytes);
 
+// Options of the bf16 forward and backward: an additive bias (bf16, rows
+// of N keys, element strides over batch and head, 0 = broadcast) and
+// dropout on P (keep iff the generator byte < keep_t, 1..256; 256 = off).
+struct FwdExtras {
+  const void* bias;
+  long long bias_stride_b, bias_stride_h;
+  unsigned long long seed;
+  uint32_t offset;
+  int keep_t;
+};
 fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int N, int d, float scale, bool causal,
-                          const LaunchCtx& ctx);
+                          const LaunchCtx& ctx, const FwdExtras* ex = nullptr);
 // Keys per row of the transposed FP8 V ([B, H, d, fp8_vt_keys(N)] codes):
 // N rounded up to 16, so that every row starts 16-byte aligned.
 inline int fp8_vt_keys(int N) { return (N + 15) & ~15; }
@@ -80,7 +90,7 @@ fa_status launch_fwd_f32(const float* q, const float* k, const float* v, float* 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
                      int H, int N, int d, float scale, bool causal, void* workspace,
-                     const LaunchCtx& ctx);
+                     const LaunchCtx& ctx, const FwdExtras* ex = nullptr);
 size_t bwd_workspace_bytes(int B, int H, int N, int d);
 int decode_num_chunks(int B, int H, int Lmax, int num_splits, int num_sms);
 size_t decode_workspace_bytes(int B, int H, int d, int chunks);

@@ -58,6 +58,21 @@
 // rounded to e4m3 (it is at most 2^8, the lazy-rescale bound, inside
 // e4m3's 448) while the row sum keeps the fp32 values; the epilogue
 // multiplies O~ by v_scale / l.
+//
+// The EX instantiation (bf16) adds the two options of "FlashAttention'i
+// Anlamak Bolum 1", 0.2 (S = Q K^T / sqrt(d) + B) and "Bellek Duvarinin
+// Fizigi", "Maskeleme ve Dropout" (dropout on P from a counter-based
+// generator driven by a seed and an offset, regenerated in the backward):
+//  * bias: each softmax thread adds bias[b, h, row, keys of the tile] / scale
+//    to its raw scores before the mask and the row maximum (16-byte loads
+//    when rows and strides allow, else 2-byte loads; prefetching them
+//    before the wait for S needs 64 more registers than the softmax has);
+//  * dropout: Philox4x32-10 with counter (key / 16, row, b H + h, offset)
+//    and key = the seed gives one byte per (row, key); the key is kept iff
+//    its byte < t, t = round(256 (1 - p)); the calls are made inside the
+//    exponential loop, one per 16 keys (forming the bits before the wait
+//    for S was slower: more live registers); the row sum uses the undropped
+//    P~, the P V operand P~ * 256 / t or 0.
 #include <cfloat>
 
 #include "fa_internal.h"
@@ -157,6 +172,47 @@ struct FwdParams {
   const float* k_scale;
   const float* v_amax;
 };
+// The bias / dropout options (EX instantiations), a kernel parameter of
+// their own: growing FwdParams changed the register allocation of the
+// other instantiations.
+struct FwdExParams {
+  const uint16_t* bias;  // bf16, element strides over b and h, rows of N
+  long long bias_sb, bias_sh;
+  int H;
+  int bias_vec;  // rows and strides are multiples of 8 elements: 16-byte loads
+  float inv_scale;
+  uint32_t seed_lo, seed_hi, rng_offset;
+  int keep_t;    // keep iff byte < keep_t; 256 = no dropout
+  float keep_scale;
+};
+
+// bias[b, h, row, key0 .. key0 + 127] / scale added to the raw scores s
+// (keys >= N are left alone: the mask removes them)
+__device__ __forceinline__ void add_bias_row(float (&s)[128], const FwdExParams& p, int N, int bh,
+                                             int row, int key0) {
+  const int b = bh / p.H, h = bh - b * p.H;
+  const uint16_t* src = p.bias + b * p.bias_sb + h * p.bias_sh + size_t(row) * N + key0;
+  const int n = min(128, N - key0);
+  if (p.bias_vec) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      if (8 * c < n) {
+        const uint4 u = *reinterpret_cast<const uint4*>(src + 8 * c);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          s[8 * c + 2 * e] = fmaf(__uint_as_float(w[e] << 16), p.inv_scale, s[8 * c + 2 * e]);
+          s[8 * c + 2 * e + 1] =
+              fmaf(__uint_as_float(w[e] & 0xffff0000u), p.inv_scale, s[8 * c + 2 * e + 1]);
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 128; ++i)
+      if (i < n) s[i] = fmaf(__uint_as_float(uint32_t(src[i]) << 16), p.inv_scale, s[i]);
+  }
+}
 
 // The work list every role of a CTA walks (G = grid size). No mask: item i
 // = (head i / n_q, Q tile i % n_q), CTA c takes c, c + G, ... (the ~G units
@@ -193,12 +249,13 @@ __device__ __forceinline__ int steps_of(int qt, int n_q) {
   return CAUSAL ? qt + 1 : n_q;
 }
 
-template <int D, bool CAUSAL, bool F8>
+template <int D, bool CAUSAL, bool F8, bool EX>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                const FwdParams p) {
+                const FwdParams p, const FwdExParams px) {
   static_assert(!F8 || D == 128, "the FP8 forward is built for d = 128");
+  static_assert(!(F8 && EX), "bias and dropout are built for the bf16 forward");
   using L = Layout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -475,6 +532,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s[128];
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
+        if constexpr (EX) {
+          if (px.bias != nullptr && row < p.N) add_bias_row(s, px, p.N, bh, row, j * kBN);
+        }
         // mask: the diagonal tile under the causal mask, and keys >= N
         int limit = p.N - j * kBN;
         if (CAUSAL && j == qt) limit = min(limit, r + 1);
@@ -546,15 +606,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
         uint64_t sum_a = f2_pack(0.f, 0.f), sum_b = sum_a;
         uint32_t pk[L::kPvSteps * 8];
+        uint32_t keep16b = 0;  // EX: keep bits of the current 16-key block
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), c2, nm2), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           if (i & 1)
             sum_b = f2_add(sum_b, f2_pack(p0, p1));
           else
             sum_a = f2_add(sum_a, f2_pack(p0, p1));
+          if constexpr (EX) {
+            if (px.keep_t < 256) {
+              // keys j*128 + 2i and + 1: bits 2i % 16 and + 1 of the call for
+              // key block (j*128 + 2i) / 16, made every eight pairs
+              if ((i & 7) == 0)
+                keep16b = keep_bits16(make_uint4(uint32_t(j * (kBN / 16) + i / 8), uint32_t(row),
+                                                 uint32_t(bh), px.rng_offset),
+                                      px.seed_lo, px.seed_hi, uint32_t(px.keep_t));
+              const uint32_t kw = keep16b >> (2 * (i & 7));
+              p0 = (kw & 1u) ? p0 * px.keep_scale : 0.f;
+              p1 = (kw & 2u) ? p1 * px.keep_scale : 0.f;
+            }
+          }
           if constexpr (F8) {
             const uint32_t h = pack_e4m3x2(p0, p1);
             pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
@@ -669,10 +743,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool F8 = false>
+template <int D, bool CAUSAL, bool F8 = false, bool EX = false>
 fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                  const CUtensorMap& mo, const FwdParams& p, const LaunchCtx& ctx) {
-  auto kern = fwd_kernel<D, CAUSAL, F8>;
+                  const CUtensorMap& mo, const FwdParams& p, const LaunchCtx& ctx,
+                  const FwdExParams& px) {
+  auto kern = fwd_kernel<D, CAUSAL, F8, EX>;
   const int smem = Layout<D, F8>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fwd)");
@@ -689,7 +764,7 @@ fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
   const int grid = p.num_items < ctx.num_sms ? p.num_items : ctx.num_sms;
   {
     ProfileScope prof(KID_FWD, ctx.stream);
-    kern<<<grid, kThreads, smem, ctx.stream>>>(mq, mk, mv, mo, p);
+    kern<<<grid, kThreads, smem, ctx.stream>>>(mq, mk, mv, mo, p, px);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
@@ -700,7 +775,7 @@ fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
 
 fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
                            int B, int H, int N, int d, float scale, bool causal,
-                           const LaunchCtx& ctx) {
+                           const LaunchCtx& ctx, const FwdExtras* ex) {
   const uint64_t BH = uint64_t(B) * uint64_t(H);
   CUtensorMap mq, mk, mv, mo;
   fa_status st;
@@ -719,11 +794,36 @@ fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, 
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load == KID_FWD;
   p.q_scale = p.k_scale = p.v_amax = nullptr;
+  FwdExParams px;
+  px.bias = nullptr;
+  px.bias_sb = px.bias_sh = 0;
+  px.H = H;
+  px.bias_vec = 0;
+  px.inv_scale = 1.0f / scale;
+  px.seed_lo = px.seed_hi = px.rng_offset = 0;
+  px.keep_t = 256;
+  px.keep_scale = 1.0f;
+  if (ex != nullptr && (ex->bias != nullptr || ex->keep_t < 256)) {
+    px.bias = static_cast<const uint16_t*>(ex->bias);
+    px.bias_sb = ex->bias_stride_b;
+    px.bias_sh = ex->bias_stride_h;
+    px.bias_vec = (N % 8 == 0 && ex->bias_stride_b % 8 == 0 && ex->bias_stride_h % 8 == 0) ? 1 : 0;
+    px.seed_lo = uint32_t(ex->seed);
+    px.seed_hi = uint32_t(ex->seed >> 32);
+    px.rng_offset = ex->offset;
+    px.keep_t = ex->keep_t;
+    px.keep_scale = 256.0f / float(ex->keep_t);
+    if (causal)
+      return d == 128 ? launch<128, true, false, true>(mq, mk, mv, mo, p, ctx, px)
+                      : launch<64, true, false, true>(mq, mk, mv, mo, p, ctx, px);
+    return d == 128 ? launch<128, false, false, true>(mq, mk, mv, mo, p, ctx, px)
+                    : launch<64, false, false, true>(mq, mk, mv, mo, p, ctx, px);
+  }
   if (causal)
-    return d == 128 ? launch<128, true>(mq, mk, mv, mo, p, ctx)
-                    : launch<64, true>(mq, mk, mv, mo, p, ctx);
-  return d == 128 ? launch<128, false>(mq, mk, mv, mo, p, ctx)
-                  : launch<64, false>(mq, mk, mv, mo, p, ctx);
+    return d == 128 ? launch<128, true>(mq, mk, mv, mo, p, ctx, px)
+                    : launch<64, true>(mq, mk, mv, mo, p, ctx, px);
+  return d == 128 ? launch<128, false>(mq, mk, mv, mo, p, ctx, px)
+                  : launch<64, false>(mq, mk, mv, mo, p, ctx, px);
 }
 
 fa_status launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* q_scale,
@@ -750,12 +850,15 @@ fa_status launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const 
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_amax = v_amax;
+  FwdExParams px{};
+  px.H = H;
+  px.keep_t = 256;
   if (d != 128) {
     set_last_error("the FP8 forward needs d = 128 (got %d)", d);
     return FA_ERR_UNSUPPORTED;
   }
-  return causal ? launch<128, true, true>(mq, mk, mv, mo, p, ctx)
-                : launch<128, false, true>(mq, mk, mv, mo, p, ctx);
+  return causal ? launch<128, true, true>(mq, mk, mv, mo, p, ctx, px)
+                : launch<128, false, true>(mq, mk, mv, mo, p, ctx, px);
 }
 
 }  // namespace fa

@@ -364,6 +364,37 @@ __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers:
+// as easy as 1, 2, 3", SC 2011): ten rounds of
+//   (c0, c1, c2, c3) -> (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1, lo(M0 c0))
+// with the key advanced by the Weyl constants between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+  constexpr uint32_t kM0 = 0xD2511F53u, kM1 = 0xCD9E8D57u;
+  constexpr uint32_t kW0 = 0x9E3779B9u, kW1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = kM0 * c.x, hi0 = __umulhi(kM0, c.x);
+    const uint32_t lo1 = kM1 * c.z, hi1 = __umulhi(kM1, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += kW0;
+    k1 += kW1;
+  }
+  return c;
+}
+
+// Dropout keep bits of one generator call: bit e (0..15) is set iff byte e
+// of Philox4x32-10(counter, key) (byte e % 4 of word e / 4, least
+// significant first) is below t
+__device__ __forceinline__ uint32_t keep_bits16(uint4 counter, uint32_t k0, uint32_t k1,
+                                                uint32_t t) {
+  const uint4 w = philox4x32_10(counter, k0, k1);
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) m |= (((ws[e >> 2] >> (8 * (e & 3))) & 0xffu) < t ? 1u : 0u) << e;
+  return m;
+}
+
 // two fp32 -> packed bf16x2 (round to nearest even); `lo` in the low half
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

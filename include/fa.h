@@ -101,6 +101,45 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o,
                      int causal, cudaStream_t stream);
 
 /*
+ * fa_fwd_ex / fa_bwd_ex -- fa_fwd / fa_bwd with the two options of the
+ * attention definition and of dropout ("FlashAttention'i Anlamak Bolum 1",
+ * 0.2: S = Q K^T / sqrt(d) + B, B an optional mask or bias; "Bellek
+ * Duvarinin Fizigi", "Maskeleme ve Dropout": dropout on P from a
+ * counter-based generator driven by a seed and an offset, the backward
+ * regenerating the same mask).
+ *   bias    : bf16, element (b, h, i, j) at bias[b*bias_stride_b +
+ *             h*bias_stride_h + i*N + j] (rows of N keys contiguous; a
+ *             stride of 0 broadcasts), or NULL. 16-byte aligned. Added to
+ *             the scaled scores before the causal mask and the row maximum;
+ *             an input only (fa_bwd_ex returns no gradient for it); -inf
+ *             entries mask (every row needs one finite score).
+ *   p_drop  : dropout probability in [0, 1); 0 = no dropout.
+ *   seed, offset : the generator's key and sequence offset. Pair (i, j) of
+ *             head (b, h) takes byte (j % 16) % 4 of word (j % 16) / 4 of
+ *             Philox4x32-10(counter = (j / 16, i, b*H + h, offset),
+ *             key = (seed mod 2^32, seed >> 32)); it is kept iff that byte
+ *             < t = round(256 (1 - p_drop)) (ties to even, 1 <= t <= 256),
+ *             and a kept P is scaled by 256 / t.
+ * O = (P * keep * 256/t) V; the LSE is that of the undropped P. fa_bwd_ex
+ * must get the same bias, p_drop, seed and offset as the forward that made
+ * o and lse. Other arguments, workspace and errors as for fa_fwd / fa_bwd.
+ */
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o,
+                    float* lse, int B, int H, int N, int d, float scale,
+                    int causal, const void* bias, long long bias_stride_b,
+                    long long bias_stride_h, float p_drop,
+                    unsigned long long seed, unsigned int offset,
+                    cudaStream_t stream);
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                    const float* lse, const void* dO, void* dq, void* dk,
+                    void* dv, int B, int H, int N, int d, float scale,
+                    int causal, const void* bias, long long bias_stride_b,
+                    long long bias_stride_h, float p_drop,
+                    unsigned long long seed, unsigned int offset,
+                    void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
+/*
  * FP8 forward with incoherent processing ("FlashAttention-3 (TR)", section
  * "FlashAttention-3'un Teknik Yenilikleri", item 3: Q and K multiplied by a
  * random orthogonal matrix before FP8 quantisation, which spreads outliers

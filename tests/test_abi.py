@@ -13,7 +13,7 @@ EXPECTED = {
     "fa_decode_workspace_size", "fa_decode_splitkv", "fa_device_status",
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_profile_begin",
     "fa_profile_end", "fa_decode_splitkv_static", "fa_decode_paged",
-    "fa_fp8_vt_keys", "fa_fp8_prepare", "fa_fwd_fp8",
+    "fa_fp8_vt_keys", "fa_fp8_prepare", "fa_fwd_fp8", "fa_fwd_ex", "fa_bwd_ex",
 }
 
 
@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     for code, name in fa.STATUS.items():
         assert lib.fa_status_string(code).decode() == name
-    assert lib.fa_abi_version() == 102
+    assert lib.fa_abi_version() == 103
 
 
 def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=8, d=64,
@@ -121,6 +121,24 @@ def test_fp8_argument_errors(lib):
     assert fwd(scale=0.0) == 1
     assert lib.fa_fp8_vt_keys(1) == 16 and lib.fa_fp8_vt_keys(32) == 32
     assert lib.fa_fp8_vt_keys(1000) == 1008 and lib.fa_fp8_vt_keys(0) == 0
+
+
+def test_bias_dropout_argument_errors(lib):
+    P = ctypes.c_void_p
+
+    def fwd(bias=None, sb=0, sh=0, p=0.1):
+        return lib.fa_fwd_ex(P(16), P(16), P(16), P(16), P(16), 1, 1, 8, 64, 0.125, 0,
+                             P(bias) if bias else None, sb, sh, p, 1, 0, None)
+
+    def bwd(p=0.1, ws=1 << 20):
+        return lib.fa_bwd_ex(P(16), P(16), P(16), P(16), P(16), P(16), P(16), P(16), P(16),
+                             1, 1, 8, 64, 0.125, 0, None, 0, 0, p, 1, 0, P(16), ws, None)
+
+    assert fwd(p=1.0) == 1 and fwd(p=-0.1) == 1 and fwd(p=float("nan")) == 1
+    assert fwd(bias=24) == 3                       # bias not 16-byte aligned
+    assert fwd(bias=16, sb=-1) == 1                # negative stride
+    assert bwd(p=1.5) == 1
+    assert bwd(ws=8) == 4                          # workspace too small
 
 
 def test_workspace_sizes(lib):

@@ -584,7 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = wait_pv_prev();
             if (!ok) break;
             tc_fence_after();
-            const float alpha = ex2_approx(m_ref - m_new);
+            // (EX: a row whose keys a -inf bias has hidden so far holds nothing
+            // yet, and 2^(-inf - m_new) would be NaN when m_new is -inf too)
+            const float alpha = (EX && m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_new);
             l_part *= alpha;
             m_ref = m_new;
 #pragma unroll
@@ -603,7 +605,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(BAR(B_DEC + (g & 1)));
         // P = 2^(s c - m_ref) by one paired FMA per two columns and MUFU ex2,
         // row sum by paired adds, packed to bf16 (e4m3 for F8) in registers
-        const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+        // a bias of -inf can hide every key a row has seen so far (m_ref =
+        // -inf): its P is then 0, formed against the reference 0
+        const float m_use = (EX && m_ref == -INFINITY) ? 0.f : m_ref;
+        const uint64_t nm2 = f2_pack(-m_use, -m_use);
         uint64_t sum_a = f2_pack(0.f, 0.f), sum_b = sum_a;
         uint32_t pk[L::kPvSteps * 8];
         uint32_t keep16b = 0;  // EX: keep bits of the current 16-key block

@@ -113,3 +113,57 @@ def test_ex_without_options_matches_plain():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     for a, b in zip(g1, g2):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("mask", ["left_pad", "window"])
+def test_bias_as_mask(mask, causal):
+    """-inf bias entries hide keys; for a left padding of 200 keys every row's
+    first key tile is hidden entirely. Rows keep at least one visible key."""
+    B, H, N, d = 1, 2, 520, 128
+    x = inputgen.make_small_inputs(401, B, H, N, d, with_grad=True)
+    i, j = np.arange(N)[:, None], np.arange(N)[None, :]
+    if mask == "left_pad":
+        hide = (j < 200) & (i >= 0)
+        if causal:
+            hide &= i >= 200  # rows before 200 would have no visible key
+    else:
+        hide = j < i - 150
+    bias = np.where(hide, -np.inf, 0.25 * np.sin(i + 2 * j)).astype(np.float32)[None, None]
+    bb = inputgen.bf16_round_bits(np.repeat(bias, H, axis=1))
+    o, lse = _run_fwd(x, causal, bb, 0.1, 5, 0)
+    keep, ks = oracle.dropout_keep(B, H, N, 5, 0, 0.1)
+    args = (f64(x["q"]), f64(x["k"]), f64(x["v"]))
+    ro, rl = oracle.attention_fwd_ex(*args, 1 / math.sqrt(d), causal, bias=f64(bb), keep=keep,
+                                     keep_scale=ks)
+    og = o.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(og))
+    assert np.all(np.abs(og - ro) <= TOL_O + 2.0 ** -8 * np.abs(ro))
+    assert max_abs(lse, rl) <= TOL_LSE
+    q, k, v, do = (bf16_device(x[n]) for n in ("q", "k", "v", "do"))
+    grads = fa.fa_bwd_ex(q, k, v, o, lse, do, causal=causal, bias=bf16_device(bb), p_drop=0.1,
+                         seed=5, offset=0)
+    torch.cuda.synchronize()
+    ref = oracle.attention_bwd_ex(*args, f64(x["do"]), 1 / math.sqrt(d), causal, bias=f64(bb),
+                                  keep=keep, keep_scale=ks)
+    for g, r in zip(grads, ref):
+        assert rel_fro(g, r) <= TOL_GRAD_REL
+
+
+def test_dropout_extreme_keep_threshold():
+    """p = 0.997: t = round(256 * 0.003) = 1, a pair is kept iff its byte is 0
+    (1 in 256) and scaled by 256. A row of O is then a sum of a few terms of
+    size ~25 that cancel, so the bf16 rounding of P (2^-9 relative per term)
+    is bounded by 2^-8 (P Z)|V|, not by |O|."""
+    B, H, N, d = 1, 1, 384, 64
+    x = inputgen.make_small_inputs(402, B, H, N, d, with_grad=True)
+    o, lse = _run_fwd(x, False, None, 0.997, 77, 3)
+    keep, ks = oracle.dropout_keep(B, H, N, 77, 3, 0.997)
+    assert ks == 256.0
+    ro, rl = oracle.attention_fwd_ex(f64(x["q"]), f64(x["k"]), f64(x["v"]), 1 / math.sqrt(d), False,
+                                     keep=keep, keep_scale=ks)
+    mag, _ = oracle.attention_fwd_ex(f64(x["q"]), f64(x["k"]), np.abs(f64(x["v"])), 1 / math.sqrt(d),
+                                     False, keep=keep, keep_scale=ks)
+    og = o.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(og - ro) <= TOL_O + 2.0 ** -8 * mag)
+    assert max_abs(lse, rl) <= TOL_LSE

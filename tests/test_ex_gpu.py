@@ -152,9 +152,10 @@ def test_bias_as_mask(mask, causal):
 
 def test_dropout_extreme_keep_threshold():
     """p = 0.997: t = round(256 * 0.003) = 1, a pair is kept iff its byte is 0
-    (1 in 256) and scaled by 256. A row of O is then a sum of a few terms of
-    size ~25 that cancel, so the bf16 rounding of P (2^-9 relative per term)
-    is bounded by 2^-8 (P Z)|V|, not by |O|."""
+    (1 in 256) and scaled by 256. A row of O is then a sum of a few large
+    terms (often one), so the error is bounded by the roundings of P and of
+    O to bf16 (unit roundoff 2^-8 each): 2^-7 (P Z)|V|, not a multiple of |O|
+    alone."""
     B, H, N, d = 1, 1, 384, 64
     x = inputgen.make_small_inputs(402, B, H, N, d, with_grad=True)
     o, lse = _run_fwd(x, False, None, 0.997, 77, 3)
@@ -165,5 +166,8 @@ def test_dropout_extreme_keep_threshold():
     mag, _ = oracle.attention_fwd_ex(f64(x["q"]), f64(x["k"]), np.abs(f64(x["v"])), 1 / math.sqrt(d),
                                      False, keep=keep, keep_scale=ks)
     og = o.float().cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(og - ro) <= TOL_O + 2.0 ** -8 * mag)
+    bad = np.abs(og - ro) - (TOL_O + 2.0 ** -7 * mag)
+    w = np.unravel_index(np.argmax(bad), bad.shape)
+    assert bad[w] <= 0, (w, og[w], ro[w], mag[w], int((bad > 0).sum()),
+                         int(keep[0, 0, w[2]].sum()))
     assert max_abs(lse, rl) <= TOL_LSE

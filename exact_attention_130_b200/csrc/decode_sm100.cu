@@ -53,6 +53,7 @@ constexpr int kRowsPerHalf = kStageTok / (2 * kConsumerWarps);  // 4
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSmHint = 148;      // B200 SM count, for the automatic split
 constexpr int kTcMinGroup = 4;    // query heads per KV head from which the tensor-core path runs
+constexpr int kTcMaxGroup = 128;  // its M rows; larger groups run on the CUDA cores
 
 template <int D>
 struct DecLayout {
@@ -524,7 +525,7 @@ fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpa
   p.status = ctx.status_word;
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load == KID_DECODE;
-  if (p.group >= kTcMinGroup) {
+  if (p.group >= kTcMinGroup && p.group <= kTcMaxGroup) {
     // large groups: the query heads of a KV head as the M rows of the tensor
     // cores (decode_tc_sm100.cu), then the same merge
     fa_status st = launch_decode_paged_tc(q, kpages, vpages, block_table, seqlens, B, Hq, Hkv,

@@ -273,7 +273,10 @@ fa_status fa_decode_splitkv(const void* q, const void* kcache,
  *   o              : bf16 [B, Hq, d];  lse : fp32 [B, Hq]  (outputs, device)
  *   Hq, Hkv        : Hq a multiple of Hkv; query head h reads KV head
  *                    h / (Hq / Hkv) (Hkv = 1: multi-query; Hkv = Hq: one KV
- *                    head per query head)
+ *                    head per query head). Groups of 4 to 128 query heads
+ *                    per KV head run on the tensor cores (the group's heads
+ *                    are the rows of the MMA), the others on the CUDA cores
+ *                    (up to four heads of a group per CTA)
  *   page_size      : 16, 32 or a multiple of 64
  *   num_splits     : chunks per sequence, 0 = automatic, <= 1024
  *   workspace      : >= fa_decode_workspace_size(B, Hq, max_pages *

@@ -187,11 +187,13 @@ def test_paged_decode_bad_page_is_reported_not_read():
     _check_paged(x, o, lse, 1 / np.sqrt(128))
 
 
-@pytest.mark.parametrize("heads", [(16, 1), (64, 1), (128, 2)], ids=["g16", "g64", "g128-2kv"])
+@pytest.mark.parametrize("heads", [(16, 1), (64, 1), (128, 2), (4, 2), (6, 2), (10, 2), (256, 1)],
+                         ids=["g16", "g64", "g128-2kv", "g2", "g3", "g5", "g256"])
 def test_paged_decode_large_groups(heads):
-    """Groups of 16, 64 and 128 query heads per KV head: the tensor-core path
-    with one, two and four softmax warps; lengths leave partial last tiles
-    over NaN-filled page rows."""
+    """Groups of 2 and 3 query heads per KV head (CUDA cores, two and one
+    heads per CTA), 5, 16 and 64 (the tensor-core path with one and two
+    softmax warps), and 256 (past the tensor-core path's 128 rows: CUDA
+    cores); lengths leave partial last tiles over NaN-filled page rows."""
     hq, hkv = heads
     x = inputgen.make_paged_decode_inputs(620 + hq, 3, hq, hkv, 128, 64, seqlens=[1, 700, 4097])
     o, lse = run_paged(x)

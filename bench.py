@@ -28,8 +28,9 @@ scaling, no collective on the data path); the timed region is bracketed by a
 barrier and a device synchronise on both sides and the per-rank time is
 reduced with MAX.
 
---impl reference times the fp64 CPU oracle (the only reference this build
-has) on a bounded sample of the same workload per step, on rank 0.
+--impl reference times the fp64 CPU oracle (the one reference
+implementation there is to time) on a bounded sample of the same workload
+per step, on rank 0.
 """
 from __future__ import annotations
 

@@ -21,7 +21,7 @@ import re
 
 __all__ = [
     "FAError", "library_path", "load_library", "exported_symbols",
-    "fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_f32", "fa_fp8_prepare", "fa_fwd_fp8",
+    "fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_dropout_keep_threshold", "fa_fwd_f32", "fa_fp8_prepare", "fa_fwd_fp8",
     "fa_fp8_vt_keys",
     "fa_bwd", "fa_bwd_workspace_size",
     "fa_decode_splitkv", "fa_decode_workspace_size", "fa_decode_splitkv_static",
@@ -68,6 +68,7 @@ _SIGNATURES = {
                        ctypes.c_longlong, ctypes.c_longlong, _F, ctypes.c_ulonglong, ctypes.c_uint,
                        _P, _S, _P]),
     "fa_fp8_vt_keys": (_I, [_I]),
+    "fa_dropout_keep_threshold": (_I, [_F]),
     "fa_fp8_prepare": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
@@ -206,6 +207,11 @@ def fa_fwd_ex(q, k, v, causal: bool = False, scale: float | None = None, bias=No
                          int(bool(causal)), bp, sb, sh, float(p_drop), int(seed), int(offset),
                          _stream(stream)))
     return o, lse
+
+
+def fa_dropout_keep_threshold(p_drop: float) -> int:
+    """The keep threshold t of fa_fwd_ex / fa_bwd_ex for p_drop (-1 if invalid)."""
+    return int(load_library().fa_dropout_keep_threshold(float(p_drop)))
 
 
 def fa_bwd_ex(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, bias=None,

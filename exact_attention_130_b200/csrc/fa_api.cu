@@ -226,7 +226,7 @@ const char* fa_status_string(fa_status s) {
 
 const char* fa_last_error(void) { return t_last_error; }
 
-int fa_abi_version(void) { return 103; }
+int fa_abi_version(void) { return 104; }
 
 void fa_set_wait_limit(unsigned long long ns) {
   g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs);
@@ -274,6 +274,12 @@ static fa_status make_extras(const void* bias, long long bias_stride_b, long lon
   ex->offset = offset;
   ex->keep_t = int(t);
   return FA_OK;
+}
+
+int fa_dropout_keep_threshold(float p_drop) {
+  FwdExtras ex;
+  if (make_extras(nullptr, 0, 0, 1, 1, 1, p_drop, 0, 0, &ex) != FA_OK) return -1;
+  return ex.keep_t;
 }
 
 fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -124,6 +124,11 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o,
  * must get the same bias, p_drop, seed and offset as the forward that made
  * o and lse. Other arguments, workspace and errors as for fa_fwd / fa_bwd.
  */
+/* The keep threshold t that fa_fwd_ex / fa_bwd_ex use for p_drop
+ * (round(256 (1 - p_drop)), ties to even, clamped to [1, 256]), or -1 for a
+ * p_drop outside [0, 1). */
+int fa_dropout_keep_threshold(float p_drop);
+
 fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o,
                     float* lse, int B, int H, int N, int d, float scale,
                     int causal, const void* bias, long long bias_stride_b,

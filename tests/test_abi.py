@@ -14,6 +14,7 @@ EXPECTED = {
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_profile_begin",
     "fa_profile_end", "fa_decode_splitkv_static", "fa_decode_paged",
     "fa_fp8_vt_keys", "fa_fp8_prepare", "fa_fwd_fp8", "fa_fwd_ex", "fa_bwd_ex",
+    "fa_dropout_keep_threshold",
 }
 
 
@@ -38,7 +39,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     for code, name in fa.STATUS.items():
         assert lib.fa_status_string(code).decode() == name
-    assert lib.fa_abi_version() == 103
+    assert lib.fa_abi_version() == 104
 
 
 def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=8, d=64,
@@ -139,6 +140,20 @@ def test_bias_dropout_argument_errors(lib):
     assert fwd(bias=16, sb=-1) == 1                # negative stride
     assert bwd(p=1.5) == 1
     assert bwd(ws=8) == 4                          # workspace too small
+
+
+def test_dropout_keep_threshold_matches_oracle(lib):
+    """The host's t = round(256 (1 - p)) (ties to even, clamped) equals the
+    oracle's for the float32 p the call receives, ties included."""
+    import numpy as np
+    import oracle
+    ps = [0.0, 0.1, 0.25, 0.5, 0.997, 0.999, 0.9999, 1e-3, 0.3, 0.7]
+    ps += [float(np.float32((2 * k + 1) / 512)) for k in range(0, 256, 7)]  # exact ties
+    ps += list(np.random.default_rng(3).random(200).astype(np.float32).astype(float))
+    for p in ps:
+        p32 = float(np.float32(p))
+        assert fa.fa_dropout_keep_threshold(p32) == oracle.keep_threshold(p32), p32
+    assert fa.fa_dropout_keep_threshold(1.0) == -1 and fa.fa_dropout_keep_threshold(-0.5) == -1
 
 
 def test_workspace_sizes(lib):

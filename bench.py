@@ -516,6 +516,34 @@ def measure_next_rows(fa, torch, dev, flush, peaks, iters=8):
         rows["fwd_fp8"][f"frac_{key}"] = round(tf / fp8_peak, 4)
     del prep, o, lse
 
+    # bias (bf16 [1, H, N, N]) and dropout 0.1 on the prefill inputs:
+    # forward without mask and causal, backward causal
+    try:
+        bias = torch.randn((1, H, N, N), device="cuda", dtype=torch.bfloat16, generator=g)
+        ex = dict(bias=bias, p_drop=0.1, seed=20265, offset=0)
+        oe = torch.empty_like(dev["q"])
+        le = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+        row = {"workload": f"prefill B={B} H={H} N={N} d={d}, bias [1, H, N, N] bf16, dropout 0.1",
+               "unit": "TFLOP/s", "peak": peaks["bf16_tflops"]}
+        for causal in (False, True):
+            ms = med_ms(lambda: fa.fa_fwd_ex(dev["q"], dev["k"], dev["v"], causal=causal, o=oe,
+                                             lse=le, **ex))
+            key = "causal" if causal else "full"
+            row[f"fwd_ms_{key}"] = round(ms, 4)
+            row[f"fwd_tflops_{key}"] = round(4.0 * B * H * N * N * d / (2 if causal else 1)
+                                             / (ms * 1e-3) / 1e12, 1)
+        fa.fa_fwd_ex(dev["q"], dev["k"], dev["v"], causal=True, o=oe, lse=le, **ex)
+        ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+        g3 = [torch.empty_like(dev["q"]) for _ in range(3)]
+        ms = med_ms(lambda: fa.fa_bwd_ex(dev["q"], dev["k"], dev["v"], oe, le, dev["do"], causal=True,
+                                         dq=g3[0], dk=g3[1], dv=g3[2], workspace=ws, **ex))
+        row["bwd_ms_causal"] = round(ms, 4)
+        row["bwd_tflops_causal"] = round(2.5 * 2.0 * B * H * N * N * d / (ms * 1e-3) / 1e12, 1)
+        rows["bias_dropout"] = row
+        del bias, oe, le, ws, g3
+    except Exception as e:  # reported in the line, never fatal to the bench
+        rows["bias_dropout"] = {"error": f"{type(e).__name__}: {e}"[:200]}
+
     # paged decode: B=8, Hq=32, Hkv=8, d=128, 64-row pages in a shuffled
     # order, lengths uniform in [16384, 32768]
     Bq, Hq, Hkv, page, cap = 8, 32, 8, 64, 32768

@@ -1,4 +1,6 @@
 """The seeded input generator: bf16 rounding and reproducibility."""
+import math
+
 import numpy as np
 import torch
 
@@ -46,3 +48,22 @@ def test_row_block_sample():
     assert len(s) == 64 and len(set(s)) == 64
     assert all(0 <= h < 32 and 0 <= blk < 128 and b == 0 for b, h, blk in s)
     assert s == inputgen.sample_row_blocks(w, 64)
+
+
+def test_fp8_inputs_recipe():
+    """Seeded and reproducible; signs are +-1; the outlier fraction is within
+    a binomial bound of the one asked for; outputs are bf16 bit patterns."""
+    a = inputgen.make_fp8_inputs(5, 2, 2, 256, 128, outlier_frac=0.01, outlier_std=10.0)
+    b = inputgen.make_fp8_inputs(5, 2, 2, 256, 128, outlier_frac=0.01, outlier_std=10.0)
+    for n in ("q", "k", "v", "signs"):
+        assert np.array_equal(a[n], b[n])
+    assert set(np.unique(a["signs"]).tolist()) <= {-1.0, 1.0} and a["signs"].shape == (128,)
+    assert a["q"].dtype == np.uint16 and a["q"].shape == (2, 2, 256, 128)
+    x = inputgen.bf16_bits_to_f32(a["q"])
+    n = x.size
+    big = np.mean(np.abs(x) > 6.0)  # N(0,1) alone exceeds 6 with probability ~2e-9
+    # a marked entry is N(0, 1 + 100): |x| > 6 with probability erfc(6 / sqrt(2 * 101))
+    p_big = 0.01 * math.erfc(6.0 / math.sqrt(2 * 101))
+    assert abs(big - p_big) < 6 * np.sqrt(p_big / n), (big, p_big)
+    plain = inputgen.make_fp8_inputs(5, 2, 2, 256, 128)
+    assert np.max(np.abs(inputgen.bf16_bits_to_f32(plain["q"]))) < 7.0

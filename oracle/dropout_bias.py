@@ -37,18 +37,19 @@ Readings taken where the pages stop (listed with the design notes):
 * the LSE is that of the undropped softmax, O = (P * keep * 256/t) V, and
   D = rowsum(dO * O) with that O.
 
-Pins (``tests/test_oracle_dropout_bias.py``): the Weyl constants against
-their closed forms (golden ratio and sqrt(3)), byte uniformity and the keep
-fraction within binomial bounds, independence of the mask from the seed and
-offset, p = 0 giving plain attention, a bias of -inf above the diagonal
-giving causal attention, a bias equal to scale * Q' K'^T giving the
-attention of the concatenated [Q, Q'] and [K, K'], a per-row constant bias
-leaving O unchanged and shifting the LSE, the mean of O over many seeds
-approaching the undropped O, and the backward against central finite
-differences of the forward at a fixed mask. The exact Philox bit stream has
-no independent reference here (no library on this machine implements
-Philox4x32): its pins are the statistical ones above, and the CUDA side is
-compared with it bit for bit through the dropout mask.
+Pins (``tests/test_oracle_dropout_bias.py``): the generator against the
+known-answer vectors its authors publish with the Random123 library
+(``tests/golden/philox4x32_10_kat.json``: zero, all-ones and pi-digit
+counter/key pairs, every output word bit for bit); the Weyl constants
+against their closed forms (golden ratio and sqrt(3)); byte uniformity and
+the keep fraction within binomial bounds; independence of the mask from the
+seed and offset; p = 0 giving plain attention; a bias of -inf above the
+diagonal giving causal attention; a bias equal to scale * Q' K'^T giving
+the attention of the concatenated [Q, Q'] and [K, K']; a per-row constant
+bias leaving O unchanged and shifting the LSE; the mean of O over many
+seeds approaching the undropped O; and the backward against central finite
+differences of the forward at a fixed mask. The CUDA side is compared with
+this generator bit for bit through the dropout mask.
 """
 from __future__ import annotations
 

@@ -1,6 +1,8 @@
 """Pins of the bias / dropout oracle (CPU only), and planted mistakes.
 
-What pins it, besides itself: the Weyl constants' closed forms; the keep
+What pins it, besides itself: the published known-answer vectors of
+Philox4x32-10 (tests/golden/philox4x32_10_kat.json); the Weyl constants'
+closed forms; the keep
 fraction and byte uniformity within binomial / chi-square bounds; p = 0
 reducing to the plain oracle; a -inf bias above the diagonal reducing to the
 causal oracle; a bias scale * Q' K'^T reducing to the plain attention of the
@@ -10,7 +12,9 @@ approaching the undropped result; and the backward against central finite
 differences of the forward at a fixed mask.
 """
 import contextlib
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -21,6 +25,25 @@ from oracle import dropout_bias as DB
 
 def _rand(seed, *shape):
     return np.random.default_rng(seed).standard_normal(shape)
+
+
+_KAT = os.path.join(os.path.dirname(__file__), "golden", "philox4x32_10_kat.json")
+
+
+def pin_philox_known_answers():
+    """Philox4x32-10 reproduces the generator authors' published
+    known-answer vectors bit for bit (an independent reference: a wrong
+    multiplier, round count, word order or key schedule changes every
+    output word)."""
+    with open(_KAT) as f:
+        vectors = json.load(f)["vectors"]
+    assert len(vectors) == 3
+    for vec in vectors:
+        c = [np.array([int(x, 16)], dtype=np.uint64) for x in vec["counter"]]
+        k0, k1 = (int(x, 16) for x in vec["key"])
+        got = [int(np.asarray(w).ravel()[0]) for w in DB.philox4x32_10(*c, k0, k1)]
+        want = [int(x, 16) for x in vec["output"]]
+        assert got == want, (vec["name"], [f"{x:08x}" for x in got])
 
 
 def pin_weyl_constants():
@@ -157,6 +180,7 @@ def pin_backward_finite_differences():
 
 
 PINS = [
+    pin_philox_known_answers,
     pin_weyl_constants,
     pin_bytes_uniform_and_keep_fraction,
     pin_mask_depends_on_seed_offset_head,
@@ -217,7 +241,40 @@ def _mut_bwd_dp_unmasked(q, k, v, do, scale, causal, bias=None, keep=None, keep_
     return dq, dk, dv
 
 
+def _philox_variant(rounds=10, swap_words=False, bump_first=False, swap_mult=False):
+    """A Philox4x32 with one plausible slip, written out independently of
+    the oracle's function so the slip is the only difference."""
+    M32 = 0xFFFFFFFF
+    m0, m1 = (DB.PHILOX_M1, DB.PHILOX_M0) if swap_mult else (DB.PHILOX_M0, DB.PHILOX_M1)
+
+    def f(c0, c1, c2, c3, k0, k1):
+        cs = np.broadcast_arrays(*[np.asarray(x, dtype=np.uint64) & np.uint64(M32)
+                                   for x in (c0, c1, c2, c3)])
+        a, b, c, d = (x.copy() for x in cs)
+        ka, kb = np.uint64(k0 & M32), np.uint64(k1 & M32)
+        for r in range(rounds):
+            if bump_first:
+                ka = (ka + np.uint64(DB.PHILOX_W0)) & np.uint64(M32)
+                kb = (kb + np.uint64(DB.PHILOX_W1)) & np.uint64(M32)
+            p0, p1 = np.uint64(m0) * a, np.uint64(m1) * c
+            a, b, c, d = ((p1 >> np.uint64(32)) ^ b ^ ka, p1 & np.uint64(M32),
+                          (p0 >> np.uint64(32)) ^ d ^ kb, p0 & np.uint64(M32))
+            if not bump_first:
+                ka = (ka + np.uint64(DB.PHILOX_W0)) & np.uint64(M32)
+                kb = (kb + np.uint64(DB.PHILOX_W1)) & np.uint64(M32)
+        out = [x.astype(np.uint32) for x in (a, b, c, d)]
+        if swap_words:
+            out = [out[1], out[0], out[3], out[2]]
+        return tuple(out)
+
+    return f
+
+
 MUTANTS = {
+    "philox_7_rounds": {"philox4x32_10": _philox_variant(rounds=7)},
+    "philox_output_words_swapped": {"philox4x32_10": _philox_variant(swap_words=True)},
+    "philox_key_bumped_before_round": {"philox4x32_10": _philox_variant(bump_first=True)},
+    "philox_multipliers_swapped": {"philox4x32_10": _philox_variant(swap_mult=True)},
     "bias_transposed": {"_scores_ex": _mut_bias_transposed},
     "bias_added_after_mask": {"_scores_ex": _mut_bias_after_mask},
     "dropout_without_rescale": {"dropout_keep": _mut_no_rescale},

@@ -82,6 +82,30 @@ def pin_rotation_is_sylvester_hadamard():
                                    rtol=0, atol=1e-4)
 
 
+def pin_rotation_fp32_error_bound():
+    """On random non-integer inputs of several magnitudes the fp32
+    butterflies equal the fp64 dense product (x * signs) H_d within the
+    standard bound for a sum evaluated in log2(d) rounded stages: each
+    output is a signed sum of all d inputs, so its error is at most
+    gamma_k * sum_i |x_i| with k = log2(d) and gamma_k = k u / (1 - k u),
+    u = 2^-24 (plus the exact conversion of x to fp32)."""
+    rng = np.random.default_rng(61)
+    u = 2.0 ** -24
+    for d in (64, 128):
+        H = scipy.linalg.hadamard(d).astype(np.float64)
+        k = int(np.log2(d))
+        gamma = k * u / (1 - k * u)
+        for mag in (1e-3, 1.0, 37.5, 1e4):
+            signs = rng.choice([-1.0, 1.0], size=d).astype(np.float32)
+            x = (mag * rng.standard_normal((64, d))).astype(np.float32)
+            exact = (x.astype(np.float64) * signs) @ H
+            got = F.hadamard_rotate_f32(x, signs).astype(np.float64)
+            bound = gamma * np.abs(x.astype(np.float64)).sum(axis=1, keepdims=True)
+            assert np.all(np.abs(got - exact) <= bound), (d, mag)
+            # and not exact everywhere: the inputs really exercise rounding
+            assert np.any(got != exact)
+
+
 def pin_rotation_identities():
     rng = np.random.default_rng(7)
     d = 128
@@ -195,6 +219,7 @@ PINS = [
     pin_encode_matches_library,
     pin_encode_saturates_and_round_trips,
     pin_rotation_is_sylvester_hadamard,
+    pin_rotation_fp32_error_bound,
     pin_rotation_identities,
     pin_quantize_exact_on_grid,
     pin_quantize_error_bound,

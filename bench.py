@@ -14,8 +14,13 @@ workload (B=4, H=16, N=2048, d=128, bf16, iid N(0,1) inputs):
 The metric is attention TFLOP/s: FLOPs are 4 B H N^2 d per forward (halved
 under the causal mask), 2.5x that for the backward, 4 H L d per decoded
 token; `value` is the whole-job throughput over all ranks. The JSON line also
-carries a per-kernel breakdown with each kernel's fraction of its roofline
-(tensor peak for the forward/backward, HBM bandwidth for decode).
+carries a per-kernel breakdown of the step with each kernel's fraction of its
+roofline (tensor peak for the forward/backward, HBM bandwidth for decode; the
+no-mask and causal forward launches apart), and, under `configs`, every
+benchmark workload timed on its own shape after the step: prefill forward
+(B=4 H=16 N=2048 d=128) without and with the causal mask, the long causal
+forward (B=1 H=32 N=16384), the backward (B=2 H=16 N=4096, causal) and the
+split-KV decode (B=8 H=32, cache lengths 16k-32k).
 
 Inputs are resident in HBM when the timed region starts; L2 (126 MB) is
 flushed between timed steps by writing a 256 MB buffer outside the timed
@@ -64,6 +69,9 @@ def parse_args():
     # single-kernel mode, for profiler captures (prints timings, no bench line)
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the FP8 forward and paged decode measured after the step")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload measurements (prefill, long causal, backward, "
+                         "decode) made after the step")
     ap.add_argument("--kernel", choices=["fwd", "fwd_ex", "fwd_fp8", "fp8_prep", "bwd", "bwd_ex",
                                          "decode", "decode_paged"],
                     default=None)
@@ -199,7 +207,8 @@ def load_peaks():
 
 
 def kernel_source_hash(name: str) -> str:
-    files = {"fwd": "fwd_sm100.cu", "bwd_dkdv": "bwd_sm100.cu", "bwd_dq": "bwd_sm100.cu",
+    files = {"fwd_full": "fwd_sm100.cu", "fwd_causal": "fwd_sm100.cu",
+             "bwd_dkdv": "bwd_sm100.cu", "bwd_dq": "bwd_sm100.cu",
              "decode_split": "decode_sm100.cu"}
     path = os.path.join(ROOT, "exact_attention_130_b200", "csrc", files.get(name, ""))
     try:
@@ -211,7 +220,8 @@ def kernel_source_hash(name: str) -> str:
 # the launch of each kernel that one bench step makes, as named in
 # profiles/traffic.json when a capture of exactly that launch is recorded
 BENCH_LAUNCH = {
-    "fwd": "bench step: fwd B=4 H=16 N=2048 d=128 (mean of no mask and causal)",
+    "fwd_full": "bench step: fwd no mask B=4 H=16 N=2048 d=128",
+    "fwd_causal": "bench step: fwd causal B=4 H=16 N=2048 d=128",
     "bwd_dkdv": "bench step: bwd causal B=4 H=16 N=2048 d=128",
     "bwd_dq": "bench step: bwd causal B=4 H=16 N=2048 d=128",
     "decode_split": "bench step: decode B=4 H=16 cache 2048 d=128",
@@ -283,11 +293,11 @@ def run_ours(args, world, rank, local):
     # rates): the dK/dV kernel runs S^T, dP^T, dV, dK (2x the causal forward),
     # the dQ kernel S, dP, dQ (1.5x)
     fc = C.fwd_flops(B, H, N, d, True)
-    flops = {
-        "fwd": C.fwd_flops(B, H, N, d, False) + fc,
+    flops = {  # per launch (each runs once per step)
+        "fwd_full": C.fwd_flops(B, H, N, d, False),
+        "fwd_causal": fc,
         "bwd_dkdv": 2.0 * fc,
         "bwd_dq": 1.5 * fc,
-        "decode_split": C.decode_flops(H, [N] * B, d),
     }
     dec_bytes = C.decode_bytes(H, [N] * B, d)
 
@@ -323,34 +333,54 @@ def run_ours(args, world, rank, local):
     total_flops = dist_sum(world, step_flops * args.steps)
     value = total_flops / (ms_max * 1e-3) / 1e12
 
-    # 2. per-kernel breakdown (CUDA events around every launch, same steps)
-    fa.fa_profile_begin()
-    timed(lambda: step(src_dev), args.steps)
-    prof = fa.fa_profile_end()
+    # 2. per-kernel breakdown: the same steps again, each call bracketed by
+    # the library's own CUDA events around every launch (on the launching
+    # stream); the two forward launches are kept apart (no mask, causal)
     peaks = load_peaks()
+    calls = [
+        ("fwd_full", lambda: fa.fa_fwd(src_dev["q"], src_dev["k"], src_dev["v"], causal=False,
+                                       o=out["o_full"], lse=out["lse_full"])),
+        ("fwd_causal", lambda: fa.fa_fwd(src_dev["q"], src_dev["k"], src_dev["v"], causal=True,
+                                         o=out["o_causal"], lse=out["lse_causal"])),
+        ("bwd", lambda: fa.fa_bwd(src_dev["q"], src_dev["k"], src_dev["v"], out["o_causal"],
+                                  out["lse_causal"], src_dev["do"], causal=True, dq=out["dq"],
+                                  dk=out["dk"], dv=out["dv"], workspace=ws_bwd)),
+        ("decode", lambda: fa.fa_decode_splitkv(src_dev["qdec"], src_dev["k"], src_dev["v"], lens,
+                                                o=out["o_dec"], lse=out["lse_dec"],
+                                                workspace=ws_dec)),
+    ]
+    prof = {}
+    for _ in range(args.steps):
+        flush.zero_()
+        for label, fn in calls:
+            fa.fa_profile_begin()
+            fn()
+            for kname, (n, tot) in fa.fa_profile_end().items():
+                key = label if kname == "fwd" else kname
+                a = prof.setdefault(key, [0, 0.0])
+                a[0] += n
+                a[1] += tot
     kernels = {}
     for name, (n, tot) in prof.items():
         avg = tot / n
         entry = {"launches": n, "avg_ms": round(avg, 5)}
-        if name in ("fwd", "bwd_dkdv", "bwd_dq"):
+        if name in flops:
             tf = flops[name] * args.steps / (tot * 1e-3) / 1e12
-            entry.update({"tflops": round(tf, 1), "frac_of_tensor_peak": round(tf / peaks["bf16_tflops"], 4)})
+            entry.update({"tflops": round(tf, 1),
+                          "frac_of_tensor_peak": round(tf / peaks["bf16_tflops"], 4)})
         elif name == "decode_split":
             gbs = dec_bytes * args.steps / (tot * 1e-3) / 1e9
             entry.update({"gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)})
         kernels[name] = entry
     dominant = max(prof, key=lambda k: prof[k][1])
     dn, dtot = prof[dominant]
-    # work of one launch: the forward runs twice per step (no mask, causal), the
-    # backward kernels once
-    per_launch_flops = flops["fwd"] / 2 if dominant == "fwd" else flops.get(dominant, 0.0)
-    if dominant in ("fwd", "bwd_dkdv", "bwd_dq"):
+    if dominant in flops:
         achieved = flops[dominant] * args.steps / (dtot * 1e-3) / 1e12
         roofline = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 1),
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": round(achieved / peaks["bf16_tflops"], 4),
                     "traffic": recorded_traffic(dominant),
-                    "algorithmic_per_launch": per_launch_flops,
+                    "algorithmic_per_launch": flops[dominant],
                     "peak_source": peaks["source"]}
     else:
         achieved = dec_bytes * args.steps / (dtot * 1e-3) / 1e9
@@ -427,6 +457,7 @@ def run_ours(args, world, rank, local):
                "pipelining": "host-to-device copies of step i+1, kernels of step i and device-to-host "
                              "copies of step i-1 on three streams, double-buffered"}
 
+    configs = None if args.no_configs else measure_configs(fa, torch, dev, flush, peaks)
     next_rows = None if args.no_next_rows else measure_next_rows(fa, torch, dev, flush, peaks)
 
     st, word = fa.fa_device_status()
@@ -460,6 +491,7 @@ def run_ours(args, world, rank, local):
         },
         "roofline": roofline,
         "kernels": kernels,
+        "configs": configs,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(),
         "e2e": e2e,
@@ -472,6 +504,103 @@ def run_ours(args, world, rank, local):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (HGX 7.7 TB/s, DGX 8 TB/s)
+
+
+def measure_configs(fa, torch, dev, flush, peaks, iters=10):
+    """Every benchmark workload on its own, after the step (not part of
+    `value`): median of `iters` launches with L2 flushed before each, CUDA
+    events on the launching stream. Rates follow the step's conventions:
+    4 B H N^2 d forward FLOPs (halved under the causal mask), backward 2.5x
+    the forward (and, separately, the split backward's own GEMM count,
+    3.5x the causal forward), decode bytes = every visible K and V row once
+    plus q, O and LSE."""
+    import numpy as np
+
+    from exact_attention_130_b200 import counters as C
+
+    def med_ms(fn):
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    tpk = peaks["bf16_tflops"]
+    res = {}
+
+    def fwd_entry(name, q, k, v, causal, workload):
+        B, H, N, d = q.shape
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+        ms = med_ms(lambda: fa.fa_fwd(q, k, v, causal=causal, o=o, lse=lse))
+        tf = C.fwd_flops(B, H, N, d, causal) / (ms * 1e-3) / 1e12
+        res[name] = {"workload": workload, "ms": round(ms, 4), "tflops": round(tf, 1),
+                     "frac": round(tf / tpk, 4), "peak": tpk, "unit": "TFLOP/s"}
+        return o, lse
+
+    # prefill (the step's own inputs), no mask and causal apart
+    wl = "prefill B=4 H=16 N=2048 d=128"
+    fwd_entry("prefill_fwd_full", dev["q"], dev["k"], dev["v"], False, wl + ", no mask")
+    fwd_entry("prefill_fwd_causal", dev["q"], dev["k"], dev["v"], True, wl + ", causal")
+
+    g = torch.Generator(device="cuda").manual_seed(20262)
+
+    def rnd(*shape):
+        return torch.randn(shape, device="cuda", dtype=torch.bfloat16, generator=g)
+
+    # long-context causal forward
+    q, k, v = rnd(1, 32, 16384, 128), rnd(1, 32, 16384, 128), rnd(1, 32, 16384, 128)
+    fwd_entry("long_fwd_causal", q, k, v, True, "long causal B=1 H=32 N=16384 d=128")
+    del q, k, v
+
+    # backward with recomputation, O and LSE from the forward
+    q, k, v, do = (rnd(2, 16, 4096, 128) for _ in range(4))
+    o, lse = fa.fa_fwd(q, k, v, causal=True)
+    ws = torch.empty(fa.fa_bwd_workspace_size(2, 16, 4096, 128), dtype=torch.uint8, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ms = med_ms(lambda: fa.fa_bwd(q, k, v, o, lse, do, causal=True, dq=dq, dk=dk, dv=dv,
+                                  workspace=ws))
+    fc = C.fwd_flops(2, 16, 4096, 128, True)
+    tf = C.bwd_flops(2, 16, 4096, 128, True) / (ms * 1e-3) / 1e12
+    tf_own = 3.5 * fc / (ms * 1e-3) / 1e12
+    res["backward_causal"] = {
+        "workload": "backward B=2 H=16 N=4096 d=128, causal (preprocess + dK/dV + dQ)",
+        "ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / tpk, 4),
+        "convention": "2.5x the causal forward FLOPs",
+        "tflops_own_gemms": round(tf_own, 1), "frac_own_gemms": round(tf_own / tpk, 4),
+        "own_gemms": "3.5x the causal forward (S^T, dP^T, dV, dK and S, dP, dQ)",
+        "peak": tpk, "unit": "TFLOP/s"}
+    del q, k, v, do, o, lse, ws, dq, dk, dv
+
+    # split-KV decode: B=8, H=32, d=128, lengths from the workload's seeded draw
+    lens_np = np.random.default_rng(20264).integers(16384, 32769, size=8).astype(np.int32)
+    lens = torch.from_numpy(lens_np).cuda()
+    kc, vc, qd = rnd(8, 32, 32768, 128), rnd(8, 32, 32768, 128), rnd(8, 32, 128)
+    ws = torch.empty(fa.fa_decode_workspace_size(8, 32, 32768, 128, 0), dtype=torch.uint8,
+                     device="cuda")
+    od = torch.empty_like(qd)
+    ld = torch.empty((8, 32), dtype=torch.float32, device="cuda")
+    ms = med_ms(lambda: fa.fa_decode_splitkv(qd, kc, vc, lens, o=od, lse=ld, workspace=ws))
+    nbytes = C.decode_bytes(32, lens_np.tolist(), 128)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    res["decode_splitkv"] = {
+        "workload": "split-KV decode B=8 H=32 d=128, cache lengths "
+                    f"{lens_np.tolist()} (uniform [16384, 32768], seeded)",
+        "us": round(ms * 1e3, 1), "bytes": nbytes, "gbs": round(gbs, 1),
+        "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
+        "peak_kind": "measured copy rate (read + write); a read-mostly kernel can exceed it",
+        "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 4), "nominal_gbs": NOMINAL_HBM_GBS,
+        "unit": "GB/s"}
+    del kc, vc
+    return res
 
 
 def measure_next_rows(fa, torch, dev, flush, peaks, iters=8):
@@ -695,8 +824,12 @@ def run_single_kernel(args):
             o, lse = fa.fa_fwd_fp8(prep, causal=bool(args.causal))
             fn = lambda: fa.fa_fwd_fp8(prep, causal=bool(args.causal), o=o, lse=lse)  # noqa: E731
     elif args.kernel == "decode":
+        # lengths drawn as the split-KV decode workload draws them (seed
+        # 20264, uniform [N/2, N]): B=8 H=32 N=32768 is that workload
+        import numpy as np
         q, kc, vc = rnd(B, H, d), rnd(B, H, N, d), rnd(B, H, N, d)
-        lens = torch.randint(N // 2, N + 1, (B,), device="cuda", dtype=torch.int32, generator=g)
+        lens = torch.from_numpy(np.random.default_rng(20264).integers(
+            N // 2, N + 1, size=B).astype(np.int32)).cuda()
         ws = torch.empty(fa.fa_decode_workspace_size(B, H, N, d, 0), dtype=torch.uint8, device="cuda")
         fn = lambda: fa.fa_decode_splitkv(q, kc, vc, lens, workspace=ws)  # noqa: E731
     elif args.kernel in ("fwd_ex", "bwd_ex"):

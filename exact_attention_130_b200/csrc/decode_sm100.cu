@@ -464,9 +464,9 @@ size_t decode_workspace_bytes(int B, int H, int d, int chunks) {
 
 fa_status launch_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens,
                         void* o, float* lse, int B, int H, int Lmax, int d, float scale,
-                        int chunks, void* workspace, const LaunchCtx& ctx) {
+                        int chunks, void* workspace, const LaunchCtx& ctx, const char* caller) {
   if ((long long)B * H > 65535LL * 65535LL || H > 65535 || B > 65535) {
-    set_last_error("fa_decode_splitkv: B and H must each be <= 65535");
+    set_last_error("%s: B and H must each be <= 65535", caller);
     return FA_ERR_UNSUPPORTED;
   }
   DecParams p;
@@ -550,13 +550,16 @@ fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpa
 //
 // fa_decode_splitkv needs a caller-provided workspace for the per-chunk
 // partial results. Some callers cannot allocate device memory at the moment
-// they decode: code running inside a stream capture, code driven by an
-// allocator that forbids cudaMalloc on the hot path, or a host that owns no
-// memory pool of its own. For them the partials live in the fixed buffer
-// below, which is part of the library image: every GPU that loads the
-// library reserves kStaticScratchBytes of device memory for it until the
-// process exits. Nothing here calls cudaMalloc, cudaFree or any allocating
-// routine.
+// they decode: a serving loop whose allocator forbids cudaMalloc on its hot
+// path (cudaMalloc can synchronise the device and stall every other
+// stream), or a host framework that passes the library only its inputs and
+// outputs and keeps no memory pool for it. For them the partials live in
+// the fixed buffer below, which is part of the library image: every GPU
+// that loads the library reserves kStaticScratchBytes of device memory for
+// it until the process exits. Nothing here calls cudaMalloc, cudaFree or
+// any allocating routine. The fa_debug_skip_load test hook does not apply
+// to this entry point (a skip armed by it stays armed for the next call
+// that honours it).
 // ---------------------------------------------------------------------------
 namespace fa {
 namespace {
@@ -626,5 +629,5 @@ extern "C" fa_status fa_decode_splitkv_static(const void* q, const void* kcache,
   // every chunk writes its own partial (empty chunks write weight 0), so no
   // part of the scratch has to start at zero
   return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Lmax, d, scale, chunks, scratch,
-                       ctx);
+                       ctx, "fa_decode_splitkv_static");
 }

@@ -31,7 +31,9 @@ constexpr int kMaxDevices = 64;
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
 
 struct DeviceState {
-  bool ready = false;
+  // set (release) after the other fields; read (acquire) before using them,
+  // so a thread that sees it set also sees the fields it guards
+  std::atomic<bool> ready{false};
   int num_sms = 0;
   int cc_major = 0, cc_minor = 0;
   unsigned int* status_word = nullptr;
@@ -65,9 +67,9 @@ fa_status device_ctx(cudaStream_t stream, LaunchCtx* ctx) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return invalid(FA_ERR_UNSUPPORTED, "device index %d", dev);
   DeviceState& ds = g_dev[dev];
-  if (!ds.ready) {
+  if (!ds.ready.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!ds.ready) {
+    if (!ds.ready.load(std::memory_order_relaxed)) {
       cudaDeviceProp prop;
       e = cudaGetDeviceProperties(&prop, dev);
       if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
@@ -82,7 +84,7 @@ fa_status device_ctx(cudaStream_t stream, LaunchCtx* ctx) {
       ds.cc_major = prop.major;
       ds.cc_minor = prop.minor;
       ds.status_word = static_cast<unsigned int*>(addr);
-      ds.ready = true;
+      ds.ready.store(true, std::memory_order_release);
     }
   }
   ctx->stream = stream;

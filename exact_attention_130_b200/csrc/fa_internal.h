@@ -106,6 +106,7 @@ fa_status launch_decode_paged_tc(const void* q, const void* kpages, const void* 
                                  const LaunchCtx& ctx);
 fa_status launch_decode(const void* q, const void* kcache, const void* vcache,
                         const int* seqlens, void* o, float* lse, int B, int H, int Lmax, int d,
-                        float scale, int chunks, void* workspace, const LaunchCtx& ctx);
+                        float scale, int chunks, void* workspace, const LaunchCtx& ctx,
+                        const char* caller = "fa_decode_splitkv");
 
 }  // namespace fa

@@ -301,9 +301,11 @@ fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
 
 /*
  * fa_decode_splitkv_static -- fa_decode_splitkv for callers that cannot
- * allocate device memory when they decode (inside a stream capture, under an
- * allocator that forbids cudaMalloc on the hot path, or with no memory pool
- * of their own). No counterpart on the pages: it is the same computation,
+ * allocate device memory when they decode: a serving loop whose allocator
+ * forbids cudaMalloc on its hot path (cudaMalloc can synchronise the device
+ * and stall every other stream), or a host framework that passes the
+ * library only its inputs and outputs and keeps no memory pool for it.
+ * No counterpart on the pages: it is the same computation,
  * with the per-chunk partials kept in an 8 MiB buffer that is part of the
  * library image instead of a caller workspace. Arguments as for
  * fa_decode_splitkv, minus the workspace.
@@ -319,6 +321,8 @@ fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
  *    nothing in it needs to start at zero. Calls that can overlap on the GPU
  *    (different streams without ordering between them) race on it and give
  *    wrong results: serialise them.
+ *  - The test hook fa_debug_skip_load does not apply here; a skip armed by
+ *    it stays armed for the next call that honours it.
  */
 fa_status fa_decode_splitkv_static(const void* q, const void* kcache,
                                    const void* vcache, const int* seqlens,

@@ -6,7 +6,8 @@
 * O within 1e-2 + 2^-8 |O_ref| and LSE within 1e-3 of the oracle's
   ``attention_fwd_ex`` with the oracle's own mask (a kept P is scaled by
   256/t, so |O| reaches ~3 in early causal rows, where the bf16 rounding
-  of P and O, each <= 2^-9 relative, exceeds a flat 1e-2); the gradients
+  of P and O, each up to the unit roundoff 2^-8 relative, exceeds a flat
+  1e-2); the gradients
   within the backward's relative Frobenius tolerance of
   ``attention_bwd_ex``;
 * biases broadcast over batch and head, rows of 16-byte and 2-byte loads

@@ -167,9 +167,11 @@ def test_fwd_nondefault_scale_and_stream():
     """scale = 0.3 (2.4x the default): peakier rows, |O| up to ~3.5.
 
     Outside the stated workloads the O tolerance is derived from the
-    arithmetic: P enters the PV product rounded to bf16 (relative error
-    <= 2^-9) and O is stored in bf16 (another 2^-9 relative), so the bound
-    used is 1e-2 + 2^-8 |O_ref| element-wise.
+    arithmetic: P enters the PV product rounded to bf16 and O is stored in
+    bf16, each with relative error at most the unit roundoff 2^-8 (8
+    significant bits, round to nearest even). The bound used is
+    1e-2 + 2^-8 |O_ref| element-wise: the two roundings of one element
+    rarely align, and the 1e-2 base covers the remainder.
     """
     x = inputgen.make_small_inputs(9, 1, 2, 300, 64)
     s = torch.cuda.Stream()

@@ -72,8 +72,8 @@ def parse_args():
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-workload measurements (prefill, long causal, backward, "
                          "decode) made after the step")
-    ap.add_argument("--kernel", choices=["fwd", "fwd_ex", "fwd_fp8", "fp8_prep", "bwd", "bwd_ex",
-                                         "decode", "decode_paged"],
+    ap.add_argument("--kernel", choices=["fwd", "fwd_pair", "fwd_ex", "fwd_fp8", "fp8_prep", "bwd",
+                                         "bwd_ex", "decode", "decode_paged"],
                     default=None)
     ap.add_argument("--hkv", type=int, default=8, help="KV heads of --kernel decode_paged")
     ap.add_argument("--page", type=int, default=64, help="page rows of --kernel decode_paged")
@@ -849,6 +849,8 @@ def run_single_kernel(args):
         o, lse = fa.fa_fwd(q, k, v, causal=bool(args.causal))
         if args.kernel == "fwd":
             fn = lambda: fa.fa_fwd(q, k, v, causal=bool(args.causal), o=o, lse=lse)  # noqa: E731
+        elif args.kernel == "fwd_pair":
+            fn = lambda: fa.fa_fwd_pair(q, k, v, causal=bool(args.causal), o=o, lse=lse)  # noqa: E731
         else:
             ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
             dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
@@ -865,7 +867,7 @@ def run_single_kernel(args):
         if args.kernel == "decode_paged":
             extra = (f" Hkv={args.hkv} page={args.page}: "
                      f"{kv_bytes / (a.elapsed_time(b) * 1e-3) / 1e9:.1f} GB/s of KV pages")
-        elif args.kernel in ("fwd", "fwd_fp8", "fwd_ex"):
+        elif args.kernel in ("fwd", "fwd_pair", "fwd_fp8", "fwd_ex"):
             fl = 4.0 * B * H * N * N * d / (2 if args.causal else 1)
             extra = f": {fl / (a.elapsed_time(b) * 1e-3) / 1e12:.1f} TFLOP/s"
         print(f"{args.kernel} B={B} H={H} N={N} d={d} causal={args.causal} "

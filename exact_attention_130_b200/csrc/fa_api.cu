@@ -249,6 +249,19 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return launch_fwd_bf16(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx);
 }
 
+fa_status fa_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int N, int d, float scale, int causal, cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, k, v, o, lse}, "fa_fwd_pair(q,k,v,o,lse)")) != FA_OK) return st;
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if (d != 128) return invalid(FA_ERR_UNSUPPORTED, "fa_fwd_pair: head dim %d (needs 128)", d);
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (causal != 0 && causal != 1) return invalid(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  return launch_fwd_pair(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx);
+}
+
 // Validates the bias / dropout options shared by fa_fwd_ex and fa_bwd_ex.
 static fa_status make_extras(const void* bias, long long bias_stride_b, long long bias_stride_h,
                              int B, int H, int N, float p_drop, unsigned long long seed,

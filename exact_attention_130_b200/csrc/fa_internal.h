@@ -75,6 +75,10 @@ struct FwdExtras {
 fa_status launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int N, int d, float scale, bool causal,
                           const LaunchCtx& ctx, const FwdExtras* ex = nullptr);
+// The same forward on CTA pairs (tcgen05 .cta_group::2), bf16, d = 128.
+fa_status launch_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int N, int d, float scale, bool causal,
+                          const LaunchCtx& ctx);
 // Keys per row of the transposed FP8 V ([B, H, d, fp8_vt_keys(N)] codes):
 // N rounded up to 16, so that every row starts 16-byte aligned.
 inline int fp8_vt_keys(int N) { return (N + 15) & ~15; }

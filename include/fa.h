@@ -90,6 +90,21 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o,
                  int causal, cudaStream_t stream);
 
 /*
+ * fa_fwd_pair -- fa_fwd computed on pairs of CTAs that share each tensor-core
+ * product ("FlashAttention-2, -3 ve -4: Utilizasyon Savasi", the Blackwell
+ * paragraph: the 2-CTA MMA mode of tcgen05). Same arguments, layouts,
+ * results (within the same tolerances) and error behaviour as fa_fwd, for
+ * d = 128 only (else FA_ERR_UNSUPPORTED). A cluster of two CTAs takes 256
+ * query rows of one head; one CTA issues M = 256 MMAs whose K and V
+ * operands are split between the two CTAs' shared memory, so each SM loads
+ * half of every K/V tile. Allocates nothing; the work units are dealt in a
+ * fixed order, so results are bitwise repeatable.
+ */
+fa_status fa_fwd_pair(const void* q, const void* k, const void* v, void* o,
+                      float* lse, int B, int H, int N, int d, float scale,
+                      int causal, cudaStream_t stream);
+
+/*
  * fa_fwd_f32 -- the same forward on fp32 tensors, computed in fp32.
  *   q, k, v, o : fp32 [B, H, N, d];  lse : fp32 [B, H, N]
  *   d : 64 or 128; N <= 4096 (a small-problem path: fp32 inputs are not

@@ -14,7 +14,7 @@ EXPECTED = {
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_profile_begin",
     "fa_profile_end", "fa_decode_splitkv_static", "fa_decode_paged",
     "fa_fp8_vt_keys", "fa_fp8_prepare", "fa_fwd_fp8", "fa_fwd_ex", "fa_bwd_ex",
-    "fa_dropout_keep_threshold",
+    "fa_dropout_keep_threshold", "fa_fwd_pair",
 }
 
 

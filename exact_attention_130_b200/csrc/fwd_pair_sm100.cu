@@ -24,7 +24,11 @@
 //    (tcgen05.commit .multicast::cluster): scores ready, P free, O~
 //    complete, K/V slots free;
 //  * the softmax warps of both CTAs arrive on the even CTA's barriers
-//    (scores read, P stored, O read): eight arrivals each;
+//    (scores read, P stored, O read): eight arrivals each. These arrivals
+//    and the waits on them use the default (CTA-scope) semantics: the
+//    tcgen05 operations they order are fenced by tcgen05.fence, and a
+//    release or acquire at cluster scope costs a memory barrier per warp
+//    (measured: the pair kernel then ran at 0.6 of its speed without it);
 //  * each CTA's TMA loads complete on its own barriers; in the odd CTA the
 //    two threads that issue MMAs in the even one instead forward each
 //    completed load to the even CTA's barriers, so each CTA can let its own
@@ -332,7 +336,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // both Q tiles into their CTAs' TMEM (after this thread's last Q K^T
         // of the previous unit, in issue order)
         ok = wait_bounded(BAR(B_Q_FULL), u & 1, wc, 11);
-        if (ok) ok = wait_bounded_cluster(BAR(B_Q_PEER), u & 1, wc, 12);
+        if (ok) ok = wait_bounded(BAR(B_Q_PEER), u & 1, wc, 12);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -344,11 +348,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int j = 0; ok && j < n; ++j, ++g) {
           const int b = g & 1;
           // S_b is free once both CTAs' softmax loaded S(g-2)
-          if (g >= 2 && !(ok = wait_bounded_cluster(BAR(B_S_FREE + b), ((g >> 1) - 1) & 1, wc, 13)))
+          if (g >= 2 && !(ok = wait_bounded(BAR(B_S_FREE + b), ((g >> 1) - 1) & 1, wc, 13)))
             break;
           const int s = g % kStages;
           ok = wait_bounded(BAR(B_K_FULL + s), (g / kStages) & 1, wc, 14);
-          if (ok) ok = wait_bounded_cluster(BAR(B_K_PEER + s), (g / kStages) & 1, wc, 15);
+          if (ok) ok = wait_bounded(BAR(B_K_PEER + s), (g / kStages) & 1, wc, 15);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kb = sbase + L::kOffK + s * L::kKHalf;
@@ -375,13 +379,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int u = 0; ok && w.next(p, bh, qp); ++u) {
         const int n = steps_of<CAUSAL>(qp, p.n_kv);
         for (int j = 0; ok && j < n; ++j, ++g) {
-          ok = wait_bounded_cluster(BAR(B_P_FULL + (g & 3)), (g >> 2) & 1, wc, 17);
+          ok = wait_bounded(BAR(B_P_FULL + (g & 3)), (g >> 2) & 1, wc, 17);
           if (!ok) break;
           const int s = g % kStages;
           ok = wait_bounded(BAR(B_V_FULL + s), (g / kStages) & 1, wc, 18);
-          if (ok) ok = wait_bounded_cluster(BAR(B_V_PEER + s), (g / kStages) & 1, wc, 19);
+          if (ok) ok = wait_bounded(BAR(B_V_PEER + s), (g / kStages) & 1, wc, 19);
           // the epilogues of the previous unit have read O~ in both CTAs
-          if (ok && j == 0) ok = wait_bounded_cluster(BAR(B_O_EMPTY), (u & 1) ^ 1, wc, 20);
+          if (ok && j == 0) ok = wait_bounded(BAR(B_O_EMPTY), (u & 1) ^ 1, wc, 20);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vb = sbase + L::kOffV + s * L::kVHalf;

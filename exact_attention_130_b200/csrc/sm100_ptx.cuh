@@ -309,42 +309,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 // arrive on an mbarrier given by its cluster address (this CTA's or the
-// other's), releasing this thread's prior writes at cluster scope
+// other's), with the default semantics; the tcgen05 operations it orders
+// are fenced by tcgen05.fence::before_thread_sync (an arrive with release
+// at cluster scope costs each warp a memory barrier, measured as the top
+// stall of the CTA-pair forward)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-// try_wait with acquire at cluster scope (for barriers the other CTA arrives on)
-__device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n"
-      ".reg .pred p;\n"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-      "selp.u32 %0, 1, 0, p;\n"
-      "}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok;
-}
-// wait_bounded for barriers that the other CTA of the pair arrives on
-__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity,
-                                                     const WaitCtl& w, uint32_t site) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 15u) == 0u) {
-      if (*w.abort_flag) return false;
-      if (global_timer_ns() - t0 > w.limit_ns) {
-        *w.abort_flag = 1;
-        atomicCAS(w.status_word, 0u, (w.kernel_id << 16) | ((site & 0xffu) << 8) | 1u);
-        __threadfence();
-        return false;
-      }
-    }
-  }
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // all threads of both CTAs of the cluster (release / acquire at cluster scope)
 __device__ __forceinline__ void cluster_sync_all() {

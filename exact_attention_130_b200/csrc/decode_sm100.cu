@@ -54,6 +54,9 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSmHint = 148;      // B200 SM count, for the automatic split
 constexpr int kTcMinGroup = 4;    // query heads per KV head from which the tensor-core path runs
 constexpr int kTcMaxGroup = 128;  // its M rows; larger groups run on the CUDA cores
+// up to this many heads per KV head, keys as the M rows (measured: as fast
+// as heads-as-rows at 4 and 8 heads, 6% slower at 16)
+constexpr int kTctMaxGroup = 8;
 
 template <int D>
 struct DecLayout {
@@ -526,11 +529,21 @@ fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpa
   p.limit_ns = ctx.wait_limit_ns;
   p.debug_skip = ctx.debug_skip_load == KID_DECODE;
   if (p.group >= kTcMinGroup && p.group <= kTcMaxGroup) {
-    // large groups: the query heads of a KV head as the M rows of the tensor
-    // cores (decode_tc_sm100.cu), then the same merge
-    fa_status st = launch_decode_paged_tc(q, kpages, vpages, block_table, seqlens, B, Hq, Hkv,
-                                          num_pages, page_size, max_pages, d, scale, chunks,
-                                          p.part_o, p.part_lse, ctx);
+    // groups of 4 to 8 heads at d = 128: the keys as the M rows of the
+    // tensor cores (decode_tct_sm100.cu); larger groups or d = 64: the query
+    // heads as the M rows (decode_tc_sm100.cu); then the same merge
+    // (its 128-key tiles must split into runs inside one page: pages of at
+    // most 64 rows, or of a multiple of 128)
+    const bool keys_as_rows = d == 128 && p.group <= kTctMaxGroup &&
+                              (page_size <= 64 || page_size % 128 == 0);
+    fa_status st =
+        keys_as_rows
+            ? launch_decode_paged_tct(q, kpages, vpages, block_table, seqlens, B, Hq, Hkv,
+                                      num_pages, page_size, max_pages, d, scale, chunks, p.part_o,
+                                      p.part_lse, ctx)
+            : launch_decode_paged_tc(q, kpages, vpages, block_table, seqlens, B, Hq, Hkv,
+                                     num_pages, page_size, max_pages, d, scale, chunks, p.part_o,
+                                     p.part_lse, ctx);
     if (st != FA_OK) return st;
     return d == 128 ? launch_merge<128>(p, B, ctx) : launch_merge<64>(p, B, ctx);
   }

@@ -108,6 +108,11 @@ fa_status launch_decode_paged_tc(const void* q, const void* kpages, const void* 
                                  int Hkv, int num_pages, int page_size, int max_pages, int d,
                                  float scale, int chunks, float* part_o, float* part_lse,
                                  const LaunchCtx& ctx);
+fa_status launch_decode_paged_tct(const void* q, const void* kpages, const void* vpages,
+                                  const int* block_table, const int* seqlens, int B, int Hq,
+                                  int Hkv, int num_pages, int page_size, int max_pages, int d,
+                                  float scale, int chunks, float* part_o, float* part_lse,
+                                  const LaunchCtx& ctx);
 fa_status launch_decode(const void* q, const void* kcache, const void* vcache,
                         const int* seqlens, void* o, float* lse, int B, int H, int Lmax, int d,
                         float scale, int chunks, void* workspace, const LaunchCtx& ctx,

@@ -200,6 +200,23 @@ def test_paged_decode_large_groups(heads):
     _check_paged(x, o, lse, 1 / np.sqrt(128))
 
 
+@pytest.mark.parametrize("page", [16, 64, 128, 192, 256])
+@pytest.mark.parametrize("heads", [(16, 4), (32, 4), (32, 2)], ids=["g4", "g8", "g16"])
+def test_paged_decode_keys_as_rows(heads, page):
+    """Groups of 4 and 8 query heads per KV head at d = 128 run with the keys
+    as the tensor cores' M rows (128-key tiles; 192-row pages, whose tiles
+    would straddle two pages, take the heads-as-rows kernel, as do groups of
+    16); lengths leave partial last tiles over NaN-filled page rows, one
+    sequence is empty, and one chunk count splits the cache into many short
+    chunks."""
+    hq, hkv = heads
+    x = inputgen.make_paged_decode_inputs(640 + hq + page, 4, hq, hkv, 128, page,
+                                          seqlens=[0, 129, 1000, 5000])
+    for splits in (0, 9):
+        o, lse = run_paged(x, splits)
+        _check_paged(x, o, lse, 1 / np.sqrt(128))
+
+
 def test_paged_decode_tensor_core_bad_page_is_reported_not_read():
     """As the bad-page test above, on the tensor-core path (4 query heads per
     KV head): no page outside the pool is read, the status says so."""

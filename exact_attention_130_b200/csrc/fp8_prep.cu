@@ -27,7 +27,7 @@
 // so a row's butterflies of stride >= 4 are warp shuffles. The transposed V
 // ([B, H, d, n_vt] codes, n_vt = N rounded up to 16, zero codes past N) goes
 // through a shared-memory tile so that both the loads and the stores are
-// coalesced.
+// coalesced (see fp8_prep_vt_kernel for the lane mapping).
 #include <cstdint>
 
 #include "fa_internal.h"
@@ -41,15 +41,6 @@ constexpr int kPrepRows = 128;  // rows per quantisation block
 constexpr int kPrepThreads = 256;
 constexpr int kRowsPerWarp = kPrepRows / (kPrepThreads / 32);
 constexpr float kE4m3Max = 448.0f;
-
-// columns 4 lane .. 4 lane + 3 of one bf16 row, as fp32 (exact)
-__device__ __forceinline__ void load_row4(const uint16_t* src, float (&x)[4]) {
-  const uint2 u = *reinterpret_cast<const uint2*>(src);
-  x[0] = __uint_as_float(u.x << 16);
-  x[1] = __uint_as_float(u.x & 0xffff0000u);
-  x[2] = __uint_as_float(u.y << 16);
-  x[3] = __uint_as_float(u.y & 0xffff0000u);
-}
 
 // (x * sign(sigma)) H_128 of one row held by a warp (4 columns per lane).
 // Every lane of the warp must call it (shuffles).
@@ -110,18 +101,29 @@ __global__ void __launch_bounds__(kPrepThreads)
 #pragma unroll
     for (int e = 0; e < 4; ++e) neg[e] = signbit(signs[lane * 4 + e]);
   }
+  // all of the warp's row loads first (16 in flight per thread), then the
+  // rotations: loading and rotating row by row left the kernel waiting on
+  // one load at a time
+  uint2 raw[kRowsPerWarp];
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    const int row = blk * kPrepRows + warp * kRowsPerWarp + i;  // the same for the whole warp
+    raw[i] = make_uint2(0u, 0u);
+    if (row < N)
+      raw[i] = *reinterpret_cast<const uint2*>(src + (head_row0 + row) * kPrepD + lane * 4);
+  }
   float x[kRowsPerWarp][4];
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < kRowsPerWarp; ++i) {
-    const int row = blk * kPrepRows + warp * kRowsPerWarp + i;  // the same for the whole warp
-    x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
-    if (row < N) {
-      load_row4(src + (head_row0 + row) * kPrepD + lane * 4, x[i]);
-      if (rot) rotate_row(x[i], neg, lane);
+    x[i][0] = __uint_as_float(raw[i].x << 16);
+    x[i][1] = __uint_as_float(raw[i].x & 0xffff0000u);
+    x[i][2] = __uint_as_float(raw[i].y << 16);
+    x[i][3] = __uint_as_float(raw[i].y & 0xffff0000u);
+    // (rows past N are zero and stay zero under the rotation)
+    if (rot) rotate_row(x[i], neg, lane);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(x[i][e]));
-    }
+    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(x[i][e]));
   }
   amax = block_max(amax, red);
   if (which == 2) {
@@ -143,33 +145,53 @@ __global__ void __launch_bounds__(kPrepThreads)
 }
 
 // blockIdx = (128-key block, head): V codes with the head's scale, written
-// transposed ([d, n_vt] per head).
+// transposed ([d, n_vt] per head). Lane l of a warp takes the dims l, l + 32,
+// l + 64, l + 96 of four consecutive keys (each load of the warp reads 64
+// contiguous bytes of one key row), packs the four keys' codes of a dim into
+// one word and stores it into a shared-memory tile of dim rows whose pitch is
+// an odd number of words, so the 32 lanes' stores hit 32 different banks;
+// the tile then leaves in 16-byte global stores along the keys.
 __global__ void __launch_bounds__(kPrepThreads)
     fp8_prep_vt_kernel(const uint16_t* __restrict__ v, int N, int n_vt,
                        const float* __restrict__ v_amax, uint8_t* __restrict__ vt8) {
-  constexpr int kPitch = kPrepRows + 16;  // bytes per transposed row (16-byte aligned)
-  __shared__ __align__(16) uint8_t t[kPrepD * kPitch];
+  constexpr int kPitchW = kPrepRows / 4 + 1;  // words per transposed row (odd)
+  __shared__ uint32_t t[kPrepD * kPitchW];
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float va = v_amax[bh];
   const float s = va > 0.f ? __fdiv_rn(va, kE4m3Max) : 1.0f;
-#pragma unroll 4
-  for (int i = 0; i < kRowsPerWarp; ++i) {
-    const int key = warp * kRowsPerWarp + i;
-    const int row = blk * kPrepRows + key;
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
-    if (row < N) load_row4(v + (size_t(bh) * N + row) * kPrepD + lane * 4, x);
-    const uint32_t c = codes4(x, s);
+  constexpr int kWarps = kPrepThreads / 32;
+#pragma unroll 1
+  for (int k4 = warp; k4 < kPrepRows / 4; k4 += kWarps) {  // a group of four keys
+    uint16_t raw[4][4];  // [key][dim group]
 #pragma unroll
-    for (int e = 0; e < 4; ++e) t[(lane * 4 + e) * kPitch + key] = uint8_t(c >> (8 * e));
+    for (int kk = 0; kk < 4; ++kk) {
+      const int row = blk * kPrepRows + k4 * 4 + kk;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        raw[kk][e] = row < N ? v[(size_t(bh) * N + row) * kPrepD + e * 32 + lane] : uint16_t(0);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int kk = 0; kk < 4; kk += 2) {
+        const float a = __uint_as_float(uint32_t(raw[kk][e]) << 16);
+        const float b = __uint_as_float(uint32_t(raw[kk + 1][e]) << 16);
+        w |= pack_e4m3x2(__fdiv_rn(a, s), __fdiv_rn(b, s)) << (8 * kk);
+      }
+      t[(e * 32 + lane) * kPitchW + k4] = w;
+    }
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < kPrepD * (kPrepRows / 16); idx += kPrepThreads) {
     const int dcol = idx / (kPrepRows / 16), chunk = idx % (kPrepRows / 16);
     const int key0 = blk * kPrepRows + chunk * 16;
-    if (key0 < n_vt)
+    if (key0 < n_vt) {
+      const uint32_t* src = t + dcol * kPitchW + chunk * 4;
       *reinterpret_cast<uint4*>(vt8 + (size_t(bh) * kPrepD + dcol) * n_vt + key0) =
-          *reinterpret_cast<const uint4*>(t + dcol * kPitch + chunk * 16);
+          make_uint4(src[0], src[1], src[2], src[3]);
+    }
   }
 }
 

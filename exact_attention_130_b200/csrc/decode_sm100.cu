@@ -499,7 +499,7 @@ fa_status launch_decode(const void* q, const void* kcache, const void* vcache, c
 fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpages,
                               const int* block_table, const int* seqlens, void* o, float* lse,
                               int B, int Hq, int Hkv, int num_pages, int page_size, int max_pages,
-                              int d, float scale, int chunks, void* workspace,
+                              int d, float scale, int chunks, bool auto_split, void* workspace,
                               const LaunchCtx& ctx) {
   if (Hq > 65535 || B > 65535) {
     set_last_error("fa_decode_paged: B and Hq must each be <= 65535");
@@ -533,14 +533,20 @@ fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpa
     // tensor cores (decode_tct_sm100.cu); larger groups or d = 64: the query
     // heads as the M rows (decode_tc_sm100.cu); then the same merge
     // (its 128-key tiles must split into runs inside one page: pages of at
-    // most 64 rows, or of a multiple of 128)
+    // most 64 rows, or of a multiple of 128). With the automatic split the
+    // keys-as-rows kernel balances whole tiles over persistent CTAs and
+    // merges its own partials.
     const bool keys_as_rows = d == 128 && p.group <= kTctMaxGroup &&
                               (page_size <= 64 || page_size % 128 == 0);
+    if (keys_as_rows && auto_split)
+      return launch_decode_paged_tct(q, kpages, vpages, block_table, seqlens, B, Hq, Hkv,
+                                     num_pages, page_size, max_pages, d, scale, 0, nullptr,
+                                     nullptr, workspace, o, lse, ctx);
     fa_status st =
         keys_as_rows
             ? launch_decode_paged_tct(q, kpages, vpages, block_table, seqlens, B, Hq, Hkv,
                                       num_pages, page_size, max_pages, d, scale, chunks, p.part_o,
-                                      p.part_lse, ctx)
+                                      p.part_lse, nullptr, nullptr, nullptr, ctx)
             : launch_decode_paged_tc(q, kpages, vpages, block_table, seqlens, B, Hq, Hkv,
                                      num_pages, page_size, max_pages, d, scale, chunks, p.part_o,
                                      p.part_lse, ctx);

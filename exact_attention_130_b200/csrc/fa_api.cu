@@ -433,7 +433,13 @@ size_t fa_decode_workspace_size(int B, int H, int Lmax, int d, int num_splits) {
   // for which the size is taken at its maximum so a buffer sized here fits
   // any device of this family)
   const int chunks = decode_num_chunks(B, H, Lmax, num_splits, 0);
-  return decode_workspace_bytes(B, H, d, chunks);
+  const size_t by_chunks = decode_workspace_bytes(B, H, d, chunks);
+  if (num_splits > 0) return by_chunks;
+  // the automatic split of the paged decode may balance tiles over
+  // persistent CTAs instead (4 to 8 query heads per KV head), whose partials
+  // need at most this much
+  const size_t balanced = decode_balanced_workspace_bytes(B, H, d);
+  return by_chunks > balanced ? by_chunks : balanced;
 }
 
 fa_status fa_decode_splitkv(const void* q, const void* kcache, const void* vcache,
@@ -496,7 +502,7 @@ fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
     return invalid(FA_ERR_INVALID_ARG, "num_splits must be in [0, 1024] (got %d)", num_splits);
   const int Lmax = max_pages * page_size;
   const int chunks = decode_num_chunks(B, Hq, Lmax, num_splits, 0);
-  const size_t need = decode_workspace_bytes(B, Hq, d, chunks);
+  const size_t need = fa_decode_workspace_size(B, Hq, Lmax, d, num_splits);
   if (workspace == nullptr || workspace_bytes < need)
     return invalid(FA_ERR_WORKSPACE, "fa_decode_paged needs %zu bytes of workspace (got %zu)",
                    need, workspace ? workspace_bytes : size_t(0));
@@ -505,7 +511,8 @@ fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
   if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
   ctx.debug_skip_load = g_debug_skip.exchange(0);
   return launch_decode_paged(q, kpages, vpages, block_table, seqlens, o, lse, B, Hq, Hkv,
-                             num_pages, page_size, max_pages, d, scale, chunks, workspace, ctx);
+                             num_pages, page_size, max_pages, d, scale, chunks, num_splits == 0,
+                             workspace, ctx);
 }
 
 void fa_profile_begin(void) {

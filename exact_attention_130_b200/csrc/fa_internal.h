@@ -101,7 +101,7 @@ size_t decode_workspace_bytes(int B, int H, int d, int chunks);
 fa_status launch_decode_paged(const void* q, const void* kpages, const void* vpages,
                               const int* block_table, const int* seqlens, void* o, float* lse,
                               int B, int Hq, int Hkv, int num_pages, int page_size, int max_pages,
-                              int d, float scale, int chunks, void* workspace,
+                              int d, float scale, int chunks, bool auto_split, void* workspace,
                               const LaunchCtx& ctx);
 fa_status launch_decode_paged_tc(const void* q, const void* kpages, const void* vpages,
                                  const int* block_table, const int* seqlens, int B, int Hq,
@@ -112,7 +112,10 @@ fa_status launch_decode_paged_tct(const void* q, const void* kpages, const void*
                                   const int* block_table, const int* seqlens, int B, int Hq,
                                   int Hkv, int num_pages, int page_size, int max_pages, int d,
                                   float scale, int chunks, float* part_o, float* part_lse,
-                                  const LaunchCtx& ctx);
+                                  void* workspace, void* o, float* lse, const LaunchCtx& ctx);
+// Bytes of workspace the balanced schedule of the keys-as-rows paged decode
+// needs (decode_tct_sm100.cu), for B sequences of H query heads.
+size_t decode_balanced_workspace_bytes(int B, int H, int d);
 fa_status launch_decode(const void* q, const void* kcache, const void* vcache,
                         const int* seqlens, void* o, float* lse, int B, int H, int Lmax, int d,
                         float scale, int chunks, void* workspace, const LaunchCtx& ctx,

@@ -243,10 +243,13 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
                  cudaStream_t stream);
 
 /*
- * fa_decode_workspace_size -- bytes of scratch fa_decode_splitkv needs for
- * per-chunk partial results: fp32 [B, H, C, d] outputs and fp32 [B, H, C]
- * log-sum-exps, C = the chunk count the call will use (num_splits, or the
- * automatic choice when num_splits == 0).
+ * fa_decode_workspace_size -- bytes of scratch fa_decode_splitkv and
+ * fa_decode_paged need for per-chunk partial results: fp32 [B, H, C, d]
+ * outputs and fp32 [B, H, C] log-sum-exps, C = the chunk count the call will
+ * use (num_splits, or the automatic choice when num_splits == 0). With
+ * num_splits == 0 the size also covers the paged decode's balanced split
+ * (fa_decode_paged below): at most B H + 2368 partials of d + 1 floats and
+ * 8 bytes per (sequence, KV head), whichever is larger.
  */
 size_t fa_decode_workspace_size(int B, int H, int Lmax, int d, int num_splits);
 
@@ -298,7 +301,13 @@ fa_status fa_decode_splitkv(const void* q, const void* kcache,
  *                    are the rows of the MMA), the others on the CUDA cores
  *                    (up to four heads of a group per CTA)
  *   page_size      : 16, 32 or a multiple of 64
- *   num_splits     : chunks per sequence, 0 = automatic, <= 1024
+ *   num_splits     : chunks per sequence, 0 = automatic, <= 1024. With 0,
+ *                    groups of 4 to 8 query heads at d = 128 (and pages of
+ *                    <= 64 rows or a multiple of 128) split the cache by
+ *                    whole 128-key tiles instead: all tiles of all
+ *                    (sequence, KV head) pairs are dealt out in equal
+ *                    contiguous ranges to persistent CTAs (two per SM),
+ *                    whatever the mix of lengths
  *   workspace      : >= fa_decode_workspace_size(B, Hq, max_pages *
  *                    page_size, d, num_splits) bytes (caller-owned, device)
  * Validation errors return before any launch. A block-table entry outside

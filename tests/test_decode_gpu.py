@@ -217,6 +217,24 @@ def test_paged_decode_keys_as_rows(heads, page):
         _check_paged(x, o, lse, 1 / np.sqrt(128))
 
 
+@pytest.mark.parametrize("page", [64, 128])
+@pytest.mark.parametrize("heads", [(16, 4), (12, 2), (16, 2)], ids=["g4", "g6", "g8"])
+def test_paged_decode_balanced_split(heads, page):
+    """The automatic split of groups of 4 to 8 query heads (d = 128) deals
+    whole 128-key tiles out to persistent CTAs in equal ranges. 45 sequences
+    (more than one warp's worth, for the CTAs' scan of the lengths), empty
+    and one-key ones, lengths on and just off a tile boundary, the rest
+    random: pieces start and end inside sequences, a sequence spans several
+    CTAs, a CTA several sequences, and rows past each length are NaN."""
+    hq, hkv = heads
+    rng = np.random.default_rng(660 + hq + page)
+    lens = rng.integers(0, 3000, size=45).astype(np.int32)
+    lens[:6] = [0, 1, 127, 128, 129, 0]
+    x = inputgen.make_paged_decode_inputs(660 + hq + page, 45, hq, hkv, 128, page, seqlens=lens)
+    o, lse = run_paged(x)
+    _check_paged(x, o, lse, 1 / np.sqrt(128))
+
+
 def test_paged_decode_tensor_core_bad_page_is_reported_not_read():
     """As the bad-page test above, on the tensor-core path (4 query heads per
     KV head): no page outside the pool is read, the status says so."""

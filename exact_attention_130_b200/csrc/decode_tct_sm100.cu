@@ -151,6 +151,13 @@ __device__ __forceinline__ bool wait_nb(uint32_t bar, uint32_t parity, const Wai
                         (w.kernel_id << 16) | ((site & 0xffu) << 8) | 1u, drain);
 }
 
+// The maximum of v over the warp (one instruction on sm_100a).
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 // TMEM loads and stores of N 32-bit columns per lane (N = 4, 8 or 16), then
 // the wait for the loads / stores.
 template <int N>
@@ -610,16 +617,14 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
       for (int h = 0; h < GH; ++h)
         x[h] = (t < valid && on(h)) ? __uint_as_float(sr[h]) * cl : -INFINITY;
-      // the tile's maximum of every head over the 128 keys
+      // the tile's maximum of every head over the 128 keys (heads past G
+      // carry -inf throughout: no branch per head, so the GH reductions
+      // overlap)
       float* rd = red + (g & 1) * kSmWarps * kNH;
 #pragma unroll
       for (int h = 0; h < GH; ++h) {
-        if (on(h)) {
-          float v = x[h];
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-          if (lane == 0) rd[warp * kNH + h] = v;
-        }
+        const float v = warp_max(x[h]);
+        if (lane == 0) rd[warp * kNH + h] = v;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(X_MAX + (g & 1)));
@@ -633,11 +638,8 @@ __global__ void __launch_bounds__(kThreads)
       float mt[GH];
 #pragma unroll
       for (int h = 0; h < GH; ++h) {
-        mt[h] = -INFINITY;
-        if (on(h)) {
-          mt[h] = fmaxf(fmaxf(rd[h], rd[kNH + h]), fmaxf(rd[2 * kNH + h], rd[3 * kNH + h]));
-          grow |= mt[h] > m[h] + kRescale;
-        }
+        mt[h] = fmaxf(fmaxf(rd[h], rd[kNH + h]), fmaxf(rd[2 * kNH + h], rd[3 * kNH + h]));
+        grow |= mt[h] > m[h] + kRescale;  // (false for a masked head: -inf > -inf)
       }
       if (it.first()) {
 #pragma unroll
@@ -674,14 +676,13 @@ __global__ void __launch_bounds__(kThreads)
       const int kb = (t & 63) * 2;  // byte of this key in its 128-byte row
 #pragma unroll
       for (int h = 0; h < GH; ++h) {
-        if (on(h)) {
-          // (a head whose keys so far are all masked has m = -inf: its P is 0)
-          const float pv = m[h] == -INFINITY ? 0.f : ex2_approx(x[h] - m[h]);
-          lp[h] += pv;
-          const uint32_t bits = pack_bf16x2(pv, 0.f) & 0xffffu;
-          *reinterpret_cast<uint16_t*>(pt + h * 128 + ((((kb >> 4) ^ (h & 7))) << 4) + (kb & 15)) =
-              uint16_t(bits);
-        }
+        // (a head whose keys so far are all masked, a head past G among
+        // them, has m = -inf: its P is 0)
+        const float pv = m[h] == -INFINITY ? 0.f : ex2_approx(x[h] - m[h]);
+        lp[h] += pv;
+        const uint32_t bits = pack_bf16x2(pv, 0.f) & 0xffffu;
+        *reinterpret_cast<uint16_t*>(pt + h * 128 + ((((kb >> 4) ^ (h & 7))) << 4) + (kb & 15)) =
+            uint16_t(bits);
       }
       if (valid < kKeys && warp == 0) {
         // the sequence's last tile: zero the V rows past its length before

@@ -685,14 +685,30 @@ def measure_next_rows(fa, torch, dev, flush, peaks, iters=8):
     ws = torch.empty(fa.fa_decode_workspace_size(Bq, Hq, cap, d, 0), dtype=torch.uint8, device="cuda")
     od = torch.empty_like(qd)
     lsed = torch.empty((Bq, Hq), dtype=torch.float32, device="cuda")
-    ms = med_ms(lambda: fa.fa_decode_paged(qd, kp, vp, table, lens, o=od, lse=lsed, workspace=ws))
+    call = lambda: fa.fa_decode_paged(qd, kp, vp, table, lens, o=od, lse=lsed, workspace=ws)  # noqa: E731
+    ms = med_ms(call)
     kv_bytes = int(lens.sum().item()) * Hkv * d * 2 * 2
     gbs = kv_bytes / (ms * 1e-3) / 1e9
+    # the split kernel alone: the library's CUDA events around its launch,
+    # over `iters` calls, each after an L2 flush
+    fa.fa_profile_begin()
+    for _ in range(iters):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    prof = fa.fa_profile_end()
+    n_split, t_split = prof.get("decode_split", (0, 0.0))
+    n_merge, t_merge = prof.get("decode_merge", (0, 0.0))
+    split_us = t_split / max(n_split, 1) * 1e3
     rows["decode_paged"] = {
         "workload": f"B={Bq} Hq={Hq} Hkv={Hkv} d={d}, {page}-row pages shuffled, lengths uniform "
-                    f"[{cap // 2}, {cap}] (tensor-core kernel: 4 query heads per KV head)",
+                    f"[{cap // 2}, {cap}] (tensor-core kernel, keys as rows: 4 query heads per "
+                    f"KV head; balanced tile split)",
         "us": round(ms * 1e3, 1), "gbs_unique_kv": round(gbs, 1), "peak": peaks["hbm_gbs"],
-        "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4)}
+        "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+        "split_kernel_us": round(split_us, 1),
+        "split_kernel_gbs": round(kv_bytes / (split_us * 1e-6) / 1e9, 1) if split_us > 0 else None,
+        "merge_kernel_us": round(t_merge / max(n_merge, 1) * 1e3, 1)}
     del kp, vp
     return rows
 

@@ -6,7 +6,7 @@ memory and the current stream. There is no CPU fallback: if the library is
 missing, every call raises.
 
 Functions carry the C names:
-    fa_fwd, fa_fwd_ex, fa_fwd_f32, fa_fp8_prepare, fa_fwd_fp8, fa_fp8_vt_keys,
+    fa_fwd, fa_fwd_ex, fa_fwd_f32, fa_fwd_tf32, fa_fp8_prepare, fa_fwd_fp8, fa_fp8_vt_keys,
     fa_bwd_ex,
     fa_bwd, fa_bwd_workspace_size,
     fa_decode_splitkv, fa_decode_workspace_size,
@@ -21,7 +21,7 @@ import re
 
 __all__ = [
     "FAError", "library_path", "load_library", "exported_symbols",
-    "fa_fwd", "fa_fwd_pair", "fa_fwd_ex", "fa_bwd_ex", "fa_dropout_keep_threshold", "fa_fwd_f32", "fa_fp8_prepare", "fa_fwd_fp8",
+    "fa_fwd", "fa_fwd_pair", "fa_fwd_ex", "fa_bwd_ex", "fa_dropout_keep_threshold", "fa_fwd_f32", "fa_fwd_tf32", "fa_fp8_prepare", "fa_fwd_fp8",
     "fa_fp8_vt_keys",
     "fa_bwd", "fa_bwd_workspace_size",
     "fa_decode_splitkv", "fa_decode_workspace_size", "fa_decode_splitkv_static",
@@ -62,6 +62,7 @@ _SIGNATURES = {
     "fa_abi_version": (_I, []),
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_tf32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_pair": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, ctypes.c_longlong,
                        ctypes.c_longlong, _F, ctypes.c_ulonglong, ctypes.c_uint, _P]),
@@ -278,6 +279,27 @@ def fa_fwd_f32(q, k, v, causal: bool = False, scale: float | None = None,
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     _check(lib.fa_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N,
+                          d, scale, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_fwd_tf32(q, k, v, causal: bool = False, scale: float | None = None,
+               o=None, lse=None, stream=None):
+    """fa_fwd_f32 with both products on the tensor cores in TF32 (inputs
+    rounded to TF32 to nearest): faster, errors ~1e-4 to 1e-3."""
+    import torch
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.float32, n)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check(lib.fa_fwd_tf32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N,
                           d, scale, int(bool(causal)), _stream(stream)))
     return o, lse
 

@@ -328,6 +328,18 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, f
   return launch_fwd_f32(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx);
 }
 
+fa_status fa_fwd_tf32(const float* q, const float* k, const float* v, float* o, float* lse, int B,
+                      int H, int N, int d, float scale, int causal, cudaStream_t stream) {
+  fa_status st;
+  if ((st = check_ptrs({q, k, v, o, lse}, "fa_fwd_tf32(q,k,v,o,lse)")) != FA_OK) return st;
+  if ((st = check_bhnd(B, H, N, d)) != FA_OK) return st;
+  if ((st = check_scale(scale)) != FA_OK) return st;
+  if (causal != 0 && causal != 1) return invalid(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  LaunchCtx ctx;
+  if ((st = device_ctx(stream, &ctx)) != FA_OK) return st;
+  return launch_fwd_tf32(q, k, v, o, lse, B, H, N, d, scale, causal != 0, ctx);
+}
+
 int fa_fp8_vt_keys(int N) { return N >= 1 && N <= 0x7ffffff0 ? fp8_vt_keys(N) : 0; }
 
 fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const float* signs, int B,

@@ -91,6 +91,9 @@ fa_status launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const 
 fa_status launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                          int B, int H, int N, int d, float scale, bool causal,
                          const LaunchCtx& ctx);
+fa_status launch_fwd_tf32(const float* q, const float* k, const float* v, float* o, float* lse,
+                         int B, int H, int N, int d, float scale, bool causal,
+                         const LaunchCtx& ctx);
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
                      int H, int N, int d, float scale, bool causal, void* workspace,

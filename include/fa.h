@@ -116,6 +116,22 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o,
                      int causal, cudaStream_t stream);
 
 /*
+ * fa_fwd_tf32 -- the forward of fa_fwd_f32 (fp32 tensors in and out, same
+ * arguments and errors) with both products on the tensor cores in TF32
+ * (tcgen05 .kind::tf32: a 10-bit mantissa, fp32 accumulation). Q, K, V and
+ * P are rounded to TF32 to nearest before the products (the tensor cores
+ * would otherwise truncate, which biases every product toward zero). The
+ * price is precision: errors of ~1e-4 to 1e-3 in O and LSE on N(0,1)
+ * inputs, inside the 1e-2 / 1e-3 bars of the bf16 forward but far from
+ * fa_fwd_f32's ~1e-6; the gain is speed (one 128-row tile per CTA, 64-key
+ * tiles, no pipelining: about 15% on a 128-row head, 2x at N = 1000).
+ * Passages as for fa_fwd.
+ */
+fa_status fa_fwd_tf32(const float* q, const float* k, const float* v, float* o,
+                      float* lse, int B, int H, int N, int d, float scale,
+                      int causal, cudaStream_t stream);
+
+/*
  * fa_fwd_ex / fa_bwd_ex -- fa_fwd / fa_bwd with the two options of the
  * attention definition and of dropout ("FlashAttention'i Anlamak Bolum 1",
  * 0.2: S = Q K^T / sqrt(d) + B, B an optional mask or bias; "Bellek

@@ -9,7 +9,7 @@ import exact_attention_130_b200 as fa
 
 EXPECTED = {
     "fa_status_string", "fa_last_error", "fa_abi_version", "fa_fwd",
-    "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd",
+    "fa_fwd_f32", "fa_fwd_tf32", "fa_bwd_workspace_size", "fa_bwd",
     "fa_decode_workspace_size", "fa_decode_splitkv", "fa_device_status",
     "fa_set_wait_limit", "fa_debug_skip_load", "fa_profile_begin",
     "fa_profile_end", "fa_decode_splitkv_static", "fa_decode_paged",

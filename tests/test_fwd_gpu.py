@@ -158,6 +158,45 @@ def test_fwd_f32_other_shapes(N, d):
         assert max_abs(o, ref_o) <= 1e-4 and max_abs(lse, ref_l) <= 1e-4
 
 
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_fwd_tiny_tf32_workload(causal):
+    """The fp32 workload (B=1, H=1, N=128, d=64) through fa_fwd_tf32, the
+    TF32 tensor-core variant: within the bf16 forward's bars (O 1e-2, LSE
+    1e-3), and, its inputs being rounded to nearest, within 2e-3 / 1e-3
+    where truncation would bias the LSE by ~1e-3."""
+    w = inputgen.WORKLOADS["tiny_f32"]
+    x = inputgen.make_attention_inputs(w)
+    q, k, v = (f32_device(x[n]) for n in ("q", "k", "v"))
+    o = Guarded((w.B, w.H, w.N, w.d), torch.float32)
+    lse = Guarded((w.B, w.H, w.N), torch.float32)
+    fa.fa_fwd_tf32(q, k, v, causal=causal, o=o.t, lse=lse.t)
+    torch.cuda.synchronize()
+    assert o.guards_intact() and lse.guards_intact()
+    ref_o, ref_l = oracle.attention_fwd(x["q"].astype(np.float64), x["k"].astype(np.float64),
+                                        x["v"].astype(np.float64), w.scale, causal)
+    assert max_abs(o.t, ref_o) <= 2e-3
+    assert max_abs(lse.t, ref_l) <= TOL_LSE
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 63, 100, 333, 1000])
+def test_fwd_tf32_other_shapes(N, d):
+    """Ragged lengths over one and several 64-key and 128-row tiles, both
+    head dims, both masks: O within 1e-2 and LSE within 1e-3 of the oracle,
+    and the two masks agree on the last row (which sees every key)."""
+    rng = np.random.default_rng(N * d + 5)
+    x = {n: rng.standard_normal((2, 2, N, d), dtype=np.float32) for n in "qkv"}
+    outs = {}
+    for causal in (False, True):
+        o, lse = fa.fa_fwd_tf32(*(f32_device(x[n]) for n in "qkv"), causal=causal)
+        torch.cuda.synchronize()
+        ref_o, ref_l = oracle.attention_fwd(*(x[n].astype(np.float64) for n in "qkv"),
+                                            1 / math.sqrt(d), causal)
+        assert max_abs(o, ref_o) <= TOL_O and max_abs(lse, ref_l) <= TOL_LSE
+        outs[causal] = (o, lse)
+    assert torch.equal(outs[False][0][:, :, -1], outs[True][0][:, :, -1])
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_fwd_growing_scores_rescale_path(d):
     """Keys grow along the sequence so the running maximum keeps rising by

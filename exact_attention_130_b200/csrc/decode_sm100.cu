@@ -123,6 +123,9 @@ template <int D, bool PAGED, int GH>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_split_kernel(const DecParams p) {
   using L = DecLayout<D>;
+  // the merge kernel, launched as a programmatic dependent, may be scheduled
+  // now: it waits for this grid's completion before reading anything
+  grid_dependents_launch();
   constexpr int kPer = D / 16;  // elements per lane (16 lanes per row)
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -379,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // combined in index order.
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecParams p) {
+  grid_dependency_wait();  // the split kernel's partials
   const int h = blockIdx.x, b = blockIdx.y;
   const size_t bh = size_t(b) * p.H + h;
   const float* pl = p.part_lse + bh * p.C;
@@ -411,7 +415,8 @@ fa_status launch_merge(const DecParams& p, int B, const LaunchCtx& ctx) {
   dim3 g2(p.H, B);
   {
     ProfileScope prof(KID_DECODE_MERGE, ctx.stream);
-    decode_merge_kernel<D><<<g2, D, 0, ctx.stream>>>(p);
+    cudaError_t e = launch_dependent(decode_merge_kernel<D>, g2, dim3(D), 0, ctx.stream, p);
+    if (e != cudaSuccess) return cuda_fail(e, "decode merge kernel launch");
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode merge kernel launch");
@@ -434,7 +439,8 @@ fa_status launch(const DecParams& p, int B, const LaunchCtx& ctx) {
   dim3 g2(p.H, B);
   {
     ProfileScope prof(KID_DECODE_MERGE, ctx.stream);
-    decode_merge_kernel<D><<<g2, D, 0, ctx.stream>>>(p);
+    e = launch_dependent(decode_merge_kernel<D>, g2, dim3(D), 0, ctx.stream, p);
+    if (e != cudaSuccess) return cuda_fail(e, "decode merge kernel launch");
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode merge kernel launch");

@@ -98,6 +98,9 @@ __global__ void __launch_bounds__(kTcThreads)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const TcParams p) {
   using L = TcLayout<D>;
+  // the merge kernel, launched as a programmatic dependent, may be scheduled
+  // now: it waits for this grid's completion before reading anything
+  grid_dependents_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

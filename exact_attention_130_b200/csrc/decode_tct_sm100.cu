@@ -339,6 +339,9 @@ __global__ void __launch_bounds__(kThreads)
     decode_tct_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const TctParams p) {
   using L = Layout;
+  // the merge kernel, launched as a programmatic dependent, may be scheduled
+  // now: it waits for this grid's completion before reading anything
+  grid_dependents_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -760,6 +763,7 @@ __global__ void __launch_bounds__(kThreads)
 // not write, after a failed launch) is reported, never read.
 __global__ void __launch_bounds__(kD) decode_merge_slots_kernel(const TctParams p, int slots,
                                                                 uint16_t* o, float* lse) {
+  grid_dependency_wait();  // the split kernel's partials and records
   const int h = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
   const size_t bh = size_t(b) * p.Hq + h;
   const int hk = h / p.group, g = h % p.group;
@@ -890,8 +894,9 @@ fa_status launch_decode_paged_tct(const void* q, const void* kpages, const void*
   if (e != cudaSuccess) return cuda_fail(e, "decode tct kernel launch");
   {
     ProfileScope prof(KID_DECODE_MERGE, ctx.stream);
-    decode_merge_slots_kernel<<<dim3(Hq, B), kD, 0, ctx.stream>>>(
-        p, slots, static_cast<uint16_t*>(o), lse);
+    e = launch_dependent(decode_merge_slots_kernel, dim3(Hq, B), dim3(kD), 0, ctx.stream, p, slots,
+                         static_cast<uint16_t*>(o), lse);
+    if (e != cudaSuccess) return cuda_fail(e, "decode merge kernel launch");
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode merge kernel launch");

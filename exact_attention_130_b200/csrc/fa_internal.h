@@ -6,6 +6,8 @@
 
 #include <cstdint>
 
+#include <utility>
+
 #include "fa.h"
 
 namespace fa {
@@ -18,6 +20,25 @@ struct LaunchCtx {
   int num_sms;
   int debug_skip_load;            // test hook, see fa_debug_skip_load()
 };
+
+// Launch `kernel` on the stream as a programmatic dependent of the kernel
+// before it: its launch overlaps that kernel's end, and the kernel itself
+// waits (grid_dependency_wait) before reading what the first one wrote.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Kernel ids recorded in the status word.
 enum KernelId : unsigned int {

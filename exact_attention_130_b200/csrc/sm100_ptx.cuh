@@ -69,6 +69,18 @@ __device__ __forceinline__ uint32_t mbar_test_wait(uint32_t bar, uint32_t parity
   return ok;
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute waits here until the grid before it on the
+// stream has completed and its memory is visible (a no-op for a kernel
+// launched without the attribute); that grid's CTAs may let it be scheduled
+// earlier by triggering.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Shared state every bounded wait of a CTA consults.
 struct WaitCtl {
   volatile int* abort_flag;       // shared memory; nonzero once any wait gave up

@@ -235,6 +235,21 @@ def test_paged_decode_balanced_split(heads, page):
     _check_paged(x, o, lse, 1 / np.sqrt(128))
 
 
+@pytest.mark.parametrize("heads", [(8, 2), (16, 2)], ids=["g4", "g8"])
+def test_paged_decode_balanced_many_short_pieces(heads):
+    """600 short sequences (0 to 300 keys: one to three tiles each), so that
+    a persistent CTA's range covers several whole segments: its pipeline
+    runs across three or more pieces, reusing both O accumulators and the Q
+    buffer, while other segments still span two CTAs."""
+    hq, hkv = heads
+    rng = np.random.default_rng(680 + hq)
+    lens = rng.integers(0, 301, size=600).astype(np.int32)
+    lens[:4] = [0, 1, 128, 129]
+    x = inputgen.make_paged_decode_inputs(680 + hq, 600, hq, hkv, 128, 64, seqlens=lens)
+    o, lse = run_paged(x)
+    _check_paged(x, o, lse, 1 / np.sqrt(128))
+
+
 def test_paged_decode_tensor_core_bad_page_is_reported_not_read():
     """As the bad-page test above, on the tensor-core path (4 query heads per
     KV head): no page outside the pool is read, the status says so."""

@@ -169,3 +169,13 @@ def test_workspace_sizes(lib):
     assert fa.fa_decode_workspace_size(8, 32, 32768, 128, 0) == ws  # auto = 16 here
     assert fa.fa_decode_workspace_size(1, 1, 100, 128, 0) > 0
     assert fa.fa_decode_workspace_size(1, 1, 100, 96, 0) == 0
+    # the automatic split also covers the paged decode's balanced schedule:
+    # B*H + 2368 partial rows of d + 1 floats and 8 bytes per (sequence, head),
+    # each region 256-aligned; larger than the chunked need for small shapes
+    a256 = lambda x: (x + 255) // 256 * 256
+    for B, H, L in ((1, 8, 2048), (3, 12, 700), (8, 32, 32768)):
+        rows = B * H + 2368
+        balanced = a256(rows * 128 * 4) + a256(rows * 4) + a256(B * H * 8)
+        auto = fa.fa_decode_workspace_size(B, H, L, 128, 0)
+        assert auto >= balanced and auto >= fa.fa_decode_workspace_size(B, H, L, 128, 1)
+    assert fa.fa_decode_workspace_size(1, 8, 2048, 128, 0) == a256((8 + 2368) * 512) + a256((8 + 2368) * 4) + a256(64)
